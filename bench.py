@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Benchmark: one MoE layer forward (hidden 1280, 64 routed experts, top-6, fused
+shared expert) on a B200, through libfocr_moe.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one forward of the layer over one batch of synthetic tokens (router,
+softmax/top-6, dispatch, routed + shared experts, combine).  The default workload
+is a single decode token through an int4 (group 64) layer with bf16 router and
+shared expert.  Steps rotate over 16 packed copies of the layer (~2.2 GB, far
+above the 126 MB L2) and over a pool of distinct input tokens, so the weights
+come from HBM.  Under torchrun every rank runs an independent replica (no data
+exchange: the path does not shard), and `value` sums all ranks' tokens over the
+slowest rank's time.  `--impl reference` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s and achieved HBM GB/s (% of B200 peak) vs CPU oracle"
+UNIT = "tokens/s"
+N_COPIES = 16
+DEFAULT_WORKLOAD = "t1_int4_g64"
+PEAK_FALLBACK_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def describe(name: str) -> dict:
+    from weight_quantized_expert_b200 import synth
+    w = synth.WORKLOADS[name]
+    tname = {0: "bf16", 1: "int8", 2: "int4"}
+    return {"workload": name, "tokens_per_step": w["T"], "routed": f"{tname[w['routed']]} g{w['group']}",
+            "shared": tname[w["shared"]] if w["shared"] == 0 else f"{tname[w['shared']]} g{w['group']}",
+            "router": "bf16", "seed": w["seed"], "hidden": 1280, "experts": "64 routed top-6 + shared 1792",
+            "l2": f"rotated over {N_COPIES} packed layer copies (> 2 GB, L2 is 126 MB) and distinct inputs"}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return PEAK_FALLBACK_GBS, "fallback"
+
+
+def sources_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "weight_quantized_expert_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """dram bytes per launch from the committed ncu summary, if it matches these sources."""
+    for f in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        txt = open(f).read()
+        m_w = re.search(r"^workload:\s*(\S+)", txt, re.M)
+        m_t = re.search(r"^traffic_bytes_per_step:\s*(\d+)", txt, re.M)
+        m_h = re.search(r"^sources_sha256:\s*(\S+)", txt, re.M)
+        if m_w and m_t and m_h and m_w.group(1) == workload and m_h.group(1) == sources_hash():
+            return int(m_t.group(1))
+    return None
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv") if os.path.isdir(
+            os.path.join(ROOT, "gpurun_out")) else f"/tmp/focr_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def oracle_rate(name: str, budget_s: float, max_tokens: int | None = None):
+    """tokens/s of the CPU oracle on a bounded sample of the workload (all host cores)."""
+    import oracle
+    from weight_quantized_expert_b200 import synth
+    w = synth.WORKLOADS[name]
+    _, layer = synth.workload(name)
+    om = oracle.OracleMoE(layer)
+    del layer
+    threads = oracle.max_threads()
+    pool = synth.hidden(w["seed"] + 1000, 4096, skew=w.get("skew", False))
+    # calibrate on one token per thread, then size the sample to the budget
+    t0 = time.perf_counter()
+    om.forward(pool[:threads], nthreads=threads)
+    dt = time.perf_counter() - t0
+    per_tok = dt / threads
+    n = max(threads, int(budget_s / max(per_tok, 1e-6)))
+    if max_tokens:
+        n = min(n, max_tokens)
+    n = min(n, pool.shape[0])
+    t0 = time.perf_counter()
+    om.forward(pool[:n], nthreads=threads)
+    dt = time.perf_counter() - t0
+    return n / dt, threads, n, dt, om, pool
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from weight_quantized_expert_b200 import synth
+    import oracle
+    w = synth.WORKLOADS[args.workload]
+    _, layer = synth.workload(args.workload)
+    om = oracle.OracleMoE(layer)
+    del layer
+    threads = oracle.max_threads()
+    T = w["T"]
+    pool = synth.hidden(w["seed"] + 1000, 4096, skew=w.get("skew", False))
+    # one step = the oracle forward of one batch of the workload's tokens (threads over tokens)
+    t0 = time.perf_counter()
+    om.forward(pool[:T], nthreads=threads)
+    per_step = time.perf_counter() - t0
+    budget = 150.0
+    steps = args.steps
+    warm = args.warmup
+    if (steps + warm) * per_step > budget:
+        warm = min(warm, 1)
+        steps = max(1, int(budget / per_step) - warm)
+    for i in range(warm):
+        om.forward(pool[(i * T) % 4000:(i * T) % 4000 + T], nthreads=threads)
+    t0 = time.perf_counter()
+    for i in range(steps):
+        s = (i * T) % 4000
+        om.forward(pool[s:s + T], nthreads=threads)
+    dt = time.perf_counter() - t0
+    value = steps * T / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": warm, "ms_per_step": dt / steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": describe(args.workload),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"{steps} steps x {T} token(s) of the workload through the CPU oracle "
+                                       f"(plain C, fp64, OpenMP over tokens)"
+                                       + ("" if steps == args.steps else
+                                          f"; steps capped from {args.steps} to bound the CPU run")},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from weight_quantized_expert_b200 import api, roofline, synth
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.WORKLOADS[args.workload]
+    T = w["T"]
+    x_np, layer = synth.workload(args.workload)
+    base = api.focr_moe_pack_weights(layer)
+    del layer
+    copies = [base] + [api.focr_moe_layer_clone(base) for _ in range(N_COPIES - 1)]
+    pool_n = 64
+    xs_np = synth.hidden(w["seed"] + 2000 + rank, pool_n * T, skew=w.get("skew", False)).reshape(pool_n, T, 1280)
+    xs = torch.from_numpy(xs_np).to(dev)
+    outs = torch.empty(pool_n, T, 1280, device=dev)
+    ws = api.new_workspace(T, dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i, st=None):
+        api.focr_moe_layer_forward(copies[i % N_COPIES], xs[i % pool_n], outs[i % pool_n], ws, stream=st)
+
+    # experts hit per step (for the algorithmic bytes): route each pool entry once
+    hits = []
+    counts = torch.empty(64, dtype=torch.int32, device=dev)
+    with torch.cuda.stream(stream):
+        for j in range(pool_n):
+            api.focr_moe_layer_forward(copies[0], xs[j], outs[j], ws, debug={"counts": counts}, stream=stream)
+            hits.append(int((counts > 0).sum().item()))
+    stream.synchronize()
+    step_bytes = [roofline.moe_layer_bytes(T, w["routed"], w["shared"], w["group"], h) for h in hits]
+
+    # warm-up (eager), then capture the K timed steps in CUDA graphs
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i, stream)
+    stream.synchronize()
+    G = 160
+    graphs = []
+    use_graph = True
+    try:
+        g_main = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_main, stream=stream):
+            for i in range(G):
+                step(i, torch.cuda.current_stream())
+        tail = args.steps % G
+        g_tail = None
+        if tail:
+            g_tail = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_tail, stream=stream):
+                for i in range(tail):
+                    step(i, torch.cuda.current_stream())
+        graphs = (g_main, g_tail)
+    except Exception as exc:  # pragma: no cover - reported in the JSON line
+        use_graph = False
+        graph_error = str(exc).splitlines()[0]
+    if use_graph:
+        with torch.cuda.stream(stream):
+            graphs[0].replay()
+        stream.synchronize()
+
+    clocks = Clocks(local_rank)
+    clocks.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        if use_graph:
+            for _ in range(args.steps // G):
+                graphs[0].replay()
+            if graphs[1] is not None:
+                graphs[1].replay()
+        else:
+            for i in range(args.steps):
+                step(i, stream)
+        ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    # steps in the timed graph replay follow the same i % pool order
+    order = [i % G for i in range(G)]
+    if use_graph:
+        per_graph = [step_bytes[i % pool_n] for i in order]
+        avg_bytes = sum(per_graph) / len(per_graph)
+    else:
+        avg_bytes = sum(step_bytes[i % pool_n] for i in range(args.steps)) / args.steps
+    ms_per_step = ms / args.steps
+    tokens = T * args.steps * world
+    value = tokens / (ms / 1e3)
+    peak, peak_kind = peaks()
+    achieved = avg_bytes / (ms_per_step / 1e3) / 1e9
+    traffic = profiled_traffic(args.workload)
+
+    # end to end through the C ABI with host buffers: H2D of x, forward, D2H of out
+    K_e2e = min(args.steps, 2000)
+    hx = torch.from_numpy(xs_np[:8].copy()).pin_memory()
+    hy = torch.empty(8, T, 1280).pin_memory()
+    dx = torch.empty(T, 1280, device=dev)
+    dy = torch.empty(T, 1280, device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(20):
+            dx.copy_(hx[i % 8], non_blocking=True)
+            api.focr_moe_layer_forward(copies[i % N_COPIES], dx, dy, ws, stream=stream)
+            hy[i % 8].copy_(dy, non_blocking=True)
+        stream.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(K_e2e):
+            dx.copy_(hx[i % 8], non_blocking=True)
+            api.focr_moe_layer_forward(copies[i % N_COPIES], dx, dy, ws, stream=stream)
+            hy[i % 8].copy_(dy, non_blocking=True)
+        e1.record(stream)
+        stream.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e_value = T * K_e2e * world / (ms_e2e / 1e3)
+    api.focr_moe_check(ws, stream)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, threads, n, dt, _, _ = oracle_rate(args.workload, budget_s=12.0)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{n} tokens of workload {args.workload} through the CPU oracle (plain C, fp64, "
+                         f"OpenMP over tokens) in {dt:.1f} s; layer quantisation excluded"}
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": dict(describe(args.workload), parallelism=f"replicas x{world}",
+                               graph=("CUDA graph replay" if use_graph else f"eager ({graph_error})")),
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                             "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+                             "kernel": "whole layer forward (router + grouped expert kernel)",
+                             "algorithmic_bytes_per_step": avg_bytes},
+                "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * 1280 * 4,
+                        "d2h_bytes_per_step": T * 1280 * 4, "steps": K_e2e},
+                "gpu_launches": 2 * args.steps,
+                "clocks": clk}
+        print(json.dumps(line), flush=True)
+    del copies
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,168 @@
+/*
+ * focr_moe -- one mixture-of-experts layer forward with group-quantised experts,
+ * for NVIDIA B200 (sm_100a).  C ABI: plain pointers and sizes, no framework types.
+ *
+ * The layer (frankenocr.pages.dev, "One forward pass", step 6; franken_ocr
+ * README, "Architecture" and "Design Philosophy"):
+ *   hidden H = 1280; a softmax router over E = 64 routed experts picks the top
+ *   k = 6 greedily and does NOT renormalise the chosen probabilities; 2 shared
+ *   experts, fused into one SwiGLU of width 1792, always contribute with weight 1;
+ *   each routed expert is a SwiGLU FFN 1280 -> 896 -> 1280:
+ *       expert(x) = D (silu(G x) * (U x)),  silu(v) = v / (1 + exp(-v))
+ *       out[t]    = sum_j p[t, idx_j] * expert_{idx_j}(x_t) + shared(x_t)
+ *   (the layer output has no residual added).
+ * Weight storage (frankenocr.pages.dev, "Four bits, one shared scale"): an int4
+ * weight is a two's-complement nibble sharing one f32 scale with its group; int8
+ * and bf16 are the other formats of the pages' quantisation recipe.
+ *
+ * Conventions for every call:
+ *   - All dimensions are fixed at compile time (the FOCR_* constants below);
+ *     anything else is FOCR_ERR_UNSUPPORTED.
+ *   - Weights are given as HOST fp32 arrays in nn.Linear orientation [out, in],
+ *     row-major, owned by the caller and only read during the call.
+ *   - Activations are DEVICE pointers owned by the caller, fp32 row-major,
+ *     16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Forward calls are asynchronous on that stream; pack/export/clone calls
+ *     synchronise before returning.
+ *   - Arguments are checked before anything is launched; on error nothing is
+ *     launched and focr_last_error() (thread-local) says why.
+ */
+#ifndef FOCR_MOE_H
+#define FOCR_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FOCR_HIDDEN 1280        /* hidden size */
+#define FOCR_EXPERTS 64         /* routed experts */
+#define FOCR_TOPK 6             /* experts per token */
+#define FOCR_INTER 896          /* routed-expert intermediate */
+#define FOCR_SHARED_INTER 1792  /* fused shared experts (2 x 896) */
+#define FOCR_VOCAB 129280       /* lm_head rows */
+#define FOCR_DENSE_INTER 6848   /* dense layer-0 intermediate */
+#define FOCR_T_MAX 8192         /* most tokens one forward call accepts */
+
+typedef enum {
+    FOCR_OK = 0,
+    FOCR_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, T out of range, short workspace */
+    FOCR_ERR_UNSUPPORTED = 2,  /* weight type / group size / dimension not supported */
+    FOCR_ERR_CUDA = 3,         /* a CUDA runtime call failed (message has the CUDA error) */
+    FOCR_ERR_OOM = 4,          /* device or host allocation failed */
+    FOCR_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out (see focr_moe_check) */
+} focr_status;
+
+typedef enum { FOCR_W_BF16 = 0, FOCR_W_INT8 = 1, FOCR_W_INT4 = 2 } focr_wtype;
+
+/* Which matrix of a packed layer focr_moe_export_quantized() returns. */
+typedef enum {
+    FOCR_MAT_GATE = 0, FOCR_MAT_UP = 1, FOCR_MAT_DOWN = 2,          /* routed expert `expert` */
+    FOCR_MAT_SHARED_GATE = 3, FOCR_MAT_SHARED_UP = 4, FOCR_MAT_SHARED_DOWN = 5,
+    FOCR_MAT_ROUTER = 6
+} focr_matrix;
+
+/* Host-side description of one layer's weights (all fp32 except the router). */
+typedef struct {
+    const float* w_gate;          /* [64, 896, 1280] */
+    const float* w_up;            /* [64, 896, 1280] */
+    const float* w_down;          /* [64, 1280, 896] */
+    const float* ws_gate;         /* [1792, 1280]    */
+    const float* ws_up;           /* [1792, 1280]    */
+    const float* ws_down;         /* [1280, 1792]    */
+    const uint16_t* w_router_bf16;/* [64, 1280] bf16 bit patterns */
+    int32_t routed_type;          /* focr_wtype of the routed experts */
+    int32_t shared_type;          /* focr_wtype of the shared expert  */
+    int32_t group_size;           /* 32, 64 or 128 (int4); 128 (int8); ignored for bf16 */
+} focr_moe_weights_desc;
+
+typedef struct focr_moe_layer focr_moe_layer;   /* opaque, device-resident, library-owned */
+
+/* Optional routing outputs of a forward call (each pointer may be NULL; DEVICE memory). */
+typedef struct {
+    float* logits;       /* [T, 64] fp32 router logits                               */
+    int32_t* topk_idx;   /* [T, 6]  chosen experts, best first (ties: lower index)   */
+    float* topk_w;       /* [T, 6]  their softmax probabilities (not renormalised)   */
+    int32_t* counts;     /* [64]    tokens routed to each expert                     */
+    int32_t* offsets;    /* [65]    exclusive prefix sum of counts                   */
+    int32_t* perm;       /* [T*6]   entries t*6+j grouped by expert, token-ascending */
+} focr_moe_route_debug;
+
+/*
+ * focr_moe_pack_weights -- quantise and lay out one layer on the device.
+ * Quantisation ("Four bits, one shared scale"): for every group of g consecutive
+ * input-axis elements of one output row, s = max|w| / Q as one fp32 division
+ * (Q = 7 for int4, 127 for int8), q = round-half-even(w / s) clamped to [-8, 7]
+ * or [-127, 127]; an all-zero group has s = 0, q = 0.  bf16 weights are rounded
+ * to nearest-even; the router is taken as given (bf16).
+ * The device layout is private (tiled for 16-byte loads and bulk copies); use
+ * focr_moe_export_quantized() to read back the canonical codes.
+ * On success *out owns device memory until focr_moe_layer_free().  Synchronises.
+ */
+focr_status focr_moe_pack_weights(const focr_moe_weights_desc* desc, focr_moe_layer** out, void* stream);
+
+/* Device copy of a packed layer (same codes, new memory).  Synchronises. */
+focr_status focr_moe_layer_clone(const focr_moe_layer* src, focr_moe_layer** out, void* stream);
+
+void focr_moe_layer_free(focr_moe_layer* layer);
+
+/* Device bytes held by a packed layer. */
+size_t focr_moe_layer_device_bytes(const focr_moe_layer* layer);
+
+/*
+ * focr_moe_export_sizes / focr_moe_export_quantized -- canonical quantised form of
+ * one matrix (for bit-exact checks).  Canonical codes: int4 as two's-complement
+ * nibbles, element 2j in bits 0-3 and 2j+1 in bits 4-7 of byte j, row-major;
+ * int8 as int8 row-major; bf16 as uint16 bit patterns row-major.  Scales: f32
+ * [rows, ceil(cols / g)] row-major (none for bf16).  `expert` is ignored for the
+ * shared matrices and the router.  Buffers are HOST memory of at least the sizes
+ * focr_moe_export_sizes() reports.  Synchronises.
+ */
+focr_status focr_moe_export_sizes(const focr_moe_layer* layer, int32_t matrix, size_t* code_bytes,
+                                  size_t* n_scales);
+focr_status focr_moe_export_quantized(const focr_moe_layer* layer, int32_t matrix, int32_t expert,
+                                      void* codes_host, size_t code_bytes, float* scales_host,
+                                      size_t n_scales);
+
+/* Workspace a forward call with up to T_max tokens needs (bytes). */
+size_t focr_moe_workspace_bytes(int32_t T_max);
+
+/*
+ * focr_moe_layer_forward -- out[T, 1280] = MoE(hidden[T, 1280]).
+ *   hidden, out : DEVICE fp32, 16-byte aligned, caller-owned; must not overlap.
+ *   1 <= T <= FOCR_T_MAX.
+ *   workspace   : DEVICE scratch of ws_bytes >= focr_moe_workspace_bytes(T), 256-byte
+ *                 aligned.  It must be zero-filled before its first use; every forward
+ *                 leaves its control words zero again.  Calls that share a workspace
+ *                 must be ordered on one stream.
+ *   dbg         : optional routing outputs (NULL for none).
+ * Steps, all on `stream`: router GEMV (fp64 accumulation of exact products,
+ * rounded to fp32) + softmax + greedy top-6 (rank by fp32 logit, ties to the
+ * lower index) + dispatch (counting sort of t*6+j by expert, stable), then the
+ * grouped expert kernel (shared expert and the selected experts, dequantised in
+ * registers, fp32 accumulation) which adds w * expert(x) into out.
+ */
+focr_status focr_moe_layer_forward(const focr_moe_layer* layer, const float* hidden, int32_t T, float* out,
+                                   void* workspace, size_t ws_bytes, const focr_moe_route_debug* dbg,
+                                   void* stream);
+
+/*
+ * focr_moe_check -- read the device error word a forward may have set in `workspace`
+ * (a bounded wait that ran out).  Synchronises `stream`.  Returns FOCR_OK or
+ * FOCR_ERR_TIMEOUT, and clears the word.
+ */
+focr_status focr_moe_check(void* workspace, void* stream);
+
+/* Thread-local description of the last error (empty string if none). */
+const char* focr_last_error(void);
+
+/* Library build string (compiler, arch). */
+const char* focr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FOCR_MOE_H */

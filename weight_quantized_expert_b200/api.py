@@ -1,0 +1,190 @@
+"""Thin Python binding of libfocr_moe (include/focr_moe.h).
+
+Argument marshalling only: every step of the layer runs in the CUDA library.  PyTorch
+provides device memory and the current stream.  There is no fallback: if the
+shared library is missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import numpy as np
+
+from . import synth
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfocr_moe.so")
+
+H, E, TOPK, I, IS, VOCAB, DENSE_I = 1280, 64, 6, 896, 1792, 129280, 6848
+T_MAX = 8192
+W_BF16, W_INT8, W_INT4 = 0, 1, 2
+(MAT_GATE, MAT_UP, MAT_DOWN, MAT_SHARED_GATE, MAT_SHARED_UP, MAT_SHARED_DOWN, MAT_ROUTER) = range(7)
+STATUS = {0: "FOCR_OK", 1: "FOCR_ERR_INVALID_ARG", 2: "FOCR_ERR_UNSUPPORTED", 3: "FOCR_ERR_CUDA",
+          4: "FOCR_ERR_OOM", 5: "FOCR_ERR_TIMEOUT"}
+
+# every symbol include/focr_moe.h declares
+EXPORTED = (
+    "focr_moe_pack_weights", "focr_moe_layer_clone", "focr_moe_layer_free", "focr_moe_layer_device_bytes",
+    "focr_moe_export_sizes", "focr_moe_export_quantized", "focr_moe_workspace_bytes", "focr_moe_layer_forward",
+    "focr_moe_check", "focr_last_error", "focr_version",
+)
+
+
+class FocrError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class WeightsDesc(ctypes.Structure):
+    _fields_ = [("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
+                ("ws_gate", ctypes.c_void_p), ("ws_up", ctypes.c_void_p), ("ws_down", ctypes.c_void_p),
+                ("w_router_bf16", ctypes.c_void_p), ("routed_type", ctypes.c_int32),
+                ("shared_type", ctypes.c_int32), ("group_size", ctypes.c_int32)]
+
+
+class RouteDebug(ctypes.Structure):
+    _fields_ = [("logits", ctypes.c_void_p), ("topk_idx", ctypes.c_void_p), ("topk_w", ctypes.c_void_p),
+                ("counts", ctypes.c_void_p), ("offsets", ctypes.c_void_p), ("perm", ctypes.c_void_p)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib():
+    """Load libfocr_moe.so (built in-tree by weight_quantized_expert_b200/build.py)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with weight_quantized_expert_b200/build.py")
+            L = ctypes.CDLL(LIB_PATH)
+            P, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+            sigs = {
+                "focr_moe_pack_weights": (i32, [ctypes.POINTER(WeightsDesc), ctypes.POINTER(P), P]),
+                "focr_moe_layer_clone": (i32, [P, ctypes.POINTER(P), P]),
+                "focr_moe_layer_free": (None, [P]),
+                "focr_moe_layer_device_bytes": (sz, [P]),
+                "focr_moe_export_sizes": (i32, [P, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]),
+                "focr_moe_export_quantized": (i32, [P, i32, i32, P, sz, P, sz]),
+                "focr_moe_workspace_bytes": (sz, [i32]),
+                "focr_moe_layer_forward": (i32, [P, P, i32, P, P, sz, ctypes.POINTER(RouteDebug), P]),
+                "focr_moe_check": (i32, [P, P]),
+                "focr_last_error": (ctypes.c_char_p, []),
+                "focr_version": (ctypes.c_char_p, []),
+            }
+            for name, (res, args) in sigs.items():
+                fn = getattr(L, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise FocrError(status, lib().focr_last_error().decode())
+
+
+def _stream(stream=None) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    return int(t.data_ptr())
+
+
+def focr_last_error() -> str:
+    return lib().focr_last_error().decode()
+
+
+def focr_version() -> str:
+    return lib().focr_version().decode()
+
+
+class MoELayer:
+    """A packed, device-resident MoE layer (owns its device memory)."""
+
+    def __init__(self, handle: int):
+        self.handle = handle
+
+    def __del__(self):
+        h, self.handle = getattr(self, "handle", None), None
+        if h and _lib is not None:
+            _lib.focr_moe_layer_free(ctypes.c_void_p(h))
+
+    @property
+    def device_bytes(self) -> int:
+        return lib().focr_moe_layer_device_bytes(ctypes.c_void_p(self.handle))
+
+
+def focr_moe_pack_weights(layer: "synth.MoELayerInputs", stream=None) -> MoELayer:
+    arrs = [np.ascontiguousarray(a, np.float32) for a in
+            (layer.gate, layer.up, layer.down, layer.sgate, layer.sup, layer.sdown)]
+    router = np.ascontiguousarray(layer.router_bf16, np.uint16)
+    assert arrs[0].shape == (E, I, H) and arrs[2].shape == (E, H, I) and arrs[3].shape == (IS, H)
+    desc = WeightsDesc(*[a.ctypes.data for a in arrs], router.ctypes.data,
+                       int(layer.routed_type), int(layer.shared_type), int(layer.group))
+    h = ctypes.c_void_p()
+    _check(lib().focr_moe_pack_weights(ctypes.byref(desc), ctypes.byref(h), _stream(stream)))
+    return MoELayer(h.value)
+
+
+def focr_moe_layer_clone(layer: MoELayer, stream=None) -> MoELayer:
+    h = ctypes.c_void_p()
+    _check(lib().focr_moe_layer_clone(ctypes.c_void_p(layer.handle), ctypes.byref(h), _stream(stream)))
+    return MoELayer(h.value)
+
+
+def focr_moe_export_quantized(layer: MoELayer, matrix: int, expert: int = 0):
+    """Canonical codes (bytes as np.uint8 / int8 / uint16) and f32 scales of one matrix."""
+    L = lib()
+    cb, ns = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(L.focr_moe_export_sizes(ctypes.c_void_p(layer.handle), matrix, ctypes.byref(cb), ctypes.byref(ns)))
+    codes = np.empty(cb.value, np.uint8)
+    scales = np.empty(ns.value, np.float32)
+    _check(L.focr_moe_export_quantized(ctypes.c_void_p(layer.handle), matrix, expert, codes.ctypes.data, cb.value,
+                                       scales.ctypes.data if ns.value else None, ns.value))
+    return codes, scales
+
+
+def focr_moe_workspace_bytes(T_max: int) -> int:
+    return int(lib().focr_moe_workspace_bytes(int(T_max)))
+
+
+def new_workspace(T_max: int, device="cuda"):
+    """A zero-filled workspace tensor for forwards with up to T_max tokens."""
+    import torch
+    return torch.zeros(focr_moe_workspace_bytes(T_max), dtype=torch.uint8, device=device)
+
+
+def focr_moe_layer_forward(layer: MoELayer, hidden, out=None, workspace=None, debug: dict | None = None,
+                           stream=None):
+    """out[T, 1280] = MoE(hidden[T, 1280]) on the current (or given) stream.
+    `debug`, if given, maps names of focr_moe_route_debug fields to device tensors to fill."""
+    import torch
+    assert hidden.is_cuda and hidden.dtype == torch.float32 and hidden.is_contiguous() and hidden.shape[-1] == H
+    T = hidden.shape[0]
+    if out is None:
+        out = torch.empty_like(hidden)
+    if workspace is None:
+        workspace = new_workspace(T, hidden.device)
+    dbg = None
+    if debug:
+        dbg = RouteDebug(*[_ptr(debug.get(f)) for f, _ in RouteDebug._fields_])
+    _check(lib().focr_moe_layer_forward(ctypes.c_void_p(layer.handle), _ptr(hidden), T, _ptr(out), _ptr(workspace),
+                                        workspace.numel(), ctypes.byref(dbg) if dbg is not None else None,
+                                        _stream(stream)))
+    return out
+
+
+def focr_moe_check(workspace, stream=None):
+    _check(lib().focr_moe_check(_ptr(workspace), _stream(stream)))

@@ -1,0 +1,319 @@
+// C ABI of libfocr_moe: argument checks, packing, export, forward.  See include/focr_moe.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "pack.h"
+
+using namespace focr;
+
+struct focr_moe_layer {
+    int32_t routed_type, shared_type, group;
+    ItemGeom rg, sg;
+    uint8_t* dev = nullptr;
+    size_t bytes = 0;
+    size_t off_router = 0, off_ritems = 0, off_rdsc = 0, off_sitems = 0, off_sdsc = 0;
+    LayerView view() const {
+        LayerView v{};
+        v.router = reinterpret_cast<const uint16_t*>(dev + off_router);
+        v.routed_items = dev + off_ritems;
+        v.routed_dscale = reinterpret_cast<const float*>(dev + off_rdsc);
+        v.shared_items = dev + off_sitems;
+        v.shared_dscale = reinterpret_cast<const float*>(dev + off_sdsc);
+        v.rg = rg;
+        v.sg = sg;
+        return v;
+    }
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+focr_status fail(focr_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+focr_status fail(focr_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return s;
+}
+
+focr_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(FOCR_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+#define CUDA_TRY(call)                                           \
+    do {                                                         \
+        cudaError_t e__ = (call);                                \
+        if (e__ != cudaSuccess) return cuda_fail(e__, #call);    \
+    } while (0)
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+focr_status check_types(int rt, int st, int g) {
+    auto ok = [&](int wt) {
+        if (wt == FOCR_W_BF16) return true;
+        if (wt == FOCR_W_INT4) return g == 32 || g == 64 || g == 128;
+        if (wt == FOCR_W_INT8) return g == 128;
+        return false;
+    };
+    if (!ok(rt)) return fail(FOCR_ERR_UNSUPPORTED, "routed weight type %d with group %d is not supported", rt, g);
+    if (!ok(st)) return fail(FOCR_ERR_UNSUPPORTED, "shared weight type %d with group %d is not supported", st, g);
+    return FOCR_OK;
+}
+
+void plan(focr_moe_layer* L) {
+    size_t o = 0;
+    L->off_router = o;
+    o = align_up(o + sizeof(uint16_t) * E * H, 256);
+    L->off_ritems = o;
+    o = align_up(o + (size_t)E * L->rg.slices * L->rg.item_bytes, 256);
+    L->off_rdsc = o;
+    o = align_up(o + sizeof(float) * (size_t)E * L->rg.dscale_expert_floats, 256);
+    L->off_sitems = o;
+    o = align_up(o + (size_t)L->sg.slices * L->sg.item_bytes, 256);
+    L->off_sdsc = o;
+    o = align_up(o + sizeof(float) * (size_t)L->sg.dscale_expert_floats, 256);
+    L->bytes = o;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* focr_last_error(void) { return g_err.c_str(); }
+
+const char* focr_version(void) {
+    static char buf[128];
+    snprintf(buf, sizeof(buf), "focr_moe sm_100a cuda %d.%d", CUDART_VERSION / 1000, (CUDART_VERSION % 1000) / 10);
+    return buf;
+}
+
+focr_status focr_moe_pack_weights(const focr_moe_weights_desc* d, focr_moe_layer** out, void* stream) {
+    g_err.clear();
+    if (!d || !out) return fail(FOCR_ERR_INVALID_ARG, "desc and out must not be NULL");
+    *out = nullptr;
+    if (!d->w_gate || !d->w_up || !d->w_down || !d->ws_gate || !d->ws_up || !d->ws_down || !d->w_router_bf16)
+        return fail(FOCR_ERR_INVALID_ARG, "a weight pointer is NULL");
+    focr_status s = check_types(d->routed_type, d->shared_type, d->group_size);
+    if (s != FOCR_OK) return s;
+    focr_moe_layer* L = new (std::nothrow) focr_moe_layer();
+    if (!L) return fail(FOCR_ERR_OOM, "host allocation failed");
+    L->routed_type = d->routed_type;
+    L->shared_type = d->shared_type;
+    L->group = d->group_size;
+    L->rg = make_geom(d->routed_type, d->group_size, I);
+    L->sg = make_geom(d->shared_type, d->group_size, IS);
+    plan(L);
+
+    std::vector<uint8_t> host;
+    try {
+        host.assign(L->bytes, 0);
+    } catch (...) {
+        delete L;
+        return fail(FOCR_ERR_OOM, "host staging of %zu bytes failed", L->bytes);
+    }
+    std::memcpy(host.data() + L->off_router, d->w_router_bf16, sizeof(uint16_t) * E * H);
+    const ItemGeom rg = L->rg;
+    uint8_t* ritems = host.data() + L->off_ritems;
+    float* rdsc = reinterpret_cast<float*>(host.data() + L->off_rdsc);
+    parallel_for(E + 1, [&](int e) {
+        if (e < E) {
+            host_pack_set(d->w_gate + (size_t)e * I * H, d->w_up + (size_t)e * I * H, d->w_down + (size_t)e * H * I,
+                          rg, ritems + (size_t)e * rg.slices * rg.item_bytes, rdsc + (size_t)e * rg.dscale_expert_floats);
+        } else {
+            host_pack_set(d->ws_gate, d->ws_up, d->ws_down, L->sg, host.data() + L->off_sitems,
+                          reinterpret_cast<float*>(host.data() + L->off_sdsc));
+        }
+    });
+
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMalloc(&L->dev, L->bytes);
+    if (e != cudaSuccess) {
+        delete L;
+        return fail(e == cudaErrorMemoryAllocation ? FOCR_ERR_OOM : FOCR_ERR_CUDA, "cudaMalloc(%zu): %s", L->bytes,
+                    cudaGetErrorString(e));
+    }
+    e = cudaMemcpyAsync(L->dev, host.data(), L->bytes, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) {
+        cudaFree(L->dev);
+        delete L;
+        return cuda_fail(e, "upload of packed layer");
+    }
+    *out = L;
+    return FOCR_OK;
+}
+
+focr_status focr_moe_layer_clone(const focr_moe_layer* src, focr_moe_layer** out, void* stream) {
+    g_err.clear();
+    if (!src || !out) return fail(FOCR_ERR_INVALID_ARG, "src and out must not be NULL");
+    *out = nullptr;
+    focr_moe_layer* L = new (std::nothrow) focr_moe_layer(*src);
+    if (!L) return fail(FOCR_ERR_OOM, "host allocation failed");
+    L->dev = nullptr;
+    cudaError_t e = cudaMalloc(&L->dev, L->bytes);
+    if (e != cudaSuccess) {
+        delete L;
+        return fail(e == cudaErrorMemoryAllocation ? FOCR_ERR_OOM : FOCR_ERR_CUDA, "cudaMalloc(%zu): %s", src->bytes,
+                    cudaGetErrorString(e));
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    e = cudaMemcpyAsync(L->dev, src->dev, L->bytes, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) {
+        cudaFree(L->dev);
+        delete L;
+        return cuda_fail(e, "clone copy");
+    }
+    *out = L;
+    return FOCR_OK;
+}
+
+void focr_moe_layer_free(focr_moe_layer* L) {
+    if (!L) return;
+    if (L->dev) cudaFree(L->dev);
+    delete L;
+}
+
+size_t focr_moe_layer_device_bytes(const focr_moe_layer* L) { return L ? L->bytes : 0; }
+
+static bool matrix_shape(const focr_moe_layer* L, int32_t m, int* wtype, int64_t* rows, int64_t* cols, int* group) {
+    switch (m) {
+        case FOCR_MAT_GATE: case FOCR_MAT_UP:
+            *wtype = L->routed_type; *rows = I; *cols = H; break;
+        case FOCR_MAT_DOWN:
+            *wtype = L->routed_type; *rows = H; *cols = I; break;
+        case FOCR_MAT_SHARED_GATE: case FOCR_MAT_SHARED_UP:
+            *wtype = L->shared_type; *rows = IS; *cols = H; break;
+        case FOCR_MAT_SHARED_DOWN:
+            *wtype = L->shared_type; *rows = H; *cols = IS; break;
+        case FOCR_MAT_ROUTER:
+            *wtype = FOCR_W_BF16; *rows = E; *cols = H; break;
+        default:
+            return false;
+    }
+    *group = is_quant(*wtype) ? L->group : 0;
+    return true;
+}
+
+focr_status focr_moe_export_sizes(const focr_moe_layer* L, int32_t matrix, size_t* code_bytes, size_t* n_scales) {
+    g_err.clear();
+    if (!L || !code_bytes || !n_scales) return fail(FOCR_ERR_INVALID_ARG, "NULL argument");
+    int wt, g;
+    int64_t rows, cols;
+    if (!matrix_shape(L, matrix, &wt, &rows, &cols, &g)) return fail(FOCR_ERR_INVALID_ARG, "unknown matrix %d", matrix);
+    const size_t n = (size_t)(rows * cols);
+    *code_bytes = wt == FOCR_W_INT4 ? n / 2 : (wt == FOCR_W_INT8 ? n : 2 * n);
+    *n_scales = is_quant(wt) ? (size_t)rows * (size_t)((cols + g - 1) / g) : 0;
+    return FOCR_OK;
+}
+
+focr_status focr_moe_export_quantized(const focr_moe_layer* L, int32_t matrix, int32_t expert, void* codes,
+                                      size_t code_bytes, float* scales, size_t n_scales) {
+    size_t need_c, need_s;
+    focr_status s = focr_moe_export_sizes(L, matrix, &need_c, &need_s);
+    if (s != FOCR_OK) return s;
+    const bool routed = matrix <= FOCR_MAT_DOWN;
+    if (routed && (expert < 0 || expert >= E)) return fail(FOCR_ERR_INVALID_ARG, "expert %d out of range", expert);
+    if (!codes || code_bytes < need_c) return fail(FOCR_ERR_INVALID_ARG, "codes buffer too small (need %zu)", need_c);
+    if (need_s && (!scales || n_scales < need_s))
+        return fail(FOCR_ERR_INVALID_ARG, "scales buffer too small (need %zu)", need_s);
+    if (matrix == FOCR_MAT_ROUTER) {
+        CUDA_TRY(cudaMemcpy(codes, L->dev + L->off_router, need_c, cudaMemcpyDeviceToHost));
+        return FOCR_OK;
+    }
+    const ItemGeom& g = routed ? L->rg : L->sg;
+    const size_t items_bytes = (size_t)g.slices * g.item_bytes;
+    const size_t item_off = routed ? L->off_ritems + (size_t)expert * items_bytes : L->off_sitems;
+    const size_t dsc_off = routed ? L->off_rdsc + sizeof(float) * (size_t)expert * g.dscale_expert_floats : L->off_sdsc;
+    std::vector<uint8_t> items(items_bytes);
+    std::vector<float> dsc(g.dscale_expert_floats);
+    CUDA_TRY(cudaMemcpy(items.data(), L->dev + item_off, items_bytes, cudaMemcpyDeviceToHost));
+    if (!dsc.empty())
+        CUDA_TRY(cudaMemcpy(dsc.data(), L->dev + dsc_off, dsc.size() * sizeof(float), cudaMemcpyDeviceToHost));
+    const int which = (matrix == FOCR_MAT_GATE || matrix == FOCR_MAT_SHARED_GATE) ? 0
+                      : (matrix == FOCR_MAT_UP || matrix == FOCR_MAT_SHARED_UP) ? 1 : 2;
+    int wt, grp;
+    int64_t rows, cols;
+    matrix_shape(L, matrix, &wt, &rows, &cols, &grp);
+    const size_t n = (size_t)(rows * cols);
+    if (wt == FOCR_W_BF16) {
+        host_unpack_matrix(items.data(), nullptr, g, which, nullptr, reinterpret_cast<uint16_t*>(codes), nullptr);
+    } else {
+        std::vector<int8_t> q(n);
+        host_unpack_matrix(items.data(), dsc.data(), g, which, q.data(), nullptr, scales);
+        if (wt == FOCR_W_INT8) {
+            std::memcpy(codes, q.data(), n);
+        } else {
+            uint8_t* c = reinterpret_cast<uint8_t*>(codes);
+            for (size_t j = 0; j < n / 2; ++j)
+                c[j] = (uint8_t)(((uint8_t)q[2 * j] & 0xFu) | (((uint8_t)q[2 * j + 1] & 0xFu) << 4));
+        }
+    }
+    return FOCR_OK;
+}
+
+size_t focr_moe_workspace_bytes(int32_t T_max) {
+    if (T_max < 1) T_max = 1;
+    if (T_max > FOCR_T_MAX) T_max = FOCR_T_MAX;
+    return ws_layout(T_max).total;
+}
+
+focr_status focr_moe_layer_forward(const focr_moe_layer* L, const float* hidden, int32_t T, float* out,
+                                   void* workspace, size_t ws_bytes, const focr_moe_route_debug* dbg, void* stream) {
+    g_err.clear();
+    if (!L || !L->dev) return fail(FOCR_ERR_INVALID_ARG, "layer is NULL");
+    if (T < 1 || T > FOCR_T_MAX) return fail(FOCR_ERR_INVALID_ARG, "T=%d outside [1, %d]", T, FOCR_T_MAX);
+    if (!hidden || !out || !workspace) return fail(FOCR_ERR_INVALID_ARG, "hidden, out and workspace must not be NULL");
+    if (!aligned(hidden, 16) || !aligned(out, 16)) return fail(FOCR_ERR_INVALID_ARG, "hidden/out must be 16-byte aligned");
+    if (!aligned(workspace, 256)) return fail(FOCR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const size_t need = ws_layout(T).total;
+    if (ws_bytes < need) return fail(FOCR_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed for T=%d", ws_bytes, need, T);
+    {
+        const char* h0 = (const char*)hidden;
+        const char* o0 = (const char*)out;
+        const size_t nb = (size_t)T * H * sizeof(float);
+        if (h0 < o0 + nb && o0 < h0 + nb) return fail(FOCR_ERR_INVALID_ARG, "hidden and out overlap");
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    const RouteView R = route_view(workspace, T);
+    const LayerView V = L->view();
+    CUDA_TRY(launch_router(hidden, T, T, V, R, out, st));
+    CUDA_TRY(launch_expert_decode(hidden, T, V, R, out, st));
+    if (dbg) {
+        if (dbg->logits) CUDA_TRY(cudaMemcpyAsync(dbg->logits, R.logits, sizeof(float) * T * E, cudaMemcpyDeviceToDevice, st));
+        if (dbg->topk_idx) CUDA_TRY(cudaMemcpyAsync(dbg->topk_idx, R.topk_idx, sizeof(int32_t) * T * K, cudaMemcpyDeviceToDevice, st));
+        if (dbg->topk_w) CUDA_TRY(cudaMemcpyAsync(dbg->topk_w, R.topk_w, sizeof(float) * T * K, cudaMemcpyDeviceToDevice, st));
+        if (dbg->counts) CUDA_TRY(cudaMemcpyAsync(dbg->counts, R.counts, sizeof(int32_t) * E, cudaMemcpyDeviceToDevice, st));
+        if (dbg->offsets) CUDA_TRY(cudaMemcpyAsync(dbg->offsets, R.offsets, sizeof(int32_t) * (E + 1), cudaMemcpyDeviceToDevice, st));
+        if (dbg->perm) CUDA_TRY(cudaMemcpyAsync(dbg->perm, R.perm, sizeof(int32_t) * T * K, cudaMemcpyDeviceToDevice, st));
+    }
+    return FOCR_OK;
+}
+
+focr_status focr_moe_check(void* workspace, void* stream) {
+    g_err.clear();
+    if (!workspace) return fail(FOCR_ERR_INVALID_ARG, "workspace is NULL");
+    cudaStream_t st = (cudaStream_t)stream;
+    int32_t* ctrl = reinterpret_cast<int32_t*>((char*)workspace + ws_layout(1).ctrl);
+    int32_t v = 0;
+    CUDA_TRY(cudaMemcpyAsync(&v, ctrl + CTRL_ERROR, sizeof(v), cudaMemcpyDeviceToHost, st));
+    CUDA_TRY(cudaStreamSynchronize(st));
+    if (v != 0) {
+        const int32_t zero = 0;
+        CUDA_TRY(cudaMemcpyAsync(ctrl + CTRL_ERROR, &zero, sizeof(zero), cudaMemcpyHostToDevice, st));
+        CUDA_TRY(cudaStreamSynchronize(st));
+        return fail(FOCR_ERR_TIMEOUT, "device wait ran out (code %d)", v);
+    }
+    return FOCR_OK;
+}
+
+}  // extern "C"

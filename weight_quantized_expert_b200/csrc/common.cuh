@@ -1,0 +1,288 @@
+// Internal definitions shared by the kernels and the C ABI of libfocr_moe.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/focr_moe.h"
+
+namespace focr {
+
+constexpr int H = FOCR_HIDDEN;
+constexpr int E = FOCR_EXPERTS;
+constexpr int K = FOCR_TOPK;
+constexpr int I = FOCR_INTER;
+constexpr int IS = FOCR_SHARED_INTER;
+
+// ---------------------------------------------------------------------------------------
+// Device layout of a SwiGLU weight set ("item" = one slice of S intermediate rows).
+//
+// For a slice [i0, i0 + S) of the intermediate axis the item block holds, contiguously:
+//   GU weights : [S/2 quads][160 units][4 rows][UB bytes]
+//                quad q = rows (gate i0+2q, gate i0+2q+1, up i0+2q, up i0+2q+1);
+//                unit u = input columns [8u, 8u+8); UB = 4 (int4), 8 (int8), 16 (bf16)
+//   GU scales  : [S/2 quads][1280/g groups][4 rows] f32          (quantised types only)
+//   D weights  : [1280 rows][16 bytes]  = down[row, i0 : i0+S]   (S*bits = 128)
+// and, outside the item block, the down scales of the whole expert:
+//   D scales   : [inter/g groups][1280 rows] f32                  (quantised types only)
+// Codes are stored offset-binary: int4 as q+8 (nibble of column 8u+2b in the low half
+// of byte b, column 8u+2b+1 in the high half), int8 as q+128; bf16 as bit patterns.
+// S is 32 (int4), 16 (int8), 8 (bf16) so a down row slice is always 16 bytes.
+// ---------------------------------------------------------------------------------------
+constexpr int UNITS = H / 8;  // 160 units of 8 input columns
+
+__host__ __device__ constexpr int slice_rows(int wtype) {
+    return wtype == FOCR_W_INT4 ? 32 : (wtype == FOCR_W_INT8 ? 16 : 8);
+}
+__host__ __device__ constexpr int unit_row_bytes(int wtype) {
+    return wtype == FOCR_W_INT4 ? 4 : (wtype == FOCR_W_INT8 ? 8 : 16);
+}
+__host__ __device__ constexpr bool is_quant(int wtype) { return wtype != FOCR_W_BF16; }
+
+struct ItemGeom {
+    int wtype, group, S, inter, slices;
+    uint32_t gu_w_bytes, gu_s_bytes, d_w_bytes, item_bytes;  // item_bytes: 128-byte multiple
+    uint32_t dscale_expert_floats;                           // inter/g * 1280 (0 for bf16)
+};
+
+__host__ __device__ inline ItemGeom make_geom(int wtype, int group, int inter) {
+    ItemGeom g{};
+    g.wtype = wtype;
+    g.group = is_quant(wtype) ? group : 0;
+    g.S = slice_rows(wtype);
+    g.inter = inter;
+    g.slices = inter / g.S;
+    g.gu_w_bytes = (uint32_t)(g.S / 2) * UNITS * 4 * unit_row_bytes(wtype);
+    g.gu_s_bytes = is_quant(wtype) ? (uint32_t)(g.S / 2) * (H / group) * 4 * 4 : 0u;
+    g.d_w_bytes = (uint32_t)H * 16;
+    uint32_t raw = g.gu_w_bytes + g.gu_s_bytes + g.d_w_bytes;
+    g.item_bytes = (raw + 127u) & ~127u;
+    g.dscale_expert_floats = is_quant(wtype) ? (uint32_t)(inter / group) * H : 0u;
+    return g;
+}
+
+// Device-side view of a packed layer (passed by value to kernels).
+struct LayerView {
+    const uint16_t* router;        // [64][1280] bf16
+    const uint8_t* routed_items;   // [64][slices][item_bytes]
+    const float* routed_dscale;    // [64][inter/g][1280]
+    const uint8_t* shared_items;   // [slices][item_bytes]
+    const float* shared_dscale;    // [1792/g][1280]
+    ItemGeom rg, sg;
+};
+
+// ---------------------------------------------------------------------------------------
+// Workspace layout (bytes from the workspace base).  Control words first; they are
+// zero on entry and every forward returns them to zero.
+// ---------------------------------------------------------------------------------------
+constexpr int ROUTER_KSPLIT = 5;          // 1280 = 5 x 256 input columns per router CTA
+constexpr int ROUTER_TB = 8;              // tokens per router CTA
+constexpr int MAX_TB = (FOCR_T_MAX + ROUTER_TB - 1) / ROUTER_TB;
+
+struct WsLayout {
+    size_t ctrl;          // int32 [MAX_TB tickets][1 global ticket][1 error word][pad]
+    size_t partial;       // f64 [KSPLIT][T_max][64]
+    size_t logits;        // f32 [T_max][64]
+    size_t topk_idx;      // i32 [T_max][6]
+    size_t topk_w;        // f32 [T_max][6]
+    size_t counts;        // i32 [64]
+    size_t offsets;       // i32 [65]
+    size_t active;        // i32 [64] experts with tokens, ascending; [64] = U
+    size_t perm;          // i32 [T_max*6]
+    size_t total;
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline WsLayout ws_layout(int T_max) {
+    WsLayout w{};
+    size_t o = 0;
+    w.ctrl = o;      o = align_up(o + sizeof(int32_t) * (MAX_TB + 64), 256);
+    w.partial = o;   o = align_up(o + sizeof(double) * ROUTER_KSPLIT * (size_t)T_max * E, 256);
+    w.logits = o;    o = align_up(o + sizeof(float) * (size_t)T_max * E, 256);
+    w.topk_idx = o;  o = align_up(o + sizeof(int32_t) * (size_t)T_max * K, 256);
+    w.topk_w = o;    o = align_up(o + sizeof(float) * (size_t)T_max * K, 256);
+    w.counts = o;    o = align_up(o + sizeof(int32_t) * E, 256);
+    w.offsets = o;   o = align_up(o + sizeof(int32_t) * (E + 1), 256);
+    w.active = o;    o = align_up(o + sizeof(int32_t) * (E + 1), 256);
+    w.perm = o;      o = align_up(o + sizeof(int32_t) * (size_t)T_max * K, 256);
+    w.total = o;
+    return w;
+}
+
+// control-word indices (int32) inside ws.ctrl
+constexpr int CTRL_GLOBAL_TICKET = MAX_TB;
+constexpr int CTRL_ERROR = MAX_TB + 1;
+
+struct RouteView {   // device pointers into the workspace
+    int32_t* ctrl;
+    double* partial;
+    float* logits;
+    int32_t* topk_idx;
+    float* topk_w;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* active;
+    int32_t* perm;
+};
+
+inline RouteView route_view(void* ws, int T_max) {
+    WsLayout L = ws_layout(T_max);
+    char* b = (char*)ws;
+    return RouteView{(int32_t*)(b + L.ctrl), (double*)(b + L.partial), (float*)(b + L.logits),
+                     (int32_t*)(b + L.topk_idx), (float*)(b + L.topk_w), (int32_t*)(b + L.counts),
+                     (int32_t*)(b + L.offsets), (int32_t*)(b + L.active), (int32_t*)(b + L.perm)};
+}
+
+// error codes a kernel may store in the error word
+constexpr int DEVERR_FULL_WAIT = 1;
+constexpr int DEVERR_EMPTY_WAIT = 2;
+
+// ------------------------------------------------------------------ launchers (per .cu)
+cudaError_t launch_router(const float* x, int T, int T_ws, const LayerView& L, const RouteView& R, float* out,
+                          cudaStream_t st);
+cudaError_t launch_expert_decode(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
+                                 cudaStream_t st);
+
+}  // namespace focr
+
+// ---------------------------------------------------------------------------------------
+// PTX helpers (device only)
+// ---------------------------------------------------------------------------------------
+#ifdef __CUDACC__
+namespace focr {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase with the given parity to complete; give up after ~limit_ns.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+// Bulk (non-tensor) async copy global -> own shared memory, completing on an mbarrier.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                         uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
+        "%4;" ::"r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// Programmatic dependent launch controls.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Named barrier over `count` threads (id != 0).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(const void* p) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
+}
+
+__device__ __forceinline__ float4 lds128f(const void* p) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
+}
+
+// ------------------------------------------------------------------ dequantisation
+// A float whose bits are 0x4B0000vv equals 2^23 + vv exactly; subtracting 2^23 + bias
+// recovers the signed code.  __byte_perm places byte j of `src` under the exponent.
+__device__ __forceinline__ float byte_to_float(uint32_t src, int j) {
+    return __uint_as_float(__byte_perm(src, 0x4B000000u, 0x7440u | (uint32_t)j));
+}
+
+// 8 int4 codes (offset-binary, columns c..c+7 of one row) -> 8 floats q in [-8, 7]
+__device__ __forceinline__ void dq_int4x8(uint32_t w, float (&q)[8]) {
+    const uint32_t lo = w & 0x0F0F0F0Fu;          // columns c, c+2, c+4, c+6
+    const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;   // columns c+1, c+3, c+5, c+7
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        q[2 * b] = byte_to_float(lo, b) - 8388616.0f;
+        q[2 * b + 1] = byte_to_float(hi, b) - 8388616.0f;
+    }
+}
+
+// 4 int8 codes (offset-binary) -> 4 floats q in [-127, 127]
+__device__ __forceinline__ void dq_int8x4(uint32_t w, float (&q)[4]) {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) q[b] = byte_to_float(w, b) - 8388736.0f;
+}
+
+// 2 bf16 -> 2 floats
+__device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& a, float& b) {
+    a = __uint_as_float(w << 16);
+    b = __uint_as_float(w & 0xFFFF0000u);
+}
+
+}  // namespace focr
+#endif
