@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--copies", type=int, default=N_COPIES, help="packed layer copies to rotate over")
+    ap.add_argument("--eager", action="store_true", help="launch every step from Python (no CUDA graph)")
     return ap.parse_args()
 
 
@@ -57,6 +59,10 @@ def describe(name: str) -> dict:
             "shared": tname[w["shared"]] if w["shared"] == 0 else f"{tname[w['shared']]} g{w['group']}",
             "router": "bf16", "seed": w["seed"], "hidden": 1280, "experts": "64 routed top-6 + shared 1792",
             "l2": f"rotated over {N_COPIES} packed layer copies (> 2 GB, L2 is 126 MB) and distinct inputs"}
+
+
+def l2_note(n_copies: int) -> str:
+    return f"rotated over {n_copies} packed layer copies (~{n_copies * 138} MB; L2 is 126 MB) and distinct inputs"
 
 
 def peaks():
@@ -217,7 +223,8 @@ def run_ours(args, rank, world, local_rank):
     x_np, layer = synth.workload(args.workload)
     base = api.focr_moe_pack_weights(layer)
     del layer
-    copies = [base] + [api.focr_moe_layer_clone(base) for _ in range(N_COPIES - 1)]
+    n_copies = max(1, args.copies)
+    copies = [base] + [api.focr_moe_layer_clone(base) for _ in range(n_copies - 1)]
     pool_n = 64
     xs_np = synth.hidden(w["seed"] + 2000 + rank, pool_n * T, skew=w.get("skew", False)).reshape(pool_n, T, 1280)
     xs = torch.from_numpy(xs_np).to(dev)
@@ -226,7 +233,7 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.Stream(device=dev)
 
     def step(i, st=None):
-        api.focr_moe_layer_forward(copies[i % N_COPIES], xs[i % pool_n], outs[i % pool_n], ws, stream=st)
+        api.focr_moe_layer_forward(copies[i % n_copies], xs[i % pool_n], outs[i % pool_n], ws, stream=st)
 
     # experts hit per step (for the algorithmic bytes): route each pool entry once
     hits = []
@@ -245,8 +252,11 @@ def run_ours(args, rank, world, local_rank):
     stream.synchronize()
     G = 160
     graphs = []
-    use_graph = True
+    use_graph = not args.eager
+    graph_error = "--eager"
     try:
+        if not use_graph:
+            raise RuntimeError("--eager")
         g_main = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_main, stream=stream):
             for i in range(G):
@@ -259,7 +269,7 @@ def run_ours(args, rank, world, local_rank):
                 for i in range(tail):
                     step(i, torch.cuda.current_stream())
         graphs = (g_main, g_tail)
-    except Exception as exc:  # pragma: no cover - reported in the JSON line
+    except Exception as exc:  # reported in the JSON line
         use_graph = False
         graph_error = str(exc).splitlines()[0]
     if use_graph:
@@ -317,7 +327,7 @@ def run_ours(args, rank, world, local_rank):
     with torch.cuda.stream(stream):
         for i in range(20):
             dx.copy_(hx[i % 8], non_blocking=True)
-            api.focr_moe_layer_forward(copies[i % N_COPIES], dx, dy, ws, stream=stream)
+            api.focr_moe_layer_forward(copies[i % n_copies], dx, dy, ws, stream=stream)
             hy[i % 8].copy_(dy, non_blocking=True)
         stream.synchronize()
         if world > 1:
@@ -327,7 +337,7 @@ def run_ours(args, rank, world, local_rank):
         e0.record(stream)
         for i in range(K_e2e):
             dx.copy_(hx[i % 8], non_blocking=True)
-            api.focr_moe_layer_forward(copies[i % N_COPIES], dx, dy, ws, stream=stream)
+            api.focr_moe_layer_forward(copies[i % n_copies], dx, dy, ws, stream=stream)
             hy[i % 8].copy_(dy, non_blocking=True)
         e1.record(stream)
         stream.synchronize()
@@ -349,7 +359,7 @@ def run_ours(args, rank, world, local_rank):
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": dict(describe(args.workload), parallelism=f"replicas x{world}",
+                "config": dict(describe(args.workload), parallelism=f"replicas x{world}", l2=l2_note(n_copies),
                                graph=("CUDA graph replay" if use_graph else f"eager ({graph_error})")),
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                              "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,

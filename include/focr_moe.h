@@ -150,6 +150,30 @@ focr_status focr_moe_layer_forward(const focr_moe_layer* layer, const float* hid
                                    void* stream);
 
 /*
+ * focr_moe_layer_forward_noalloc -- the same forward as focr_moe_layer_forward, for
+ * callers that cannot allocate device memory where they run the layer (a plug-in or
+ * callback inside an application that owns the device memory budget, or
+ * latency-critical code that must not call cudaMalloc, which can block and
+ * synchronise the device).  The pages have no counterpart of this entry point.
+ *   - Allocates nothing: no cudaMalloc/cudaFree and no allocating library routine.
+ *     Its scratch is a fixed array of FOCR_NOALLOC_SCRATCH_BYTES in the library's
+ *     device image, held by every GPU that loads the library until process exit.
+ *   - 1 <= T <= FOCR_NOALLOC_T_MAX; a larger T is rejected with FOCR_ERR_INVALID_ARG.
+ *   - hidden, out, dbg, stream: as for focr_moe_layer_forward (caller-owned buffers).
+ *   - The first call on a device looks up the array's device address and zero-fills
+ *     it synchronously; make that first call before any stream capture.  Every later
+ *     call clears the control words asynchronously on `stream` before the forward.
+ *   - All calls share the one array and it keeps the last call's contents: calls that
+ *     overlap on the GPU (other streams, other host threads) race and give wrong
+ *     results.  Serialise them on one stream.
+ *   - A device wait that runs out is cleared by the next call rather than reported.
+ */
+#define FOCR_NOALLOC_T_MAX 320
+#define FOCR_NOALLOC_SCRATCH_BYTES 929792
+focr_status focr_moe_layer_forward_noalloc(const focr_moe_layer* layer, const float* hidden, int32_t T, float* out,
+                                           const focr_moe_route_debug* dbg, void* stream);
+
+/*
  * focr_moe_check -- read the device error word a forward may have set in `workspace`
  * (a bounded wait that ran out).  Synchronises `stream`.  Returns FOCR_OK or
  * FOCR_ERR_TIMEOUT, and clears the word.

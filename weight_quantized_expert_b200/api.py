@@ -28,8 +28,9 @@ STATUS = {0: "FOCR_OK", 1: "FOCR_ERR_INVALID_ARG", 2: "FOCR_ERR_UNSUPPORTED", 3:
 EXPORTED = (
     "focr_moe_pack_weights", "focr_moe_layer_clone", "focr_moe_layer_free", "focr_moe_layer_device_bytes",
     "focr_moe_export_sizes", "focr_moe_export_quantized", "focr_moe_workspace_bytes", "focr_moe_layer_forward",
-    "focr_moe_check", "focr_last_error", "focr_version",
+    "focr_moe_check", "focr_last_error", "focr_version", "focr_moe_layer_forward_noalloc",
 )
+NOALLOC_T_MAX = 320
 
 
 class FocrError(RuntimeError):
@@ -73,6 +74,7 @@ def lib():
                 "focr_moe_workspace_bytes": (sz, [i32]),
                 "focr_moe_layer_forward": (i32, [P, P, i32, P, P, sz, ctypes.POINTER(RouteDebug), P]),
                 "focr_moe_check": (i32, [P, P]),
+                "focr_moe_layer_forward_noalloc": (i32, [P, P, i32, P, ctypes.POINTER(RouteDebug), P]),
                 "focr_last_error": (ctypes.c_char_p, []),
                 "focr_version": (ctypes.c_char_p, []),
             }
@@ -183,6 +185,22 @@ def focr_moe_layer_forward(layer: MoELayer, hidden, out=None, workspace=None, de
     _check(lib().focr_moe_layer_forward(ctypes.c_void_p(layer.handle), _ptr(hidden), T, _ptr(out), _ptr(workspace),
                                         workspace.numel(), ctypes.byref(dbg) if dbg is not None else None,
                                         _stream(stream)))
+    return out
+
+
+def focr_moe_layer_forward_noalloc(layer: MoELayer, hidden, out=None, debug: dict | None = None, stream=None):
+    """The forward for callers that cannot allocate device memory: the library's own fixed
+    scratch array replaces the workspace (T <= NOALLOC_T_MAX; calls must not overlap)."""
+    import torch
+    assert hidden.is_cuda and hidden.dtype == torch.float32 and hidden.is_contiguous() and hidden.shape[-1] == H
+    T = hidden.shape[0]
+    if out is None:
+        out = torch.empty_like(hidden)
+    dbg = None
+    if debug:
+        dbg = RouteDebug(*[_ptr(debug.get(f)) for f, _ in RouteDebug._fields_])
+    _check(lib().focr_moe_layer_forward_noalloc(ctypes.c_void_p(layer.handle), _ptr(hidden), T, _ptr(out),
+                                                ctypes.byref(dbg) if dbg is not None else None, _stream(stream)))
     return out
 
 

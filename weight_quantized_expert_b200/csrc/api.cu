@@ -86,6 +86,14 @@ void plan(focr_moe_layer* L) {
 
 }  // namespace
 
+namespace focr {
+// Record a message for focr_last_error() from another translation unit of the library.
+focr_status report_error(focr_status s, const char* msg) {
+    g_err = msg;
+    return s;
+}
+}  // namespace focr
+
 extern "C" {
 
 const char* focr_last_error(void) { return g_err.c_str(); }

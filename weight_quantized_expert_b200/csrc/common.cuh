@@ -92,9 +92,9 @@ struct WsLayout {
     size_t total;
 };
 
-inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-inline WsLayout ws_layout(int T_max) {
+constexpr WsLayout ws_layout(int T_max) {
     WsLayout w{};
     size_t o = 0;
     w.ctrl = o;      o = align_up(o + sizeof(int32_t) * (MAX_TB + 64), 256);
