@@ -169,7 +169,7 @@ focr_status focr_moe_layer_forward(const focr_moe_layer* layer, const float* hid
  *   - A device wait that runs out is cleared by the next call rather than reported.
  */
 #define FOCR_NOALLOC_T_MAX 320
-#define FOCR_NOALLOC_SCRATCH_BYTES 929792
+#define FOCR_NOALLOC_SCRATCH_BYTES 110592
 focr_status focr_moe_layer_forward_noalloc(const focr_moe_layer* layer, const float* hidden, int32_t T, float* out,
                                            const focr_moe_route_debug* dbg, void* stream);
 

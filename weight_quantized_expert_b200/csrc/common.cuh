@@ -17,19 +17,29 @@ constexpr int IS = FOCR_SHARED_INTER;
 // ---------------------------------------------------------------------------------------
 // Device layout of a SwiGLU weight set ("item" = one slice of S intermediate rows).
 //
-// For a slice [i0, i0 + S) of the intermediate axis the item block holds, contiguously:
-//   GU weights : [S/2 quads][160 units][4 rows][UB bytes]
-//                quad q = rows (gate i0+2q, gate i0+2q+1, up i0+2q, up i0+2q+1);
-//                unit u = input columns [8u, 8u+8); UB = 4 (int4), 8 (int8), 16 (bf16)
-//   GU scales  : [S/2 quads][1280/g groups][4 rows] f32          (quantised types only)
-//   D weights  : [1280 rows][16 bytes]  = down[row, i0 : i0+S]   (S*bits = 128)
+// The decode kernel feeds 16x8x16 tensor-core fragments straight from registers, so the
+// packer stores every weight where the lane that needs it will load it.  For a slice
+// [i0, i0 + S) of the intermediate axis, tile t (of S/8) stacks 8 gate rows over the 8
+// matching up rows: tile row g < 8 is gate row i0+8t+g, tile row g+8 is up row i0+8t+g.
+// Lane L = 4*gr + c of a warp holds, for k-step q (input columns 16q .. 16q+15), the
+// eight A-fragment elements
+//   e0..e7 = (gr, k0) (gr, k0+1) (gr+8, k0) (gr+8, k0+1) (gr, k0+8) (gr, k0+9) (gr+8, k0+8) (gr+8, k0+9)
+// with k0 = 16q + 2c.  The item block holds, contiguously:
+//   GU weights : [tile][q / KPV][lane][KPV * FB bytes]   FB = 4 (int4), 8 (int8), 16 (bf16),
+//                KPV = 16 / FB k-steps per 16-byte lane vector
+//   GU scales  : [tile][1280/g groups][8 gr][2 (gate, up)] f32      (quantised types only)
+//   D weights  : [80 output tiles][lane][8 bytes]  rows 16m+gr, 16m+gr+8 of down[:, i0 : i0+S]
+//                (int4: two k-steps; int8: one k-step; bf16: one 16x8x8 step, elements
+//                (gr, 2c) (gr, 2c+1) (gr+8, 2c) (gr+8, 2c+1))
 // and, outside the item block, the down scales of the whole expert:
-//   D scales   : [inter/g groups][1280 rows] f32                  (quantised types only)
-// Codes are stored offset-binary: int4 as q+8 (nibble of column 8u+2b in the low half
-// of byte b, column 8u+2b+1 in the high half), int8 as q+128; bf16 as bit patterns.
-// S is 32 (int4), 16 (int8), 8 (bf16) so a down row slice is always 16 bytes.
+//   D scales   : [inter/g groups][1280 rows] f32                     (quantised types only)
+// Codes are offset-binary: int4 q+8 with e0..e7 in nibble slots 0,4,1,5,2,6,3,7 of a
+// 32-bit word (so one mask pulls a register pair); int8 q+128 in bytes e0..e7; bf16 as
+// bit patterns.  S is 32 (int4), 16 (int8), 8 (bf16): a down row slice is always 16 bytes.
 // ---------------------------------------------------------------------------------------
-constexpr int UNITS = H / 8;  // 160 units of 8 input columns
+constexpr int UNITS = H / 8;  // 160 units of 8 input columns (item size bookkeeping)
+constexpr int KSTEPS = H / 16;  // 80 k-steps of 16 input columns
+constexpr int OTILES = H / 16;  // 80 output tiles of 16 rows
 
 __host__ __device__ constexpr int slice_rows(int wtype) {
     return wtype == FOCR_W_INT4 ? 32 : (wtype == FOCR_W_INT8 ? 16 : 8);
@@ -37,7 +47,23 @@ __host__ __device__ constexpr int slice_rows(int wtype) {
 __host__ __device__ constexpr int unit_row_bytes(int wtype) {
     return wtype == FOCR_W_INT4 ? 4 : (wtype == FOCR_W_INT8 ? 8 : 16);
 }
+__host__ __device__ constexpr int frag_bytes(int wtype) { return unit_row_bytes(wtype); }
+__host__ __device__ constexpr int ksteps_per_vec(int wtype) { return 16 / frag_bytes(wtype); }
 __host__ __device__ constexpr bool is_quant(int wtype) { return wtype != FOCR_W_BF16; }
+// nibble slot of A-fragment element j (int4)
+__host__ __device__ constexpr int nibble_slot(int j) { return (j >> 1) | ((j & 1) << 2); }
+
+// compile-time sizes of an item block (G = group size; ignored for bf16)
+__host__ __device__ constexpr uint32_t gu_w_bytes_of(int wtype) {
+    return (uint32_t)(slice_rows(wtype) / 8) * KSTEPS * 32 * frag_bytes(wtype);
+}
+__host__ __device__ constexpr uint32_t gu_s_bytes_of(int wtype, int G) {
+    return is_quant(wtype) ? (uint32_t)(slice_rows(wtype) / 8) * (H / G) * 16 * 4 : 0u;
+}
+__host__ __device__ constexpr uint32_t d_w_bytes_of() { return (uint32_t)OTILES * 32 * 8; }
+__host__ __device__ constexpr uint32_t blk_bytes_of(int wtype, int G) {
+    return gu_w_bytes_of(wtype) + gu_s_bytes_of(wtype, G) + d_w_bytes_of();
+}
 
 struct ItemGeom {
     int wtype, group, S, inter, slices;
@@ -52,9 +78,9 @@ __host__ __device__ inline ItemGeom make_geom(int wtype, int group, int inter) {
     g.S = slice_rows(wtype);
     g.inter = inter;
     g.slices = inter / g.S;
-    g.gu_w_bytes = (uint32_t)(g.S / 2) * UNITS * 4 * unit_row_bytes(wtype);
-    g.gu_s_bytes = is_quant(wtype) ? (uint32_t)(g.S / 2) * (H / group) * 4 * 4 : 0u;
-    g.d_w_bytes = (uint32_t)H * 16;
+    g.gu_w_bytes = gu_w_bytes_of(wtype);
+    g.gu_s_bytes = is_quant(wtype) ? gu_s_bytes_of(wtype, group) : 0u;
+    g.d_w_bytes = d_w_bytes_of();
     uint32_t raw = g.gu_w_bytes + g.gu_s_bytes + g.d_w_bytes;
     g.item_bytes = (raw + 127u) & ~127u;
     g.dscale_expert_floats = is_quant(wtype) ? (uint32_t)(inter / group) * H : 0u;
@@ -75,13 +101,12 @@ struct LayerView {
 // Workspace layout (bytes from the workspace base).  Control words first; they are
 // zero on entry and every forward returns them to zero.
 // ---------------------------------------------------------------------------------------
-constexpr int ROUTER_KSPLIT = 5;          // 1280 = 5 x 256 input columns per router CTA
+constexpr int ROUTER_KSPLIT = 8;          // 1280 = 8 x 160 input columns: one CTA each of a cluster
 constexpr int ROUTER_TB = 8;              // tokens per router CTA
 constexpr int MAX_TB = (FOCR_T_MAX + ROUTER_TB - 1) / ROUTER_TB;
 
 struct WsLayout {
     size_t ctrl;          // int32 [MAX_TB tickets][1 global ticket][1 error word][pad]
-    size_t partial;       // f64 [KSPLIT][T_max][64]
     size_t logits;        // f32 [T_max][64]
     size_t topk_idx;      // i32 [T_max][6]
     size_t topk_w;        // f32 [T_max][6]
@@ -98,7 +123,6 @@ constexpr WsLayout ws_layout(int T_max) {
     WsLayout w{};
     size_t o = 0;
     w.ctrl = o;      o = align_up(o + sizeof(int32_t) * (MAX_TB + 64), 256);
-    w.partial = o;   o = align_up(o + sizeof(double) * ROUTER_KSPLIT * (size_t)T_max * E, 256);
     w.logits = o;    o = align_up(o + sizeof(float) * (size_t)T_max * E, 256);
     w.topk_idx = o;  o = align_up(o + sizeof(int32_t) * (size_t)T_max * K, 256);
     w.topk_w = o;    o = align_up(o + sizeof(float) * (size_t)T_max * K, 256);
@@ -116,7 +140,6 @@ constexpr int CTRL_ERROR = MAX_TB + 1;
 
 struct RouteView {   // device pointers into the workspace
     int32_t* ctrl;
-    double* partial;
     float* logits;
     int32_t* topk_idx;
     float* topk_w;
@@ -129,7 +152,7 @@ struct RouteView {   // device pointers into the workspace
 inline RouteView route_view(void* ws, int T_max) {
     WsLayout L = ws_layout(T_max);
     char* b = (char*)ws;
-    return RouteView{(int32_t*)(b + L.ctrl), (double*)(b + L.partial), (float*)(b + L.logits),
+    return RouteView{(int32_t*)(b + L.ctrl), (float*)(b + L.logits),
                      (int32_t*)(b + L.topk_idx), (float*)(b + L.topk_w), (int32_t*)(b + L.counts),
                      (int32_t*)(b + L.offsets), (int32_t*)(b + L.active), (int32_t*)(b + L.perm)};
 }
@@ -191,12 +214,25 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// try_wait that may suspend the thread for up to `hint_ns` while the phase is pending
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete; give up after ~limit_ns.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
         if (globaltimer_ns() - t0 > limit_ns) return false;
     }
 }
@@ -209,6 +245,11 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         "%4;" ::"r"(smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
+}
+
+// Bulk prefetch of global memory into L2 (no shared memory involved).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ uint64_t policy_evict_first() {

@@ -27,7 +27,7 @@ namespace {
 
 constexpr WsLayout kNoallocLayout = ws_layout(FOCR_NOALLOC_T_MAX);
 static_assert(kNoallocLayout.total == FOCR_NOALLOC_SCRATCH_BYTES, "header constant out of date");
-constexpr size_t kCtrlBytes = kNoallocLayout.partial;   // control words sit before the partials
+constexpr size_t kCtrlBytes = kNoallocLayout.logits;    // control words sit before the logits
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FOCR_NOALLOC_SCRATCH_BYTES];
 

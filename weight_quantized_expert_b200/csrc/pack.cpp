@@ -74,31 +74,53 @@ Quantised quantise(const float* w, int64_t rows, int64_t cols, int wtype, int gr
     return out;
 }
 
-// write the 8 input columns [c, c+8) of one row in the unit encoding of `wtype`
-void put_unit(const Quantised& m, int wtype, int64_t cols, int64_t row, int64_t c, uint8_t* dst) {
-    if (wtype == FOCR_W_INT4) {
-        const int8_t* q = m.q.data() + row * cols + c;
-        for (int b = 0; b < 4; ++b)
-            dst[b] = (uint8_t)(((q[2 * b] + 8) & 0xF) | (((q[2 * b + 1] + 8) & 0xF) << 4));
-    } else if (wtype == FOCR_W_INT8) {
-        const int8_t* q = m.q.data() + row * cols + c;
-        for (int b = 0; b < 8; ++b) dst[b] = (uint8_t)(q[b] + 128);
-    } else {
-        std::memcpy(dst, m.b.data() + row * cols + c, 16);
-    }
+// Where every code of one item lives.  `fn(matrix, row, col, byte_offset, nibble_slot)` is
+// called once per weight of the item: matrix 0 gate / 1 up / 2 down (row, col in that
+// matrix), byte_offset from the item block start, nibble_slot in 0..7 (int4) or -1.
+template <class Fn>
+void visit_item(const ItemGeom& g, int slice, Fn&& fn) {
+    const int wt = g.wtype;
+    const int fb = frag_bytes(wt), kpv = ksteps_per_vec(wt);
+    const int i0 = slice * g.S;
+    for (int t = 0; t < g.S / 8; ++t)
+        for (int q = 0; q < KSTEPS; ++q)
+            for (int L = 0; L < 32; ++L) {
+                const int gr = L >> 2, c = L & 3;
+                const size_t vec = ((size_t)(t * (KSTEPS / kpv) + q / kpv) * 32 + L) * 16 + (q % kpv) * fb;
+                for (int j = 0; j < 8; ++j) {
+                    const int trow = gr + 8 * ((j >> 1) & 1);
+                    const int col = 16 * q + 2 * c + (j & 1) + 8 * (j >> 2);
+                    const int mat = trow < 8 ? 0 : 1;
+                    const int row = i0 + 8 * t + (trow & 7);
+                    if (wt == FOCR_W_INT4) fn(mat, row, col, vec, nibble_slot(j));
+                    else if (wt == FOCR_W_INT8) fn(mat, row, col, vec + j, -1);
+                    else fn(mat, row, col, vec + 2 * j, -1);
+                }
+            }
+    const size_t d0 = g.gu_w_bytes + g.gu_s_bytes;
+    for (int m = 0; m < OTILES; ++m)
+        for (int L = 0; L < 32; ++L) {
+            const int gr = L >> 2, c = L & 3;
+            const size_t base = d0 + ((size_t)m * 32 + L) * 8;
+            if (wt == FOCR_W_BF16) {
+                for (int j = 0; j < 4; ++j)
+                    fn(2, 16 * m + gr + 8 * (j >> 1), i0 + 2 * c + (j & 1), base + 2 * j, -1);
+            } else {
+                const int nq = wt == FOCR_W_INT4 ? 2 : 1;
+                for (int q = 0; q < nq; ++q)
+                    for (int j = 0; j < 8; ++j) {
+                        const int row = 16 * m + gr + 8 * ((j >> 1) & 1);
+                        const int col = i0 + 16 * q + 2 * c + (j & 1) + 8 * (j >> 2);
+                        if (wt == FOCR_W_INT4) fn(2, row, col, base + 4 * q, nibble_slot(j));
+                        else fn(2, row, col, base + j, -1);
+                    }
+            }
+        }
 }
 
-void get_unit(int wtype, const uint8_t* src, int8_t* q8, uint16_t* b16) {
-    if (wtype == FOCR_W_INT4) {
-        for (int b = 0; b < 4; ++b) {
-            q8[2 * b] = (int8_t)((src[b] & 0xF) - 8);
-            q8[2 * b + 1] = (int8_t)((src[b] >> 4) - 8);
-        }
-    } else if (wtype == FOCR_W_INT8) {
-        for (int b = 0; b < 8; ++b) q8[b] = (int8_t)((int)src[b] - 128);
-    } else {
-        std::memcpy(b16, src, 16);
-    }
+// GU scale slot of (tile t, group gi, tile-row gr, matrix 0 gate / 1 up), in floats.
+inline size_t gu_scale_index(int ngk, int t, int gi, int gr, int mat) {
+    return ((size_t)(t * ngk + gi) * 8 + gr) * 2 + mat;
 }
 
 }  // namespace
@@ -110,35 +132,37 @@ void host_pack_set(const float* gate, const float* up, const float* down, const 
     const Quantised qg = quantise(gate, g.inter, H, wt, g.group);
     const Quantised qu = quantise(up, g.inter, H, wt, g.group);
     const Quantised qd = quantise(down, H, g.inter, wt, g.group);
-    const int ub = unit_row_bytes(wt);
+    const Quantised* m3[3] = {&qg, &qu, &qd};
+    const int64_t cols3[3] = {H, H, g.inter};
     const int ngk = is_quant(wt) ? H / g.group : 0;
     for (int sl = 0; sl < g.slices; ++sl) {
         uint8_t* blk = items + (size_t)sl * g.item_bytes;
         std::memset(blk, 0, g.item_bytes);
-        const int i0 = sl * g.S;
-        for (int quad = 0; quad < g.S / 2; ++quad) {
-            for (int u = 0; u < UNITS; ++u) {
-                for (int r = 0; r < 4; ++r) {
-                    const Quantised& m = (r < 2) ? qg : qu;
-                    const int64_t row = i0 + 2 * quad + (r & 1);
-                    put_unit(m, wt, H, row, 8 * u, blk + ((size_t)(quad * UNITS + u) * 4 + r) * ub);
-                }
+        visit_item(g, sl, [&](int mat, int row, int col, size_t off, int slot) {
+            const Quantised& m = *m3[mat];
+            const size_t e = (size_t)row * cols3[mat] + col;
+            if (wt == FOCR_W_INT4) {
+                const uint32_t code = (uint32_t)((m.q[e] + 8) & 0xF);
+                uint32_t w;
+                std::memcpy(&w, blk + off, 4);
+                w |= code << (4 * slot);
+                std::memcpy(blk + off, &w, 4);
+            } else if (wt == FOCR_W_INT8) {
+                blk[off] = (uint8_t)(m.q[e] + 128);
+            } else {
+                std::memcpy(blk + off, &m.b[e], 2);
             }
-            if (is_quant(wt)) {
-                float* sc = (float*)(blk + g.gu_w_bytes) + (size_t)quad * ngk * 4;
-                for (int grp = 0; grp < ngk; ++grp)
-                    for (int r = 0; r < 4; ++r) {
-                        const Quantised& m = (r < 2) ? qg : qu;
-                        const int64_t row = i0 + 2 * quad + (r & 1);
-                        sc[grp * 4 + r] = m.s[(size_t)(row * m.ng + grp)];
+        });
+        if (is_quant(wt)) {
+            float* sc = reinterpret_cast<float*>(blk + g.gu_w_bytes);
+            const int i0 = sl * g.S;
+            for (int t = 0; t < g.S / 8; ++t)
+                for (int gi = 0; gi < ngk; ++gi)
+                    for (int gr = 0; gr < 8; ++gr) {
+                        const int64_t row = i0 + 8 * t + gr;
+                        sc[gu_scale_index(ngk, t, gi, gr, 0)] = qg.s[(size_t)(row * qg.ng + gi)];
+                        sc[gu_scale_index(ngk, t, gi, gr, 1)] = qu.s[(size_t)(row * qu.ng + gi)];
                     }
-            }
-        }
-        uint8_t* dw = blk + g.gu_w_bytes + g.gu_s_bytes;
-        for (int h = 0; h < H; ++h) {
-            uint8_t* dst = dw + (size_t)h * 16;
-            // the row slice down[h, i0 : i0 + S] is S codes = 16 bytes in every format
-            for (int c = 0; c < g.S; c += 8) put_unit(qd, wt, g.inter, h, i0 + c, dst + (c / 8) * ub);
         }
     }
     if (is_quant(wt)) {
@@ -152,40 +176,30 @@ void host_pack_set(const float* gate, const float* up, const float* down, const 
 void host_unpack_matrix(const uint8_t* items, const float* dscale, const ItemGeom& g, int which, int8_t* q,
                         uint16_t* b16, float* s) {
     const int wt = g.wtype;
-    const int ub = unit_row_bytes(wt);
     const int ngk = is_quant(wt) ? H / g.group : 0;
-    int8_t q8[8];
-    uint16_t bb[8];
+    const int64_t cols = which == 2 ? g.inter : H;
     for (int sl = 0; sl < g.slices; ++sl) {
         const uint8_t* blk = items + (size_t)sl * g.item_bytes;
-        const int i0 = sl * g.S;
-        if (which < 2) {
-            for (int quad = 0; quad < g.S / 2; ++quad)
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int r = which * 2 + rr;
-                    const int64_t row = i0 + 2 * quad + rr;
-                    for (int u = 0; u < UNITS; ++u) {
-                        get_unit(wt, blk + ((size_t)(quad * UNITS + u) * 4 + r) * ub, q8, bb);
-                        for (int j = 0; j < 8; ++j) {
-                            if (is_quant(wt)) q[row * H + 8 * u + j] = q8[j];
-                            else b16[row * H + 8 * u + j] = bb[j];
-                        }
-                    }
-                    if (is_quant(wt)) {
-                        const float* sc = (const float*)(blk + g.gu_w_bytes) + (size_t)quad * ngk * 4;
-                        for (int grp = 0; grp < ngk; ++grp) s[row * ngk + grp] = sc[grp * 4 + r];
-                    }
-                }
-        } else {
-            const uint8_t* dw = blk + g.gu_w_bytes + g.gu_s_bytes;
-            for (int h = 0; h < H; ++h)
-                for (int c = 0; c < g.S; c += 8) {
-                    get_unit(wt, dw + (size_t)h * 16 + (c / 8) * ub, q8, bb);
-                    for (int j = 0; j < 8; ++j) {
-                        if (is_quant(wt)) q[(int64_t)h * g.inter + i0 + c + j] = q8[j];
-                        else b16[(int64_t)h * g.inter + i0 + c + j] = bb[j];
-                    }
-                }
+        visit_item(g, sl, [&](int mat, int row, int col, size_t off, int slot) {
+            if (mat != which) return;
+            const size_t e = (size_t)row * cols + col;
+            if (wt == FOCR_W_INT4) {
+                uint32_t w;
+                std::memcpy(&w, blk + off, 4);
+                q[e] = (int8_t)((int)((w >> (4 * slot)) & 0xF) - 8);
+            } else if (wt == FOCR_W_INT8) {
+                q[e] = (int8_t)((int)blk[off] - 128);
+            } else {
+                std::memcpy(&b16[e], blk + off, 2);
+            }
+        });
+        if (which < 2 && is_quant(wt)) {
+            const float* sc = reinterpret_cast<const float*>(blk + g.gu_w_bytes);
+            const int i0 = sl * g.S;
+            for (int t = 0; t < g.S / 8; ++t)
+                for (int gi = 0; gi < ngk; ++gi)
+                    for (int gr = 0; gr < 8; ++gr)
+                        s[(int64_t)(i0 + 8 * t + gr) * ngk + gi] = sc[gu_scale_index(ngk, t, gi, gr, which)];
         }
     }
     if (which == 2 && is_quant(wt)) {

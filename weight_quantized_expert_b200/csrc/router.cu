@@ -9,18 +9,27 @@
 // so logits are accumulated in fp64 and rounded once to fp32; experts are ranked by
 // (fp32 logit descending, index ascending).  Softmax is evaluated in fp32.
 //
-// Grid: (ceil(T / 8) token blocks) x (5 column blocks of 256).  Each CTA writes fp64
-// partial logits; the last CTA of a token block (atomic ticket) sums the five
-// partials in a fixed order, runs softmax + top-6 for its 8 tokens (one warp per
-// token), and the last token block to finish performs the dispatch.  Tickets are
-// reset by the CTAs that consume them, so the workspace control words end at zero.
+// Grid: one thread-block cluster of 8 CTAs per block of TB <= 8 tokens.  CTA r of a
+// cluster computes fp64 partial logits over input columns [160 r, 160 r + 160) and
+// writes them into CTA 0's shared memory (distributed shared memory); after one
+// cluster barrier CTA 0 sums the eight partials in a fixed order, runs softmax + top-6
+// (one warp per token) and, when the batch has a single token block, the dispatch
+// straight from shared memory.  With several token blocks each cluster publishes its
+// top-6 and the last one to finish (atomic ticket, reset after use) does the dispatch.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace focr {
 namespace {
 
 constexpr int RT_THREADS = 256;
-constexpr int KCOLS = H / ROUTER_KSPLIT;  // 256
+constexpr int RC = ROUTER_KSPLIT;         // CTAs per cluster
+constexpr int KCOLS = H / RC;             // 160 columns per CTA
+constexpr int PART_COLS = KCOLS / 4;      // 40 columns per thread
+constexpr int NVEC = PART_COLS / 8;       // 5 vectors of 8 bf16
 
 struct RouterParams {
     const float* x;
@@ -42,141 +51,43 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i) {
     }
 }
 
-__global__ void __launch_bounds__(RT_THREADS) router_kernel(RouterParams p) {
-    pdl_wait();                 // inputs may come from the previous kernel on the stream
-    pdl_launch_dependents();    // let the expert kernel start its routing-free work
-
-    __shared__ float xs[ROUTER_TB][KCOLS];
-    __shared__ float lg[ROUTER_TB][E];
-    __shared__ int flag;
-    __shared__ int cnt[E];
-    __shared__ int cursor[E];
-    __shared__ int wc[RT_THREADS / 32][E];
-
-    const int tid = threadIdx.x;
-    const int tb = blockIdx.x, kb = blockIdx.y;
-    const int t0 = tb * ROUTER_TB;
-    const int nt = min(ROUTER_TB, p.T - t0);
-    const int k0 = kb * KCOLS;
-
-    // zero the layer output (the expert kernel adds into it after this grid completes)
-    {
-        const int nblk = gridDim.x * gridDim.y;
-        const int b = blockIdx.y * gridDim.x + blockIdx.x;
-        float4* o4 = reinterpret_cast<float4*>(p.out);
-        const int n4 = p.T * H / 4;
-        for (int i = b * RT_THREADS + tid; i < n4; i += nblk * RT_THREADS) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-
-    for (int i = tid; i < ROUTER_TB * KCOLS / 4; i += RT_THREADS) {
-        const int t = i / (KCOLS / 4), c = (i % (KCOLS / 4)) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (t < nt) v = *reinterpret_cast<const float4*>(p.x + (size_t)(t0 + t) * H + k0 + c);
-        *reinterpret_cast<float4*>(&xs[t][c]) = v;
-    }
-    __syncthreads();
-
-    // thread -> (expert e, quarter of the 256 columns)
-    const int e = tid >> 2, part = tid & 3;
-    double acc[ROUTER_TB];
-#pragma unroll
-    for (int t = 0; t < ROUTER_TB; ++t) acc[t] = 0.0;
-    const uint16_t* wrow = p.wr + (size_t)e * H + k0 + part * 64;
-#pragma unroll 2
-    for (int c = 0; c < 64; c += 8) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(wrow + c);
-        float w[8];
-        bf16x2_to_f32(wv.x, w[0], w[1]);
-        bf16x2_to_f32(wv.y, w[2], w[3]);
-        bf16x2_to_f32(wv.z, w[4], w[5]);
-        bf16x2_to_f32(wv.w, w[6], w[7]);
-#pragma unroll
-        for (int t = 0; t < ROUTER_TB; ++t)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[t] = fma((double)xs[t][part * 64 + c + j], (double)w[j], acc[t]);
-    }
-#pragma unroll
-    for (int t = 0; t < ROUTER_TB; ++t) {
-        acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 1);
-        acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 2);
-    }
-    if (part == 0)
-        for (int t = 0; t < nt; ++t) p.R.partial[((size_t)kb * p.T + t0 + t) * E + e] = acc[t];
-
-    // ---- last column block of this token block: logits, softmax, top-6
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) flag = (atomicAdd(&p.R.ctrl[tb], 1) == ROUTER_KSPLIT - 1);
-    __syncthreads();
-    if (!flag) return;
-    __threadfence();
-    for (int i = tid; i < ROUTER_TB * E; i += RT_THREADS) {
-        const int t = i / E, ee = i % E;
-        if (t < nt) {
-            double s = 0.0;
-            for (int b = 0; b < ROUTER_KSPLIT; ++b)
-                s += __ldcg(&p.R.partial[((size_t)b * p.T + t0 + t) * E + ee]);
-            const float l = (float)s;
-            lg[t][ee] = l;
-            p.R.logits[(size_t)(t0 + t) * E + ee] = l;
-        }
-    }
-    if (tid == 0) p.R.ctrl[tb] = 0;
-    __syncthreads();
-
-    const int warp = tid >> 5, lane = tid & 31;
-    if (warp < nt) {
-        const int t = warp;
-        float v0 = lg[t][lane], v1 = lg[t][lane + 32];
-        // softmax denominator (fp32), max over 64
-        float m = fmaxf(v0, v1);
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float den = expf(v0 - m) + expf(v1 - m);
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-        bool taken0 = false, taken1 = false;
-        for (int j = 0; j < K; ++j) {
-            // best remaining candidate of this lane (lower index first on ties)
-            float cv = -INFINITY;
-            int ci = 0x7fffffff;
-            if (!taken0) { cv = v0; ci = lane; }
-            if (!taken1 && (v1 > cv || (v1 == cv && lane + 32 < ci))) { cv = v1; ci = lane + 32; }
-            warp_argmax(cv, ci);
-            if (ci == lane) taken0 = true;
-            if (ci == lane + 32) taken1 = true;
-            if (lane == 0) {
-                p.R.topk_idx[(size_t)(t0 + t) * K + j] = ci;
-                p.R.topk_w[(size_t)(t0 + t) * K + j] = expf(cv - m) / den;
-            }
-        }
-    }
-
-    // ---- last token block overall: dispatch
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) flag = (atomicAdd(&p.R.ctrl[CTRL_GLOBAL_TICKET], 1) == (int)gridDim.x - 1);
-    __syncthreads();
-    if (!flag) return;
-    __threadfence();
-
+// counts / offsets / active list / stable permutation of the T*6 entries (idx: shared or global)
+template <bool FROM_SMEM>
+__device__ void dispatch(const RouterParams& p, const int* sidx, int* cnt, int* cursor, int (*wc)[E]) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = p.T * K;
     if (tid < E) cnt[tid] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += RT_THREADS) atomicAdd(&cnt[__ldcg(&p.R.topk_idx[i])], 1);
+    for (int i = tid; i < n; i += RT_THREADS) atomicAdd(&cnt[FROM_SMEM ? sidx[i] : __ldcg(&p.R.topk_idx[i])], 1);
     __syncthreads();
-    if (tid == 0) {
-        int run = 0, u = 0;
-        for (int ee = 0; ee < E; ++ee) {
-            p.R.counts[ee] = cnt[ee];
-            p.R.offsets[ee] = run;
-            cursor[ee] = run;
-            if (cnt[ee] > 0) p.R.active[u++] = ee;
-            run += cnt[ee];
+    if (warp == 0) {
+        // 64 experts, two per lane: exclusive scan and compaction of the experts with tokens
+        const int c0 = cnt[2 * lane], c1 = cnt[2 * lane + 1];
+        int incl = c0 + c1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
         }
-        p.R.offsets[E] = run;
-        p.R.active[E] = u;
-        p.R.ctrl[CTRL_GLOBAL_TICKET] = 0;
+        const int ex0 = incl - c0 - c1;
+        p.R.counts[2 * lane] = c0;
+        p.R.counts[2 * lane + 1] = c1;
+        p.R.offsets[2 * lane] = ex0;
+        p.R.offsets[2 * lane + 1] = ex0 + c0;
+        cursor[2 * lane] = ex0;
+        cursor[2 * lane + 1] = ex0 + c0;
+        if (lane == 31) p.R.offsets[E] = incl;
+        const int h0 = c0 > 0, h1 = c1 > 0;
+        int hincl = h0 + h1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, hincl, o);
+            if (lane >= o) hincl += v;
+        }
+        int pos = hincl - h0 - h1;
+        if (h0) p.R.active[pos++] = 2 * lane;
+        if (h1) p.R.active[pos] = 2 * lane + 1;
+        if (lane == 31) p.R.active[E] = hincl;
     }
     __syncthreads();
     // stable scatter in chunks of 256 entries: rank = cursor + earlier warps + earlier lanes
@@ -184,7 +95,7 @@ __global__ void __launch_bounds__(RT_THREADS) router_kernel(RouterParams p) {
         for (int i = tid; i < (RT_THREADS / 32) * E; i += RT_THREADS) (&wc[0][0])[i] = 0;
         __syncthreads();
         const int i = base + tid;
-        const int ee = i < n ? __ldcg(&p.R.topk_idx[i]) : -1;
+        const int ee = i < n ? (FROM_SMEM ? sidx[i] : __ldcg(&p.R.topk_idx[i])) : -1;
         const unsigned same = __match_any_sync(0xffffffffu, ee);
         const unsigned lower = same & ((1u << lane) - 1u);
         if (ee >= 0 && lower == 0) wc[warp][ee] = __popc(same);
@@ -204,13 +115,147 @@ __global__ void __launch_bounds__(RT_THREADS) router_kernel(RouterParams p) {
     }
 }
 
+template <int TB>
+__global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_kernel(RouterParams p) {
+    cg::cluster_group cluster = cg::this_cluster();
+    __shared__ double part_s[RC][TB][E];     // filled in CTA 0 by all CTAs of the cluster
+    __shared__ double xs[TB][KCOLS];
+    __shared__ float lg[TB][E];
+    __shared__ int sidx[TB * K];
+    __shared__ int flag;
+    __shared__ int cnt[E];
+    __shared__ int cursor[E];
+    __shared__ int wc[RT_THREADS / 32][E];
+
+    const int tid = threadIdx.x;
+    const int r = (int)cluster.block_rank();
+    const int tb = blockIdx.x / RC;
+    const int t0 = tb * TB;
+    const int nt = min(TB, p.T - t0);
+    const int k0 = r * KCOLS;
+
+    // router weights are layer constants: fetch them before waiting on the previous kernel
+    const int e = tid >> 2, part = tid & 3;
+    const uint16_t* wrow = p.wr + (size_t)e * H + k0 + part * PART_COLS;
+    uint4 wv[NVEC];
+#pragma unroll
+    for (int v = 0; v < NVEC; ++v) wv[v] = __ldg(reinterpret_cast<const uint4*>(wrow + 8 * v));
+
+    pdl_wait();                 // x may come from the previous kernel on the stream
+    pdl_launch_dependents();    // let the expert kernel start its routing-free work
+
+    // zero the layer output (the expert kernel adds into it after this grid completes)
+    {
+        const int nblk = gridDim.x;
+        float4* o4 = reinterpret_cast<float4*>(p.out);
+        const int n4 = p.T * H / 4;
+        for (int i = blockIdx.x * RT_THREADS + tid; i < n4; i += nblk * RT_THREADS)
+            o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+
+    for (int i = tid; i < TB * KCOLS; i += RT_THREADS) {
+        const int t = i / KCOLS, c = i % KCOLS;
+        xs[t][c] = t < nt ? (double)p.x[(size_t)(t0 + t) * H + k0 + c] : 0.0;
+    }
+    __syncthreads();
+
+    // thread -> (expert e, quarter of the CTA's columns); products are exact in fp64
+    double acc[TB];
+#pragma unroll
+    for (int t = 0; t < TB; ++t) acc[t] = 0.0;
+#pragma unroll
+    for (int v = 0; v < NVEC; ++v) {
+        float w[8];
+        bf16x2_to_f32(wv[v].x, w[0], w[1]);
+        bf16x2_to_f32(wv[v].y, w[2], w[3]);
+        bf16x2_to_f32(wv[v].z, w[4], w[5]);
+        bf16x2_to_f32(wv[v].w, w[6], w[7]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const double wd = (double)w[j];
+#pragma unroll
+            for (int t = 0; t < TB; ++t) acc[t] = fma(xs[t][part * PART_COLS + 8 * v + j], wd, acc[t]);
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < TB; ++t) {
+        acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 1);
+        acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 2);
+    }
+    if (part == 0) {
+        double* dst = cluster.map_shared_rank(&part_s[r][0][0], 0);
+#pragma unroll
+        for (int t = 0; t < TB; ++t) dst[t * E + e] = acc[t];
+    }
+    cluster.sync();            // partials of all eight CTAs are in CTA 0
+    if (r != 0) return;
+
+    // ---- CTA 0: logits (fixed summation order), softmax, top-6
+    for (int i = tid; i < TB * E; i += RT_THREADS) {
+        const int t = i / E, ee = i % E;
+        if (t < nt) {
+            double s = 0.0;
+#pragma unroll
+            for (int b = 0; b < RC; ++b) s += part_s[b][t][ee];
+            const float l = (float)s;
+            lg[t][ee] = l;
+            p.R.logits[(size_t)(t0 + t) * E + ee] = l;
+        }
+    }
+    __syncthreads();
+
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp < nt) {
+        const int t = warp;
+        const float v0 = lg[t][lane], v1 = lg[t][lane + 32];
+        float m = fmaxf(v0, v1);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float den = expf(v0 - m) + expf(v1 - m);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        bool taken0 = false, taken1 = false;
+        for (int j = 0; j < K; ++j) {
+            // best remaining candidate of this lane (lower index first on ties)
+            float cv = -INFINITY;
+            int ci = 0x7fffffff;
+            if (!taken0) { cv = v0; ci = lane; }
+            if (!taken1 && (v1 > cv || (v1 == cv && lane + 32 < ci))) { cv = v1; ci = lane + 32; }
+            warp_argmax(cv, ci);
+            if (ci == lane) taken0 = true;
+            if (ci == lane + 32) taken1 = true;
+            if (lane == 0) {
+                sidx[t * K + j] = ci;
+                p.R.topk_idx[(size_t)(t0 + t) * K + j] = ci;
+                p.R.topk_w[(size_t)(t0 + t) * K + j] = expf(cv - m) / den;
+            }
+        }
+    }
+    __syncthreads();
+
+    if (gridDim.x == RC) {     // one token block: dispatch from shared memory
+        dispatch<true>(p, sidx, cnt, cursor, wc);
+        return;
+    }
+    // ---- several token blocks: the last one to finish dispatches
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) flag = (atomicAdd(&p.R.ctrl[CTRL_GLOBAL_TICKET], 1) == (int)(gridDim.x / RC) - 1);
+    __syncthreads();
+    if (!flag) return;
+    __threadfence();
+    if (tid == 0) p.R.ctrl[CTRL_GLOBAL_TICKET] = 0;
+    dispatch<false>(p, sidx, cnt, cursor, wc);
+}
+
 }  // namespace
 
 cudaError_t launch_router(const float* x, int T, int /*T_ws*/, const LayerView& L, const RouteView& R, float* out,
                           cudaStream_t st) {
     RouterParams p{x, T, L.router, R, out};
+    const int TB = T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : 8));
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((T + ROUTER_TB - 1) / ROUTER_TB, ROUTER_KSPLIT);
+    cfg.gridDim = dim3(((T + TB - 1) / TB) * RC);
     cfg.blockDim = dim3(RT_THREADS);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
@@ -219,7 +264,12 @@ cudaError_t launch_router(const float* x, int T, int /*T_ws*/, const LayerView& 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, router_kernel, p);
+    switch (TB) {
+        case 1: return cudaLaunchKernelEx(&cfg, router_kernel<1>, p);
+        case 2: return cudaLaunchKernelEx(&cfg, router_kernel<2>, p);
+        case 4: return cudaLaunchKernelEx(&cfg, router_kernel<4>, p);
+        default: return cudaLaunchKernelEx(&cfg, router_kernel<8>, p);
+    }
 }
 
 }  // namespace focr
