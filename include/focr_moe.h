@@ -130,13 +130,20 @@ focr_status focr_moe_export_quantized(const focr_moe_layer* layer, int32_t matri
 /* Workspace a forward call with up to T_max tokens needs (bytes). */
 size_t focr_moe_workspace_bytes(int32_t T_max);
 
+/* Length of the workspace prefix (control words, k-split partial sums and their arrival
+ * counters) that must be zero when a forward starts and that every forward leaves zero.
+ * It does not depend on T_max.  Zeroing these bytes makes a workspace usable again after
+ * focr_moe_check reported a device error. */
+size_t focr_moe_workspace_zero_bytes(void);
+
 /*
  * focr_moe_layer_forward -- out[T, 1280] = MoE(hidden[T, 1280]).
  *   hidden, out : DEVICE fp32, 16-byte aligned, caller-owned; must not overlap.
  *   1 <= T <= FOCR_T_MAX.
  *   workspace   : DEVICE scratch of ws_bytes >= focr_moe_workspace_bytes(T), 256-byte
  *                 aligned.  It must be zero-filled before its first use; every forward
- *                 leaves its control words zero again.  Calls that share a workspace
+ *                 leaves its first focr_moe_workspace_zero_bytes() bytes zero again, so
+ *                 calls with different T may share it.  Calls that share a workspace
  *                 must be ordered on one stream.
  *   dbg         : optional routing outputs (NULL for none).
  * Steps, all on `stream`: router GEMV (fp64 accumulation of exact products,
@@ -169,9 +176,42 @@ focr_status focr_moe_layer_forward(const focr_moe_layer* layer, const float* hid
  *   - A device wait that runs out is cleared by the next call rather than reported.
  */
 #define FOCR_NOALLOC_T_MAX 320
-#define FOCR_NOALLOC_SCRATCH_BYTES 110592
+#define FOCR_NOALLOC_SCRATCH_BYTES 7332352
 focr_status focr_moe_layer_forward_noalloc(const focr_moe_layer* layer, const float* hidden, int32_t T, float* out,
                                            const focr_moe_route_debug* dbg, void* stream);
+
+/* Flags of the *_ex / dense forwards. */
+#define FOCR_FWD_RESIDUAL 1   /* out = hidden + layer(hidden) instead of layer(hidden) */
+
+/*
+ * focr_moe_layer_forward_ex -- focr_moe_layer_forward with flags (0 or FOCR_FWD_RESIDUAL).
+ * With FOCR_FWD_RESIDUAL the output starts as a copy of `hidden` (the decoder's residual
+ * stream h <- h + MoE(h)); arguments and workspace rules are otherwise the same.
+ */
+focr_status focr_moe_layer_forward_ex(const focr_moe_layer* layer, const float* hidden, int32_t T, float* out,
+                                      void* workspace, size_t ws_bytes, const focr_moe_route_debug* dbg,
+                                      int32_t flags, void* stream);
+
+/*
+ * Dense SwiGLU MLP of decoder layer 0 (frankenocr.pages.dev, "One forward pass", step 6:
+ * layer 0 is a dense SwiGLU MLP): out = D (silu(G x) * (U x)) with G, U [6848, 1280] and
+ * D [1280, 6848] (HOST fp32, [out, in] row-major).  Quantisation as focr_moe_pack_weights
+ * (int8 with group 128 in the decode recipe; 6848 = 53 x 128 + 64, so the last group of
+ * a down row has 64 elements and its own scale).  The forward runs on the grouped expert
+ * kernel as a single always-on weight set.
+ */
+typedef struct focr_dense_mlp focr_dense_mlp;
+focr_status focr_dense_mlp_pack(const float* w_gate, const float* w_up, const float* w_down, int32_t wtype,
+                                int32_t group, focr_dense_mlp** out, void* stream);
+void focr_dense_mlp_free(focr_dense_mlp* mlp);
+/* Canonical codes/scales of matrix 0 (gate), 1 (up) or 2 (down), formats as focr_moe_export_quantized;
+ * codes: rows*cols (int8), rows*cols/2 (int4) or 2*rows*cols (bf16) bytes, scales rows*ceil(cols/g). */
+focr_status focr_dense_mlp_export_quantized(const focr_dense_mlp* mlp, int32_t matrix, void* codes_host,
+                                            size_t code_bytes, float* scales_host, size_t n_scales);
+/* x, out: DEVICE fp32 [T, 1280], 16-byte aligned, not overlapping; workspace as for
+ * focr_moe_layer_forward (focr_moe_workspace_bytes(T)); flags 0 or FOCR_FWD_RESIDUAL. */
+focr_status focr_dense_mlp_forward(const focr_dense_mlp* mlp, const float* x, int32_t T, float* out,
+                                   void* workspace, size_t ws_bytes, int32_t flags, void* stream);
 
 /*
  * focr_moe_check -- read the device error word a forward may have set in `workspace`
@@ -179,6 +219,46 @@ focr_status focr_moe_layer_forward_noalloc(const focr_moe_layer* layer, const fl
  * FOCR_ERR_TIMEOUT, and clears the word.
  */
 focr_status focr_moe_check(void* workspace, void* stream);
+
+/* ------------------------------------------------------------------ decode-step companions
+ * Source: frankenocr.pages.dev, "One forward pass", step 7 -- the final RMSNorm feeds an
+ * lm_head GEMV from 1,280 to 129,280 logits, and greedy decoding picks the argmax;
+ * "Four bits, one shared scale" -- int8 on lm_head.
+ */
+
+typedef struct focr_lm_head focr_lm_head;   /* opaque, device-resident, library-owned */
+
+/*
+ * focr_lm_head_pack -- quantise the lm_head [129280, 1280] (HOST fp32, row-major) to int8
+ * with one scale per row (s = max|w_row| / 127 in fp32, q = round-half-even(w / s)
+ * clamped to [-127, 127]; an all-zero row has s = 0) and lay it out on the device.
+ * Synchronises.
+ */
+focr_status focr_lm_head_pack(const float* w, focr_lm_head** out, void* stream);
+void focr_lm_head_free(focr_lm_head* head);
+
+/* Canonical codes (int8 [129280, 1280] row-major) and row scales (f32 [129280]) to HOST memory. */
+focr_status focr_lm_head_export(const focr_lm_head* head, int8_t* codes_host, float* scales_host);
+
+/* Workspace a focr_lm_head_gemv call with up to T_max tokens needs (bytes). */
+size_t focr_lm_head_workspace_bytes(int32_t T_max);
+
+/*
+ * focr_lm_head_gemv -- logits[t, n] = s_n * sum_k q_nk x[t, k] and argmax[t] (ties to the
+ * lowest row).  x: DEVICE fp32 [T, 1280], 16-byte aligned; logits: DEVICE fp32 [T, 129280]
+ * or NULL; argmax: DEVICE int32 [T].  1 <= T <= FOCR_T_MAX.  workspace: DEVICE, 256-byte
+ * aligned, >= focr_lm_head_workspace_bytes(T), zero-filled before first use (left with its
+ * control word zero).  Asynchronous on `stream`.
+ */
+focr_status focr_lm_head_gemv(const focr_lm_head* head, const float* x, int32_t T, float* logits,
+                              int32_t* argmax, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * focr_rmsnorm -- out[t] = x[t] / sqrt(mean(x[t]^2) + eps) * gamma (gamma NULL: 1).
+ * x, out: DEVICE fp32 [T, 1280], 16-byte aligned (may be the same buffer); gamma: DEVICE
+ * fp32 [1280] or NULL.  Asynchronous on `stream`.
+ */
+focr_status focr_rmsnorm(const float* x, const float* gamma, int32_t T, float eps, float* out, void* stream);
 
 /* Thread-local description of the last error (empty string if none). */
 const char* focr_last_error(void);

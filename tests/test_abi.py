@@ -44,6 +44,9 @@ def test_workspace_size_grows_with_tokens():
     # clamped outside [1, T_MAX]
     assert api.focr_moe_workspace_bytes(0) == sizes[0]
     assert api.focr_moe_workspace_bytes(10 ** 6) == sizes[-1]
+    # the zero-on-entry prefix is the same for every T and lies inside every workspace
+    z = api.focr_moe_workspace_zero_bytes()
+    assert 0 < z < sizes[0] and z % 256 == 0
 
 
 def test_forward_rejects_bad_arguments_without_launching():

@@ -5,6 +5,7 @@ dispatch (counts, offsets, permutation).  Floating point: the layer output withi
 per-token relative error of 2e-3 (max |gpu - oracle| / max |oracle| over the 1280
 outputs of a token; fp32 accumulation), router weights within 1e-5.
 """
+import functools
 import os
 
 import numpy as np
@@ -145,8 +146,35 @@ def test_repeated_calls_reuse_workspace():
     np.testing.assert_array_equal(g1["perm"], g3["perm"])
     assert per_token_rel_err(g3["out"], g1["out"]).max() < 1e-5
     assert_parity(g2, om.forward(x2, nthreads=NTHREADS))
-    # control words back to zero after every forward
-    assert int(ws[:4352].count_nonzero()) == 0
+    # control words, k-split sums and counters back to zero after every forward
+    zb = api.focr_moe_workspace_zero_bytes()
+    assert int(ws[:zb].count_nonzero()) == 0
+    # decode-size calls of different T on the same workspace
+    for T in (1, 8, 3):
+        x = synth.hidden(45 + T, T)
+        assert_parity(run_gpu(packed, x, ws), om.forward(x, nthreads=NTHREADS))
+        assert int(ws[:zb].count_nonzero()) == 0
+
+
+# every weight-type pairing the kernels instantiate beyond the ones above, on the
+# decode path (T <= 8: gate/up kernel + down kernel) and the grouped path (T > 8)
+MIXED = [
+    (W4, W4, 64), (W4, W4, 32), (W4, W8, 128), (W8, WB, 128), (W8, W4, 128),
+    (WB, WB, 128), (WB, W4, 32), (WB, W8, 128),
+]
+
+
+@functools.lru_cache(maxsize=1)   # one mixed layer alive at a time (T varies fastest below)
+def mixed_case(routed, shared, group):
+    return moe_case.__wrapped__(5, routed, shared, group)
+
+
+@pytest.mark.parametrize("T", [3, 12])
+@pytest.mark.parametrize("routed,shared,group", MIXED)
+def test_mixed_weight_types(routed, shared, group, T):
+    om, packed = mixed_case(routed, shared, group)
+    x = synth.hidden(50 + T, T)
+    assert_parity(run_gpu(packed, x), om.forward(x, nthreads=NTHREADS))
 
 
 def test_uniform_router_ties_pick_lowest_experts():

@@ -27,9 +27,14 @@ STATUS = {0: "FOCR_OK", 1: "FOCR_ERR_INVALID_ARG", 2: "FOCR_ERR_UNSUPPORTED", 3:
 # every symbol include/focr_moe.h declares
 EXPORTED = (
     "focr_moe_pack_weights", "focr_moe_layer_clone", "focr_moe_layer_free", "focr_moe_layer_device_bytes",
-    "focr_moe_export_sizes", "focr_moe_export_quantized", "focr_moe_workspace_bytes", "focr_moe_layer_forward",
+    "focr_moe_export_sizes", "focr_moe_export_quantized", "focr_moe_workspace_bytes",
+    "focr_moe_workspace_zero_bytes", "focr_moe_layer_forward",
     "focr_moe_check", "focr_last_error", "focr_version", "focr_moe_layer_forward_noalloc",
+    "focr_moe_layer_forward_ex", "focr_lm_head_pack", "focr_lm_head_free", "focr_lm_head_export",
+    "focr_lm_head_workspace_bytes", "focr_lm_head_gemv", "focr_rmsnorm", "focr_dense_mlp_pack",
+    "focr_dense_mlp_free", "focr_dense_mlp_export_quantized", "focr_dense_mlp_forward",
 )
+FWD_RESIDUAL = 1
 NOALLOC_T_MAX = 320
 
 
@@ -72,9 +77,21 @@ def lib():
                 "focr_moe_export_sizes": (i32, [P, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]),
                 "focr_moe_export_quantized": (i32, [P, i32, i32, P, sz, P, sz]),
                 "focr_moe_workspace_bytes": (sz, [i32]),
+                "focr_moe_workspace_zero_bytes": (sz, []),
                 "focr_moe_layer_forward": (i32, [P, P, i32, P, P, sz, ctypes.POINTER(RouteDebug), P]),
                 "focr_moe_check": (i32, [P, P]),
                 "focr_moe_layer_forward_noalloc": (i32, [P, P, i32, P, ctypes.POINTER(RouteDebug), P]),
+                "focr_moe_layer_forward_ex": (i32, [P, P, i32, P, P, sz, ctypes.POINTER(RouteDebug), i32, P]),
+                "focr_lm_head_pack": (i32, [P, ctypes.POINTER(P), P]),
+                "focr_lm_head_free": (None, [P]),
+                "focr_lm_head_export": (i32, [P, P, P]),
+                "focr_lm_head_workspace_bytes": (sz, [i32]),
+                "focr_lm_head_gemv": (i32, [P, P, i32, P, P, P, sz, P]),
+                "focr_rmsnorm": (i32, [P, P, i32, ctypes.c_float, P, P]),
+                "focr_dense_mlp_pack": (i32, [P, P, P, i32, i32, ctypes.POINTER(P), P]),
+                "focr_dense_mlp_free": (None, [P]),
+                "focr_dense_mlp_export_quantized": (i32, [P, i32, P, sz, P, sz]),
+                "focr_dense_mlp_forward": (i32, [P, P, i32, P, P, sz, i32, P]),
                 "focr_last_error": (ctypes.c_char_p, []),
                 "focr_version": (ctypes.c_char_p, []),
             }
@@ -162,6 +179,11 @@ def focr_moe_workspace_bytes(T_max: int) -> int:
     return int(lib().focr_moe_workspace_bytes(int(T_max)))
 
 
+def focr_moe_workspace_zero_bytes() -> int:
+    """Bytes at the start of a workspace that are zero between forwards."""
+    return int(lib().focr_moe_workspace_zero_bytes())
+
+
 def new_workspace(T_max: int, device="cuda"):
     """A zero-filled workspace tensor for forwards with up to T_max tokens."""
     import torch
@@ -169,7 +191,7 @@ def new_workspace(T_max: int, device="cuda"):
 
 
 def focr_moe_layer_forward(layer: MoELayer, hidden, out=None, workspace=None, debug: dict | None = None,
-                           stream=None):
+                           stream=None, flags: int = 0):
     """out[T, 1280] = MoE(hidden[T, 1280]) on the current (or given) stream.
     `debug`, if given, maps names of focr_moe_route_debug fields to device tensors to fill."""
     import torch
@@ -182,9 +204,10 @@ def focr_moe_layer_forward(layer: MoELayer, hidden, out=None, workspace=None, de
     dbg = None
     if debug:
         dbg = RouteDebug(*[_ptr(debug.get(f)) for f, _ in RouteDebug._fields_])
-    _check(lib().focr_moe_layer_forward(ctypes.c_void_p(layer.handle), _ptr(hidden), T, _ptr(out), _ptr(workspace),
-                                        workspace.numel(), ctypes.byref(dbg) if dbg is not None else None,
-                                        _stream(stream)))
+    _check(lib().focr_moe_layer_forward_ex(ctypes.c_void_p(layer.handle), _ptr(hidden), T, _ptr(out),
+                                           _ptr(workspace), workspace.numel(),
+                                           ctypes.byref(dbg) if dbg is not None else None, int(flags),
+                                           _stream(stream)))
     return out
 
 
@@ -206,3 +229,105 @@ def focr_moe_layer_forward_noalloc(layer: MoELayer, hidden, out=None, debug: dic
 
 def focr_moe_check(workspace, stream=None):
     _check(lib().focr_moe_check(_ptr(workspace), _stream(stream)))
+
+
+# ---------------------------------------------------------------- decode-step companions
+
+class LMHead:
+    """A packed int8 lm_head (owns its device memory)."""
+
+    def __init__(self, handle: int):
+        self.handle = handle
+
+    def __del__(self):
+        h, self.handle = getattr(self, "handle", None), None
+        if h and _lib is not None:
+            _lib.focr_lm_head_free(ctypes.c_void_p(h))
+
+
+def focr_lm_head_pack(w, stream=None) -> LMHead:
+    w = np.ascontiguousarray(w, np.float32)
+    assert w.shape == (VOCAB, H)
+    h = ctypes.c_void_p()
+    _check(lib().focr_lm_head_pack(w.ctypes.data, ctypes.byref(h), _stream(stream)))
+    return LMHead(h.value)
+
+
+def focr_lm_head_export(head: LMHead):
+    codes = np.empty((VOCAB, H), np.int8)
+    scales = np.empty(VOCAB, np.float32)
+    _check(lib().focr_lm_head_export(ctypes.c_void_p(head.handle), codes.ctypes.data, scales.ctypes.data))
+    return codes, scales
+
+
+def focr_lm_head_workspace_bytes(T_max: int) -> int:
+    return int(lib().focr_lm_head_workspace_bytes(int(T_max)))
+
+
+def focr_lm_head_gemv(head: LMHead, x, argmax=None, logits=None, workspace=None, stream=None):
+    """argmax[T] (int32) and optionally logits[T, 129280] of the int8 lm_head."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous() and x.shape[-1] == H
+    T = x.shape[0]
+    if argmax is None:
+        argmax = torch.empty(T, dtype=torch.int32, device=x.device)
+    if workspace is None:
+        workspace = torch.zeros(focr_lm_head_workspace_bytes(T), dtype=torch.uint8, device=x.device)
+    _check(lib().focr_lm_head_gemv(ctypes.c_void_p(head.handle), _ptr(x), T, _ptr(logits), _ptr(argmax),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)))
+    return argmax
+
+
+def focr_rmsnorm(x, gamma=None, eps: float = 1e-6, out=None, stream=None):
+    import torch
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous() and x.shape[-1] == H
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().focr_rmsnorm(_ptr(x), _ptr(gamma), x.shape[0], float(eps), _ptr(out), _stream(stream)))
+    return out
+
+
+class DenseMLP:
+    """A packed dense SwiGLU MLP (decoder layer 0; owns its device memory)."""
+
+    def __init__(self, handle: int, wtype: int, group: int):
+        self.handle, self.wtype, self.group = handle, wtype, group
+
+    def __del__(self):
+        h, self.handle = getattr(self, "handle", None), None
+        if h and _lib is not None:
+            _lib.focr_dense_mlp_free(ctypes.c_void_p(h))
+
+
+def focr_dense_mlp_pack(gate, up, down, wtype: int = W_INT8, group: int = 128, stream=None) -> DenseMLP:
+    arrs = [np.ascontiguousarray(a, np.float32) for a in (gate, up, down)]
+    assert arrs[0].shape == (DENSE_I, H) and arrs[2].shape == (H, DENSE_I)
+    h = ctypes.c_void_p()
+    _check(lib().focr_dense_mlp_pack(arrs[0].ctypes.data, arrs[1].ctypes.data, arrs[2].ctypes.data, int(wtype),
+                                     int(group), ctypes.byref(h), _stream(stream)))
+    return DenseMLP(h.value, wtype, group)
+
+
+def focr_dense_mlp_export_quantized(mlp: DenseMLP, matrix: int):
+    rows, cols = (DENSE_I, H) if matrix < 2 else (H, DENSE_I)
+    n = rows * cols
+    cb = n // 2 if mlp.wtype == W_INT4 else (n if mlp.wtype == W_INT8 else 2 * n)
+    ns = rows * ((cols + mlp.group - 1) // mlp.group) if mlp.wtype != W_BF16 else 0
+    codes = np.empty(cb, np.uint8)
+    scales = np.empty(ns, np.float32)
+    _check(lib().focr_dense_mlp_export_quantized(ctypes.c_void_p(mlp.handle), matrix, codes.ctypes.data, cb,
+                                                 scales.ctypes.data if ns else None, ns))
+    return codes, scales
+
+
+def focr_dense_mlp_forward(mlp: DenseMLP, x, out=None, workspace=None, flags: int = 0, stream=None):
+    import torch
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous() and x.shape[-1] == H
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        workspace = new_workspace(T, x.device)
+    _check(lib().focr_dense_mlp_forward(ctypes.c_void_p(mlp.handle), _ptr(x), T, _ptr(out), _ptr(workspace),
+                                        workspace.numel(), int(flags), _stream(stream)))
+    return out

@@ -7,6 +7,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "lm_head.h"
 #include "pack.h"
 
 using namespace focr;
@@ -275,10 +276,14 @@ size_t focr_moe_workspace_bytes(int32_t T_max) {
     return ws_layout(T_max).total;
 }
 
-focr_status focr_moe_layer_forward(const focr_moe_layer* L, const float* hidden, int32_t T, float* out,
-                                   void* workspace, size_t ws_bytes, const focr_moe_route_debug* dbg, void* stream) {
+size_t focr_moe_workspace_zero_bytes(void) { return ws_layout(1).a16; }
+
+focr_status focr_moe_layer_forward_ex(const focr_moe_layer* L, const float* hidden, int32_t T, float* out,
+                                      void* workspace, size_t ws_bytes, const focr_moe_route_debug* dbg, int32_t flags,
+                                      void* stream) {
     g_err.clear();
     if (!L || !L->dev) return fail(FOCR_ERR_INVALID_ARG, "layer is NULL");
+    if (flags & ~FOCR_FWD_RESIDUAL) return fail(FOCR_ERR_INVALID_ARG, "unknown flags 0x%x", (unsigned)flags);
     if (T < 1 || T > FOCR_T_MAX) return fail(FOCR_ERR_INVALID_ARG, "T=%d outside [1, %d]", T, FOCR_T_MAX);
     if (!hidden || !out || !workspace) return fail(FOCR_ERR_INVALID_ARG, "hidden, out and workspace must not be NULL");
     if (!aligned(hidden, 16) || !aligned(out, 16)) return fail(FOCR_ERR_INVALID_ARG, "hidden/out must be 16-byte aligned");
@@ -294,8 +299,9 @@ focr_status focr_moe_layer_forward(const focr_moe_layer* L, const float* hidden,
     cudaStream_t st = (cudaStream_t)stream;
     const RouteView R = route_view(workspace, T);
     const LayerView V = L->view();
-    CUDA_TRY(launch_router(hidden, T, T, V, R, out, st));
-    CUDA_TRY(launch_expert_decode(hidden, T, V, R, out, st));
+    CUDA_TRY(launch_router(hidden, T, T, V, R, out, (flags & FOCR_FWD_RESIDUAL) ? hidden : nullptr, st));
+    if (T <= SMALL_T) CUDA_TRY(launch_decode_small(hidden, T, V, R, out, false, st));
+    else CUDA_TRY(launch_expert_decode(hidden, T, V, R, out, false, st));
     if (dbg) {
         if (dbg->logits) CUDA_TRY(cudaMemcpyAsync(dbg->logits, R.logits, sizeof(float) * T * E, cudaMemcpyDeviceToDevice, st));
         if (dbg->topk_idx) CUDA_TRY(cudaMemcpyAsync(dbg->topk_idx, R.topk_idx, sizeof(int32_t) * T * K, cudaMemcpyDeviceToDevice, st));
@@ -304,6 +310,225 @@ focr_status focr_moe_layer_forward(const focr_moe_layer* L, const float* hidden,
         if (dbg->offsets) CUDA_TRY(cudaMemcpyAsync(dbg->offsets, R.offsets, sizeof(int32_t) * (E + 1), cudaMemcpyDeviceToDevice, st));
         if (dbg->perm) CUDA_TRY(cudaMemcpyAsync(dbg->perm, R.perm, sizeof(int32_t) * T * K, cudaMemcpyDeviceToDevice, st));
     }
+    return FOCR_OK;
+}
+
+// ------------------------------------------------------------------ lm_head + RMSNorm
+
+struct focr_lm_head {
+    uint8_t* dev = nullptr;   // codes (V * H bytes) then scales (V floats)
+    size_t bytes = 0;
+};
+
+focr_status focr_lm_head_pack(const float* w, focr_lm_head** out, void* stream) {
+    g_err.clear();
+    if (!w || !out) return fail(FOCR_ERR_INVALID_ARG, "w and out must not be NULL");
+    *out = nullptr;
+    const size_t code_bytes = (size_t)FOCR_VOCAB * H, bytes = code_bytes + sizeof(float) * FOCR_VOCAB;
+    std::vector<uint8_t> host;
+    try {
+        host.resize(bytes);
+    } catch (...) {
+        return fail(FOCR_ERR_OOM, "host staging of %zu bytes failed", bytes);
+    }
+    host_pack_lm_head(w, FOCR_VOCAB, host.data(), reinterpret_cast<float*>(host.data() + code_bytes));
+    focr_lm_head* L = new (std::nothrow) focr_lm_head();
+    if (!L) return fail(FOCR_ERR_OOM, "host allocation failed");
+    cudaError_t e = cudaMalloc(&L->dev, bytes);
+    if (e != cudaSuccess) {
+        delete L;
+        return fail(e == cudaErrorMemoryAllocation ? FOCR_ERR_OOM : FOCR_ERR_CUDA, "cudaMalloc(%zu): %s", bytes,
+                    cudaGetErrorString(e));
+    }
+    L->bytes = bytes;
+    cudaStream_t st = (cudaStream_t)stream;
+    e = cudaMemcpyAsync(L->dev, host.data(), bytes, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) {
+        cudaFree(L->dev);
+        delete L;
+        return cuda_fail(e, "upload of packed lm_head");
+    }
+    *out = L;
+    return FOCR_OK;
+}
+
+void focr_lm_head_free(focr_lm_head* L) {
+    if (!L) return;
+    if (L->dev) cudaFree(L->dev);
+    delete L;
+}
+
+focr_status focr_lm_head_export(const focr_lm_head* L, int8_t* codes, float* scales) {
+    g_err.clear();
+    if (!L || !codes || !scales) return fail(FOCR_ERR_INVALID_ARG, "NULL argument");
+    const size_t code_bytes = (size_t)FOCR_VOCAB * H;
+    std::vector<uint8_t> host(code_bytes);
+    CUDA_TRY(cudaMemcpy(host.data(), L->dev, code_bytes, cudaMemcpyDeviceToHost));
+    CUDA_TRY(cudaMemcpy(scales, L->dev + code_bytes, sizeof(float) * FOCR_VOCAB, cudaMemcpyDeviceToHost));
+    host_unpack_lm_head(host.data(), FOCR_VOCAB, codes);
+    return FOCR_OK;
+}
+
+size_t focr_lm_head_workspace_bytes(int32_t T_max) {
+    if (T_max < 1) T_max = 1;
+    if (T_max > FOCR_T_MAX) T_max = FOCR_T_MAX;
+    int grid = 1024;   // upper bound on the CTAs of one launch (one per SM)
+    return align_up(256 + sizeof(unsigned long long) * (size_t)grid * T_max, 256);
+}
+
+focr_status focr_lm_head_gemv(const focr_lm_head* L, const float* x, int32_t T, float* logits, int32_t* argmax,
+                              void* workspace, size_t ws_bytes, void* stream) {
+    g_err.clear();
+    if (!L || !L->dev) return fail(FOCR_ERR_INVALID_ARG, "lm_head is NULL");
+    if (T < 1 || T > FOCR_T_MAX) return fail(FOCR_ERR_INVALID_ARG, "T=%d outside [1, %d]", T, FOCR_T_MAX);
+    if (!x || !argmax || !workspace) return fail(FOCR_ERR_INVALID_ARG, "x, argmax and workspace must not be NULL");
+    if (!aligned(x, 16) || !aligned(workspace, 256)) return fail(FOCR_ERR_INVALID_ARG, "misaligned x or workspace");
+    if (ws_bytes < focr_lm_head_workspace_bytes(T))
+        return fail(FOCR_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, focr_lm_head_workspace_bytes(T));
+    const int grid = lm_head_grid();
+    if (grid > 1024) return fail(FOCR_ERR_UNSUPPORTED, "%d SMs exceed the workspace plan", grid);
+    const uint4* codes = reinterpret_cast<const uint4*>(L->dev);
+    const float* scales = reinterpret_cast<const float*>(L->dev + (size_t)FOCR_VOCAB * H);
+    CUDA_TRY(launch_lm_head(codes, scales, x, T, logits, argmax, workspace, (cudaStream_t)stream));
+    return FOCR_OK;
+}
+
+focr_status focr_rmsnorm(const float* x, const float* gamma, int32_t T, float eps, float* out, void* stream) {
+    g_err.clear();
+    if (T < 1 || T > FOCR_T_MAX) return fail(FOCR_ERR_INVALID_ARG, "T=%d outside [1, %d]", T, FOCR_T_MAX);
+    if (!x || !out) return fail(FOCR_ERR_INVALID_ARG, "x and out must not be NULL");
+    if (!aligned(x, 16) || !aligned(out, 16) || (gamma && !aligned(gamma, 16)))
+        return fail(FOCR_ERR_INVALID_ARG, "x, out and gamma must be 16-byte aligned");
+    if (!(eps >= 0.f)) return fail(FOCR_ERR_INVALID_ARG, "eps must be >= 0");
+    CUDA_TRY(launch_rmsnorm(x, gamma, T, eps, out, (cudaStream_t)stream));
+    return FOCR_OK;
+}
+
+focr_status focr_moe_layer_forward(const focr_moe_layer* L, const float* hidden, int32_t T, float* out,
+                                   void* workspace, size_t ws_bytes, const focr_moe_route_debug* dbg, void* stream) {
+    return focr_moe_layer_forward_ex(L, hidden, T, out, workspace, ws_bytes, dbg, 0, stream);
+}
+
+// ------------------------------------------------------------------ dense SwiGLU MLP (layer 0)
+
+struct focr_dense_mlp {
+    int32_t wtype, group;
+    ItemGeom g;
+    uint8_t* dev = nullptr;
+    size_t bytes = 0, off_items = 0, off_dsc = 0;
+};
+
+focr_status focr_dense_mlp_pack(const float* w_gate, const float* w_up, const float* w_down, int32_t wtype,
+                                int32_t group, focr_dense_mlp** out, void* stream) {
+    g_err.clear();
+    if (!w_gate || !w_up || !w_down || !out) return fail(FOCR_ERR_INVALID_ARG, "NULL argument");
+    *out = nullptr;
+    focr_status s = check_types(wtype, wtype, group);
+    if (s != FOCR_OK) return s;
+    focr_dense_mlp* M = new (std::nothrow) focr_dense_mlp();
+    if (!M) return fail(FOCR_ERR_OOM, "host allocation failed");
+    M->wtype = wtype;
+    M->group = is_quant(wtype) ? group : 0;
+    M->g = make_geom(wtype, group, FOCR_DENSE_INTER);
+    M->off_items = 0;
+    M->off_dsc = align_up((size_t)M->g.slices * M->g.item_bytes, 256);
+    M->bytes = align_up(M->off_dsc + sizeof(float) * (size_t)M->g.dscale_expert_floats, 256);
+    std::vector<uint8_t> host;
+    try {
+        host.assign(M->bytes, 0);
+    } catch (...) {
+        delete M;
+        return fail(FOCR_ERR_OOM, "host staging of %zu bytes failed", M->bytes);
+    }
+    host_pack_set(w_gate, w_up, w_down, M->g, host.data(), reinterpret_cast<float*>(host.data() + M->off_dsc));
+    cudaError_t e = cudaMalloc(&M->dev, M->bytes);
+    if (e != cudaSuccess) {
+        delete M;
+        return fail(e == cudaErrorMemoryAllocation ? FOCR_ERR_OOM : FOCR_ERR_CUDA, "cudaMalloc(%zu): %s", M->bytes,
+                    cudaGetErrorString(e));
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    e = cudaMemcpyAsync(M->dev, host.data(), M->bytes, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) {
+        cudaFree(M->dev);
+        delete M;
+        return cuda_fail(e, "upload of packed dense MLP");
+    }
+    *out = M;
+    return FOCR_OK;
+}
+
+void focr_dense_mlp_free(focr_dense_mlp* M) {
+    if (!M) return;
+    if (M->dev) cudaFree(M->dev);
+    delete M;
+}
+
+focr_status focr_dense_mlp_export_quantized(const focr_dense_mlp* M, int32_t matrix, void* codes, size_t code_bytes,
+                                            float* scales, size_t n_scales) {
+    g_err.clear();
+    if (!M || !codes) return fail(FOCR_ERR_INVALID_ARG, "NULL argument");
+    if (matrix < 0 || matrix > 2) return fail(FOCR_ERR_INVALID_ARG, "unknown matrix %d", matrix);
+    const int64_t rows = matrix < 2 ? FOCR_DENSE_INTER : H, cols = matrix < 2 ? H : FOCR_DENSE_INTER;
+    const size_t n = (size_t)(rows * cols);
+    const int wt = M->wtype;
+    const size_t need_c = wt == FOCR_W_INT4 ? n / 2 : (wt == FOCR_W_INT8 ? n : 2 * n);
+    const size_t need_s = is_quant(wt) ? (size_t)rows * (size_t)((cols + M->group - 1) / M->group) : 0;
+    if (code_bytes < need_c) return fail(FOCR_ERR_INVALID_ARG, "codes buffer too small (need %zu)", need_c);
+    if (need_s && (!scales || n_scales < need_s))
+        return fail(FOCR_ERR_INVALID_ARG, "scales buffer too small (need %zu)", need_s);
+    std::vector<uint8_t> items((size_t)M->g.slices * M->g.item_bytes);
+    std::vector<float> dsc(M->g.dscale_expert_floats);
+    CUDA_TRY(cudaMemcpy(items.data(), M->dev + M->off_items, items.size(), cudaMemcpyDeviceToHost));
+    if (!dsc.empty())
+        CUDA_TRY(cudaMemcpy(dsc.data(), M->dev + M->off_dsc, dsc.size() * sizeof(float), cudaMemcpyDeviceToHost));
+    if (wt == FOCR_W_BF16) {
+        host_unpack_matrix(items.data(), nullptr, M->g, matrix, nullptr, reinterpret_cast<uint16_t*>(codes), nullptr);
+    } else {
+        std::vector<int8_t> q(n);
+        host_unpack_matrix(items.data(), dsc.data(), M->g, matrix, q.data(), nullptr, scales);
+        if (wt == FOCR_W_INT8) {
+            std::memcpy(codes, q.data(), n);
+        } else {
+            uint8_t* c = reinterpret_cast<uint8_t*>(codes);
+            for (size_t j = 0; j < n / 2; ++j)
+                c[j] = (uint8_t)(((uint8_t)q[2 * j] & 0xFu) | (((uint8_t)q[2 * j + 1] & 0xFu) << 4));
+        }
+    }
+    return FOCR_OK;
+}
+
+focr_status focr_dense_mlp_forward(const focr_dense_mlp* M, const float* x, int32_t T, float* out, void* workspace,
+                                   size_t ws_bytes, int32_t flags, void* stream) {
+    g_err.clear();
+    if (!M || !M->dev) return fail(FOCR_ERR_INVALID_ARG, "dense MLP is NULL");
+    if (flags & ~FOCR_FWD_RESIDUAL) return fail(FOCR_ERR_INVALID_ARG, "unknown flags 0x%x", (unsigned)flags);
+    if (T < 1 || T > FOCR_T_MAX) return fail(FOCR_ERR_INVALID_ARG, "T=%d outside [1, %d]", T, FOCR_T_MAX);
+    if (!x || !out || !workspace) return fail(FOCR_ERR_INVALID_ARG, "x, out and workspace must not be NULL");
+    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(workspace, 256))
+        return fail(FOCR_ERR_INVALID_ARG, "misaligned x, out or workspace");
+    if (ws_bytes < ws_layout(T).total)
+        return fail(FOCR_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, ws_layout(T).total);
+    const size_t nb = (size_t)T * H * sizeof(float);
+    {
+        const char* a = (const char*)x;
+        const char* b = (const char*)out;
+        if (a < b + nb && b < a + nb) return fail(FOCR_ERR_INVALID_ARG, "x and out overlap");
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    if (flags & FOCR_FWD_RESIDUAL) CUDA_TRY(cudaMemcpyAsync(out, x, nb, cudaMemcpyDeviceToDevice, st));
+    else CUDA_TRY(cudaMemsetAsync(out, 0, nb, st));
+    LayerView v{};
+    v.shared_items = M->dev + M->off_items;
+    v.shared_dscale = reinterpret_cast<const float*>(M->dev + M->off_dsc);
+    v.routed_items = v.shared_items;
+    v.routed_dscale = v.shared_dscale;
+    v.rg = M->g;
+    v.sg = M->g;
+    if (T <= SMALL_T) CUDA_TRY(launch_decode_small(x, T, v, route_view(workspace, T), out, true, st));
+    else CUDA_TRY(launch_expert_decode(x, T, v, route_view(workspace, T), out, true, st));
     return FOCR_OK;
 }
 

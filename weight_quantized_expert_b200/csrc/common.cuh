@@ -32,7 +32,7 @@ constexpr int IS = FOCR_SHARED_INTER;
 //                (int4: two k-steps; int8: one k-step; bf16: one 16x8x8 step, elements
 //                (gr, 2c) (gr, 2c+1) (gr+8, 2c) (gr+8, 2c+1))
 // and, outside the item block, the down scales of the whole expert:
-//   D scales   : [inter/g groups][1280 rows] f32                     (quantised types only)
+//   D scales   : [ceil(inter/g) groups][1280 rows] f32               (quantised types only)
 // Codes are offset-binary: int4 q+8 with e0..e7 in nibble slots 0,4,1,5,2,6,3,7 of a
 // 32-bit word (so one mask pulls a register pair); int8 q+128 in bytes e0..e7; bf16 as
 // bit patterns.  S is 32 (int4), 16 (int8), 8 (bf16): a down row slice is always 16 bytes.
@@ -68,7 +68,7 @@ __host__ __device__ constexpr uint32_t blk_bytes_of(int wtype, int G) {
 struct ItemGeom {
     int wtype, group, S, inter, slices;
     uint32_t gu_w_bytes, gu_s_bytes, d_w_bytes, item_bytes;  // item_bytes: 128-byte multiple
-    uint32_t dscale_expert_floats;                           // inter/g * 1280 (0 for bf16)
+    uint32_t dscale_expert_floats;                           // ceil(inter/g) * 1280 (0 for bf16)
 };
 
 __host__ __device__ inline ItemGeom make_geom(int wtype, int group, int inter) {
@@ -83,7 +83,7 @@ __host__ __device__ inline ItemGeom make_geom(int wtype, int group, int inter) {
     g.d_w_bytes = d_w_bytes_of();
     uint32_t raw = g.gu_w_bytes + g.gu_s_bytes + g.d_w_bytes;
     g.item_bytes = (raw + 127u) & ~127u;
-    g.dscale_expert_floats = is_quant(wtype) ? (uint32_t)(inter / group) * H : 0u;
+    g.dscale_expert_floats = is_quant(wtype) ? (uint32_t)((inter + group - 1) / group) * H : 0u;
     return g;
 }
 
@@ -91,7 +91,7 @@ __host__ __device__ inline ItemGeom make_geom(int wtype, int group, int inter) {
 struct LayerView {
     const uint16_t* router;        // [64][1280] bf16
     const uint8_t* routed_items;   // [64][slices][item_bytes]
-    const float* routed_dscale;    // [64][inter/g][1280]
+    const float* routed_dscale;    // [64][ceil(inter/g)][1280]
     const uint8_t* shared_items;   // [slices][item_bytes]
     const float* shared_dscale;    // [1792/g][1280]
     ItemGeom rg, sg;
@@ -106,7 +106,14 @@ constexpr int ROUTER_TB = 8;              // tokens per router CTA
 constexpr int MAX_TB = (FOCR_T_MAX + ROUTER_TB - 1) / ROUTER_TB;
 
 struct WsLayout {
+    // regions that are zero on entry and that every forward leaves zero; their offsets do
+    // not depend on T_max, so calls with different T may share one workspace
     size_t ctrl;          // int32 [MAX_TB tickets][1 global ticket][1 error word][pad]
+    size_t gacc;          // f32 [GU_TILES][32 lanes][4]  gate/up sums of k-split tiles (T <= 8)
+    size_t tcnt;          // i32 [GU_TILES]               their arrival counters
+    // regions every forward writes before reading
+    size_t a16;           // uint2 [A16_STEPS][32]   f16 a fragments (int4 / int8 down, T <= 8)
+    size_t abf;           // uint2 [ABF_STEPS][32]   bf16 a hi, lo fragments (bf16 down, T <= 8)
     size_t logits;        // f32 [T_max][64]
     size_t topk_idx;      // i32 [T_max][6]
     size_t topk_w;        // f32 [T_max][6]
@@ -117,12 +124,23 @@ struct WsLayout {
     size_t total;
 };
 
+// gate/up tiles of 8 intermediates: a shared set of up to IS_MAX intermediates, then 64
+// routed experts (896/8 each); a set of IS_MAX = 6848 covers the dense layer
+constexpr int IS_MAX = FOCR_DENSE_INTER;
+constexpr int GU_TILES = IS_MAX / 8 + E * (I / 8);
+constexpr int A16_STEPS = IS_MAX / 16 + E * (I / 16);   // k-steps of 16 intermediates
+constexpr int ABF_STEPS = IS_MAX / 8 + E * (I / 8);     // k-steps of 8 intermediates
+
 constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 constexpr WsLayout ws_layout(int T_max) {
     WsLayout w{};
     size_t o = 0;
     w.ctrl = o;      o = align_up(o + sizeof(int32_t) * (MAX_TB + 64), 256);
+    w.gacc = o;      o = align_up(o + sizeof(float) * 4 * 32 * (size_t)GU_TILES, 256);
+    w.tcnt = o;      o = align_up(o + sizeof(int32_t) * (size_t)GU_TILES, 256);
+    w.a16 = o;       o = align_up(o + 8 * 32 * (size_t)A16_STEPS, 256);
+    w.abf = o;       o = align_up(o + 8 * 32 * (size_t)ABF_STEPS, 256);
     w.logits = o;    o = align_up(o + sizeof(float) * (size_t)T_max * E, 256);
     w.topk_idx = o;  o = align_up(o + sizeof(int32_t) * (size_t)T_max * K, 256);
     w.topk_w = o;    o = align_up(o + sizeof(float) * (size_t)T_max * K, 256);
@@ -147,6 +165,10 @@ struct RouteView {   // device pointers into the workspace
     int32_t* offsets;
     int32_t* active;
     int32_t* perm;
+    float* gacc;
+    int32_t* tcnt;
+    uint2* a16;
+    uint2* abf;
 };
 
 inline RouteView route_view(void* ws, int T_max) {
@@ -154,7 +176,8 @@ inline RouteView route_view(void* ws, int T_max) {
     char* b = (char*)ws;
     return RouteView{(int32_t*)(b + L.ctrl), (float*)(b + L.logits),
                      (int32_t*)(b + L.topk_idx), (float*)(b + L.topk_w), (int32_t*)(b + L.counts),
-                     (int32_t*)(b + L.offsets), (int32_t*)(b + L.active), (int32_t*)(b + L.perm)};
+                     (int32_t*)(b + L.offsets), (int32_t*)(b + L.active), (int32_t*)(b + L.perm),
+                     (float*)(b + L.gacc), (int32_t*)(b + L.tcnt), (uint2*)(b + L.a16), (uint2*)(b + L.abf)};
 }
 
 // error codes a kernel may store in the error word
@@ -162,10 +185,15 @@ constexpr int DEVERR_FULL_WAIT = 1;
 constexpr int DEVERR_EMPTY_WAIT = 2;
 
 // ------------------------------------------------------------------ launchers (per .cu)
+// resid: NULL zeroes `out` before the experts add into it; otherwise `out` starts as a copy of resid
 cudaError_t launch_router(const float* x, int T, int T_ws, const LayerView& L, const RouteView& R, float* out,
-                          cudaStream_t st);
+                          const float* resid, cudaStream_t st);
 cudaError_t launch_expert_decode(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
-                                 cudaStream_t st);
+                                 bool shared_only, cudaStream_t st);
+// T <= SMALL_T: gate/up + swiglu kernel, then the down kernel (decode_small.cu)
+constexpr int SMALL_T = 8;
+cudaError_t launch_decode_small(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
+                                bool shared_only, cudaStream_t st);
 
 }  // namespace focr
 

@@ -10,14 +10,16 @@
 // Work: an "item" is one slice of S intermediate rows of one expert (common.cuh; ~60-77
 // KB).  Items are numbered shared-expert slices first, then the slices of every expert
 // that received tokens (ascending id); CTA b of a persistent grid (one per SM) takes
-// items b, b+G, ...  A producer warp streams item blocks into a two-slot shared-memory
+// items b, b+G, ...  A producer warp streams item blocks into a 2- or 3-slot shared-memory
 // ring with bulk async copies (cp.async.bulk + mbarrier) and publishes each item's
-// expert id next to it; 16 consumer warps compute:
-//   phase 1  [g; u] = [G; U]_slice x  -- warp (tile, k-part): mma.sync m16n8k16; int4/int8
-//            codes become exact f16 values in registers and are multiplied by their group
-//            scale (f16); bf16 weights feed bf16 MMAs as stored; k-parts summed in shared memory
+// expert id next to it; 20 consumer warps compute:
+//   phase 1  [g; u] = [G; U]_slice x  -- warp w covers input columns [64w, 64w + 64) of every
+//            tile with mma.sync m16n8k16 (x's fragments stay in its registers); int4/int8
+//            codes become exact f16 values and each scale group's fp32 accumulator is
+//            multiplied by its scale; bf16 weights feed bf16 MMAs as stored; the twenty
+//            column parts are summed in shared memory
 //   swiglu   a = silu(g) * u * w_route  (fp32, then f16 phase-2 B fragments)
-//   phase 2  y = D[:, slice] a          -- warp owns 5 of the 80 output tiles
+//   phase 2  y = D[:, slice] a          -- warp owns 4 of the 80 output tiles
 // Tokens are the 8 columns of the n8 fragments.  With T <= 8 every item uses the same
 // columns (the batch), routed weights of tokens that did not pick the expert are 0, and
 // the layer output stays in registers across all of a CTA's items: one flush of atomics
@@ -28,45 +30,48 @@
 // and no output is added before it (the router zeroes `out`).  Every mbarrier wait is
 // bounded in time; on expiry the kernel records an error word and stops.
 //
-// Precision: int4/int8 weights enter the MMA as f16(q * s) (one rounding, relative 2^-11;
-// scales below f16's normal range lose bits) with x and a rounded to f16; bf16 weights
-// enter unchanged and x and a are split into bf16 hi + lo parts (two MMAs, about 16
-// significant bits); every product accumulates in fp32.
+// Precision: int4/int8 codes are exact in f16 and scales are applied in fp32; x and a are
+// rounded to f16 (relative 2^-11) for them.  bf16 weights enter unchanged and x and a are
+// split into bf16 hi + lo parts (two MMAs, about 16 significant bits).  Every product
+// accumulates in fp32.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "fragments.cuh"
 
 namespace focr {
 namespace {
 
-constexpr int NCW = 16;                      // consumer warps
+constexpr int NCW = 20;                      // consumer warps
 constexpr int NCT = NCW * 32;                // consumer threads
 constexpr int NTHREADS = NCT + 32;           // + producer warp
-constexpr int NSLOT = 2;
 constexpr int NTOK = 8;                      // tokens per fragment (n8)
-constexpr uint32_t SLOT_BYTES = 76800;       // largest item (int4 g32) + its down scales
 constexpr uint32_t DSC_BYTES = H * 4;        // one group's down scales
-constexpr int TILES_PER_WARP = OTILES / NCW; // 5
+constexpr int TILES_PER_WARP = OTILES / NCW; // 4
+constexpr int KSW = KSTEPS / NCW;            // 4 k-steps of phase 1 per warp
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s
 
-template <int RW, int SW>
+// Ring slots are sized for the kernel's own item types; three slots when they fit.
+template <int RW, int SW, int G>
 struct SmemLayout {
-    static constexpr bool F16 = is_quant(RW) || is_quant(SW);     // some expert uses f16 MMAs
-    static constexpr bool BF16 = !is_quant(RW) || !is_quant(SW);  // some expert uses bf16 MMAs
+    static constexpr uint32_t item_r = blk_bytes_of(RW, G) + (is_quant(RW) ? DSC_BYTES : 0u);
+    static constexpr uint32_t item_s = blk_bytes_of(SW, G) + (is_quant(SW) ? DSC_BYTES : 0u);
+    static constexpr uint32_t slot_bytes = ((item_r > item_s ? item_r : item_s) + 127u) & ~127u;
+    static constexpr uint32_t rest = 4 * 4 * 32 * 4 + 2 * 32 * 8 + 32 * 8 + 2 * NTOK * 4 + 2 * NTOK * K * 4 + 16 +
+                                     2 * 3 * 8 + 16;
+    static constexpr int nslot = 3 * slot_bytes + rest <= 232448 ? 3 : 2;
     static constexpr uint32_t slots = 0;
-    static constexpr uint32_t xh = slots + NSLOT * SLOT_BYTES;          // [80][32] uint2: f16 x B frags
-    static constexpr uint32_t xb = xh + (F16 ? KSTEPS * 32 * 8 : 0);    // [80][32] uint4: bf16 x hi, lo frags
-    static constexpr uint32_t red = xb + (BF16 ? KSTEPS * 32 * 16 : 0); // [16 tasks][32] float4
-    static constexpr uint32_t ah = red + 16 * 32 * 16;                  // [2][32] uint2: f16 a B frags
+    static constexpr uint32_t acc = slots + nslot * slot_bytes;         // [4 tiles][4 comps][32] f32 phase-1 sums
+    static constexpr uint32_t ah = acc + 4 * 4 * 32 * 4;                // [2][32] uint2: f16 a B frags
     static constexpr uint32_t abf = ah + 2 * 32 * 8;                    // [32] uint2: bf16 a hi, lo frags
     static constexpr uint32_t wn = abf + 32 * 8;                        // [NTOK] f32 route weights
     static constexpr uint32_t tok = wn + NTOK * 4;                      // [NTOK] i32 token ids
     static constexpr uint32_t ridx = tok + NTOK * 4;                    // [NTOK][6] i32 (T <= 8)
     static constexpr uint32_t rw = ridx + NTOK * K * 4;                 // [NTOK][6] f32 (T <= 8)
-    static constexpr uint32_t rec = rw + NTOK * K * 4;                  // [NSLOT] i32 expert of the slot's item
-    static constexpr uint32_t bars = rec + 16;                          // full[NSLOT], empty[NSLOT]
-    static constexpr uint32_t misc = bars + 2 * NSLOT * 8;
+    static constexpr uint32_t rec = rw + NTOK * K * 4;                  // [nslot] i32 expert of the slot's item
+    static constexpr uint32_t bars = rec + 16;                          // full[nslot], empty[nslot]
+    static constexpr uint32_t misc = bars + 2 * 3 * 8;
     static constexpr uint32_t total = misc + 16;
     static_assert(total <= 232448, "shared memory budget");
 };
@@ -77,209 +82,122 @@ struct ExpertParams {
     float* out;
     LayerView L;
     RouteView R;
+    int shared_only;   // a single dense SwiGLU (the "shared" weight set), no routing
 };
 
-// ------------------------------------------------------------------ fragments
-struct Frag4 {
-    uint32_t r[4];
+// ------------------------------------------------------------------ x fragments (registers)
+// Warp w owns k-steps 4w .. 4w+3 of phase 1 for every item, so its B fragments of x stay in
+// registers: h[j] = f16 (for int4/int8 experts), b[j] = bf16 hi (b0, b1), lo (b0, b1) (for
+// bf16 experts).  Lane (n = lane / 4, c = lane % 4) holds columns 16q+2c, +1 and 16q+2c+8,
+// +9 of token column n; tok[n] < 0 gives zeros.
+template <bool F16, bool BF16>
+struct XFrags {
+    uint32_t h[F16 ? KSW : 1][2];
+    uint32_t b[BF16 ? KSW : 1][4];
 };
 
-__device__ __forceinline__ void mma16816(float (&d)[4], const Frag4& a, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a.r[0]), "r"(a.r[1]), "r"(a.r[2]), "r"(a.r[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void mma1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(b0));
-}
-
-__device__ __forceinline__ void mma16816_bf16(float (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void mma1688_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(b0));
-}
-
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t d;
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
-    uint32_t d;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-    return d;
-}
-
-constexpr uint32_t H2_1032 = 0x64086408u;   // (1032, 1032)
-constexpr uint32_t H2_1152 = 0x64806480u;   // (1152, 1152)
-constexpr uint32_t H2_1_16 = 0x2C002C00u;   // (1/16, 1/16)
-constexpr uint32_t H2_M72 = 0xD480D480u;    // (-72, -72)
-
-// 8 int4 codes (offset-binary, slots 0,4 | 1,5 | 2,6 | 3,7) -> A fragment, exact q in f16.
-// (w & mask) | 0x6400 reads as 1024 + n (low nibble) or 1024 + 16 n (second nibble).
-__device__ __forceinline__ Frag4 dq_int4(uint32_t w) {
-    Frag4 f;
-    const uint32_t w8 = w >> 8;
-    f.r[0] = hsub2((w & 0x000F000Fu) | 0x64006400u, H2_1032);
-    f.r[1] = hfma2((w & 0x00F000F0u) | 0x64006400u, H2_1_16, H2_M72);
-    f.r[2] = hsub2((w8 & 0x000F000Fu) | 0x64006400u, H2_1032);
-    f.r[3] = hfma2((w8 & 0x00F000F0u) | 0x64006400u, H2_1_16, H2_M72);
-    return f;
-}
-
-// 8 int8 codes (offset-binary bytes e0..e7) -> A fragment; 0x64bb reads as 1024 + bb
-__device__ __forceinline__ Frag4 dq_int8(uint32_t w0, uint32_t w1) {
-    Frag4 f;
-    f.r[0] = hsub2(__byte_perm(w0, 0x64646464u, 0x4140), H2_1152);
-    f.r[1] = hsub2(__byte_perm(w0, 0x64646464u, 0x4342), H2_1152);
-    f.r[2] = hsub2(__byte_perm(w1, 0x64646464u, 0x4140), H2_1152);
-    f.r[3] = hsub2(__byte_perm(w1, 0x64646464u, 0x4342), H2_1152);
-    return f;
-}
-
-__device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
-    uint32_t d;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
-    return d;
-}
-
-// bf16 hi + lo split of two fp32 values: returns {hi pair, lo pair}
-__device__ __forceinline__ uint2 split_bf16x2(float a, float b) {
-    const uint32_t hi = f32x2_to_bf16x2(a, b);
-    const float ra = a - __uint_as_float(hi << 16), rb = b - __uint_as_float(hi & 0xFFFF0000u);
-    return make_uint2(hi, f32x2_to_bf16x2(ra, rb));
+template <bool F16, bool BF16>
+__device__ __forceinline__ void load_x_frags(const float* x, const int* tok, int warp, int lane,
+                                             XFrags<F16, BF16>& xf) {
+    const int tk = tok[lane >> 2];
+    float2 lo[KSW], hi[KSW];
+#pragma unroll
+    for (int j = 0; j < KSW; ++j) {
+        lo[j] = hi[j] = make_float2(0.f, 0.f);
+        if (tk >= 0) {
+            const float* row = x + (size_t)tk * H + 16 * (KSW * warp + j) + 2 * (lane & 3);
+            lo[j] = __ldg(reinterpret_cast<const float2*>(row));
+            hi[j] = __ldg(reinterpret_cast<const float2*>(row + 8));
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < KSW; ++j) {
+        if constexpr (F16) {
+            xf.h[j][0] = f32x2_to_f16x2(lo[j].x, lo[j].y);
+            xf.h[j][1] = f32x2_to_f16x2(hi[j].x, hi[j].y);
+        }
+        if constexpr (BF16) {
+            const uint2 a = split_bf16x2(lo[j].x, lo[j].y), b = split_bf16x2(hi[j].x, hi[j].y);
+            xf.b[j][0] = a.x;
+            xf.b[j][1] = b.x;
+            xf.b[j][2] = a.y;
+            xf.b[j][3] = b.y;
+        }
+    }
 }
 
 // ------------------------------------------------------------------ phase 1: gate/up
-// QN k-steps starting at q0 of tile t; PH = q0 % (G / 16) is a compile-time phase so every
-// group boundary, and the scale register it uses, is known at compile time.
-template <int W, int G, int PH>
-__device__ __forceinline__ void gate_up_quant(const char* slot, const uint2* xh, float (&tot)[4], int t, int q0,
+// Every tile of the item over this warp's four k-steps.  int4/int8 codes become exact f16
+// values and the fp32 accumulator of each scale group is multiplied by its group scale
+// (the four k-steps lie in one group for g >= 64, in two for g = 32).
+template <int W, int G, bool F16, bool BF16>
+__device__ __forceinline__ void phase_gate_up(const char* slot, const XFrags<F16, BF16>& xf, float* acc_s, int warp,
                                               int lane) {
     constexpr int NT = slice_rows(W) / 8;
-    constexpr int KP = NCW / NT;
-    constexpr int QN = KSTEPS / KP;
-    constexpr int KPV = ksteps_per_vec(W);
-    constexpr int SPG = G / 16;
-    constexpr int NGK = H / G;
-    constexpr int NGW = (PH + QN - 1) / SPG + 1;      // groups this warp touches
     const int gr = lane >> 2;
-    const uint4* gw = reinterpret_cast<const uint4*>(slot) + (t * (KSTEPS / KPV) + q0 / KPV) * 32 + lane;
-    const uint2* xb = xh + q0 * 32 + lane;
-    const float2* gs = reinterpret_cast<const float2*>(slot + gu_w_bytes_of(W)) + (t * NGK + (q0 - PH) / SPG) * 8 + gr;
-    uint32_t sg[NGW], su[NGW];   // (gate, gate) and (up, up) scales as f16x2
 #pragma unroll
-    for (int g = 0; g < NGW; ++g) {
-        const float2 v = gs[g * 8];
-        sg[g] = f32x2_to_f16x2(v.x, v.x);
-        su[g] = f32x2_to_f16x2(v.y, v.y);
-    }
-    float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};   // even / odd k-steps
+    for (int t = 0; t < NT; ++t) {
+        float tot[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (!is_quant(W)) {
+            const uint4* gw = reinterpret_cast<const uint4*>(slot) + (t * KSTEPS + KSW * warp) * 32 + lane;
 #pragma unroll
-    for (int qv = 0; qv < QN / KPV; ++qv) {
-        const uint4 v = gw[qv * 32];
-        const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int j = 0; j < KPV; ++j) {
-            const int qq = qv * KPV + j;
-            const int g = (PH + qq) / SPG;
-            const uint2 b = xb[qq * 32];
-            Frag4 a;
-            if constexpr (W == FOCR_W_INT4) a = dq_int4(vv[j]);
-            else a = dq_int8(vv[2 * j], vv[2 * j + 1]);
-            a.r[0] = hmul2(a.r[0], sg[g]);
-            a.r[1] = hmul2(a.r[1], su[g]);
-            a.r[2] = hmul2(a.r[2], sg[g]);
-            a.r[3] = hmul2(a.r[3], su[g]);
-            if (qq & 1) mma16816(acc1, a, b.x, b.y);
-            else mma16816(acc0, a, b.x, b.y);
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) tot[r] = acc0[r] + acc1[r];
-}
-
-template <int W, int G>
-__device__ __forceinline__ void phase_gate_up(const char* slot, const uint2* xh, const uint4* xbf, float4* red,
-                                              int warp, int lane) {
-    constexpr int NT = slice_rows(W) / 8;       // tiles per item
-    constexpr int KP = NCW / NT;                // k-parts
-    constexpr int QN = KSTEPS / KP;             // k-steps per warp
-    const int t = warp % NT, part = warp / NT;
-    const int q0 = part * QN;
-    float tot[4];
-    if constexpr (!is_quant(W)) {
-        // bf16 weights as stored; x as bf16 hi + lo
-        const uint4* gw = reinterpret_cast<const uint4*>(slot) + (t * KSTEPS + q0) * 32 + lane;
-        const uint4* xb = xbf + q0 * 32 + lane;
-        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int q = 0; q < QN; ++q) {
-            const uint4 a = gw[q * 32];
-            const uint4 b = xb[q * 32];
-            if (q & 1) {
-                mma16816_bf16(acc1, a, b.x, b.y);
-                mma16816_bf16(acc1, a, b.z, b.w);
+            for (int j = 0; j < KSW; ++j) {
+                const uint4 a = gw[j * 32];
+                mma16816_bf16(tot, a, xf.b[j][0], xf.b[j][1]);   // x hi
+                mma16816_bf16(tot, a, xf.b[j][2], xf.b[j][3]);   // x lo
+            }
+        } else {
+            constexpr int NGK = H / G;
+            uint32_t wv[8];
+            if constexpr (W == FOCR_W_INT4) {
+                const uint4 v = reinterpret_cast<const uint4*>(slot)[(t * (KSTEPS / 4) + warp) * 32 + lane];
+                wv[0] = v.x; wv[1] = v.y; wv[2] = v.z; wv[3] = v.w;
             } else {
-                mma16816_bf16(acc0, a, b.x, b.y);
-                mma16816_bf16(acc0, a, b.z, b.w);
+                const uint4* g8 = reinterpret_cast<const uint4*>(slot) + (t * (KSTEPS / 2) + 2 * warp) * 32 + lane;
+                const uint4 v0 = g8[0], v1 = g8[32];
+                wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w;
+                wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
+            }
+            const float2* gs = reinterpret_cast<const float2*>(slot + gu_w_bytes_of(W)) + t * NGK * 8 + gr;
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int j = 0; j < KSW; ++j) {
+                Frag4 a;
+                if constexpr (W == FOCR_W_INT4) a = dq_int4(wv[j]);
+                else a = dq_int8(wv[2 * j], wv[2 * j + 1]);
+                mma16816(acc[G == 32 ? j >> 1 : 0], a, xf.h[j][0], xf.h[j][1]);
+            }
+            constexpr int NG = G == 32 ? 2 : 1;
+#pragma unroll
+            for (int h = 0; h < NG; ++h) {
+                const int gi = G == 32 ? 2 * warp + h : (KSW * warp * 16) / G;
+                const float2 sc = gs[gi * 8];
+                tot[0] = fmaf(acc[h][0], sc.x, tot[0]);
+                tot[1] = fmaf(acc[h][1], sc.x, tot[1]);
+                tot[2] = fmaf(acc[h][2], sc.y, tot[2]);
+                tot[3] = fmaf(acc[h][3], sc.y, tot[3]);
             }
         }
+        // the twenty warps' partial sums meet in shared memory ([tile][component][lane])
 #pragma unroll
-        for (int r = 0; r < 4; ++r) tot[r] = acc0[r] + acc1[r];
-    } else {
-        constexpr int SPG = G / 16;
-        switch (q0 % SPG) {
-            case 0: gate_up_quant<W, G, 0>(slot, xh, tot, t, q0, lane); break;
-            case 2: if constexpr (SPG > 2) gate_up_quant<W, G, 2 % SPG>(slot, xh, tot, t, q0, lane); break;
-            case 4: if constexpr (SPG > 4) gate_up_quant<W, G, 4 % SPG>(slot, xh, tot, t, q0, lane); break;
-            default: if constexpr (SPG > 6) gate_up_quant<W, G, 6 % SPG>(slot, xh, tot, t, q0, lane); break;
-        }
+        for (int r = 0; r < 4; ++r) atomicAdd(acc_s + (t * 4 + r) * 32 + lane, tot[r]);
     }
-    red[warp * 32 + lane] = make_float4(tot[0], tot[1], tot[2], tot[3]);
 }
 
 // ------------------------------------------------------------------ swiglu -> phase-2 B fragments
+// One thread per (tile, lane) reads the summed g and u (and clears them for the next item);
+// a = silu(g) * u * w_route goes into the phase-2 B fragments.
 template <int W>
-__device__ __forceinline__ void swiglu_to_frag(const float4* red, __half* ah, __nv_bfloat16* abf, const float* wn,
+__device__ __forceinline__ void swiglu_to_frag(float* acc_s, __half* ah, __nv_bfloat16* abf, const float* wn,
                                                int ctid) {
     constexpr int NT = slice_rows(W) / 8;
-    constexpr int KP = NCW / NT;
     if (ctid >= NT * 32) return;
     const int t = ctid >> 5, lane = ctid & 31;
+    float4 s;
+    float* a4 = acc_s + t * 4 * 32 + lane;
+    s.x = a4[0]; s.y = a4[32]; s.z = a4[64]; s.w = a4[96];
+    a4[0] = a4[32] = a4[64] = a4[96] = 0.f;
     const int gr = lane >> 2, c = lane & 3;
-    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int p = 0; p < KP; ++p) {
-        const float4 v = red[(p * NT + t) * 32 + lane];
-        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
-    }
     // s.x, s.y: gate of intermediate 8t+gr for tokens 2c, 2c+1; s.z, s.w: up
     const float a[2] = {s.x / (1.f + __expf(-s.x)) * s.z * wn[2 * c], s.y / (1.f + __expf(-s.y)) * s.w * wn[2 * c + 1]};
     const int i = 8 * t + gr;                     // slice-local intermediate index = k of phase 2
@@ -346,49 +264,21 @@ __device__ __forceinline__ void phase_down(const char* slot, const uint2* ah, co
 
 __device__ __forceinline__ void consumer_sync() { named_bar_sync(1, NCT); }
 
-// x rows of up to 8 tokens -> B fragments.  Entry (q, lane), n = lane / 4, c = lane % 4, holds
-// columns 16q+2c, +1 (first register) and 16q+2c+8, +9 (second) of token column n:
-// xh as f16, xb as bf16 hi then lo.  tok[n] < 0 gives a zero column.  All loads of a thread
-// are issued before any conversion.
-template <bool F16, bool BF16>
-__device__ __forceinline__ void build_x_frags(const float* x, const int* tok, uint2* xh, uint4* xb, int ctid) {
-    constexpr int PER = KSTEPS * 32 / NCT;   // 5 entries per thread
-    float2 lo[PER], hi[PER];
-#pragma unroll
-    for (int r = 0; r < PER; ++r) {
-        const int i = ctid + r * NCT;
-        const int q = i >> 5, ln = i & 31;
-        const int tk = tok[ln >> 2];
-        lo[r] = hi[r] = make_float2(0.f, 0.f);
-        if (tk >= 0) {
-            const float* row = x + (size_t)tk * H + 16 * q + 2 * (ln & 3);
-            lo[r] = __ldg(reinterpret_cast<const float2*>(row));
-            hi[r] = __ldg(reinterpret_cast<const float2*>(row + 8));
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < PER; ++r) {
-        const int i = ctid + r * NCT;
-        if constexpr (F16) xh[i] = make_uint2(f32x2_to_f16x2(lo[r].x, lo[r].y), f32x2_to_f16x2(hi[r].x, hi[r].y));
-        if constexpr (BF16) {
-            const uint2 a = split_bf16x2(lo[r].x, lo[r].y), b = split_bf16x2(hi[r].x, hi[r].y);
-            xb[i] = make_uint4(a.x, b.x, a.y, b.y);
-        }
-    }
-}
-
 // one item's phases, dispatched on whether it is a routed or a shared-expert item
 template <int RW, int SW, int G>
 struct ItemOps {
-    static __device__ __forceinline__ void gate_up(bool routed, const char* slot, const uint2* xh, const uint4* xb,
-                                                   float4* red, int warp, int lane) {
-        if (routed) phase_gate_up<RW, G>(slot, xh, xb, red, warp, lane);
-        else phase_gate_up<SW, G>(slot, xh, xb, red, warp, lane);
+    static constexpr bool F16 = is_quant(RW) || is_quant(SW);
+    static constexpr bool BF16 = !is_quant(RW) || !is_quant(SW);
+    using XF = XFrags<F16, BF16>;
+    static __device__ __forceinline__ void gate_up(bool routed, const char* slot, const XF& xf, float* acc, int warp,
+                                                   int lane) {
+        if (routed) phase_gate_up<RW, G>(slot, xf, acc, warp, lane);
+        else phase_gate_up<SW, G>(slot, xf, acc, warp, lane);
     }
-    static __device__ __forceinline__ void swiglu(bool routed, const float4* red, __half* ah, __nv_bfloat16* abf,
+    static __device__ __forceinline__ void swiglu(bool routed, float* acc, __half* ah, __nv_bfloat16* abf,
                                                   const float* wn, int ctid) {
-        if (routed) swiglu_to_frag<RW>(red, ah, abf, wn, ctid);
-        else swiglu_to_frag<SW>(red, ah, abf, wn, ctid);
+        if (routed) swiglu_to_frag<RW>(acc, ah, abf, wn, ctid);
+        else swiglu_to_frag<SW>(acc, ah, abf, wn, ctid);
     }
     static __device__ __forceinline__ void down(bool routed, const char* slot, const uint2* ah, const uint2* abf,
                                                 int warp, int lane, float (&y)[TILES_PER_WARP][4], bool accumulate) {
@@ -399,7 +289,10 @@ struct ItemOps {
 
 template <int RW, int SW, int G>
 __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams p) {
-    using SL = SmemLayout<RW, SW>;
+    using SL = SmemLayout<RW, SW, G>;
+    constexpr int NSLOT = SL::nslot;
+    constexpr uint32_t SLOT_BYTES = SL::slot_bytes;
+    using Ops = ItemOps<RW, SW, G>;
     extern __shared__ __align__(128) char smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + SL::bars);
     uint64_t* empty = full + NSLOT;
@@ -412,12 +305,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
     if (tid == 0) {
         for (int s = 0; s < NSLOT; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], NCW);   // every consumer warp releases the slot
         }
         fence_barrier_init();
         okflag[0] = 1;   // consumer wait result
         okflag[1] = 0;   // abort
     }
+    for (int i = tid; i < 4 * 4 * 32; i += NTHREADS) reinterpret_cast<float*>(smem + SL::acc)[i] = 0.f;
     __syncthreads();
 
     if (warp == NCW) {
@@ -445,8 +339,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
             }
         };
         for (int item = blockIdx.x; item < n_shared; item += gridDim.x) prefetch_item(item);
-        int n_items = 0x7fffffff;
-        bool waited = false;
+        int n_items = p.shared_only ? n_shared : 0x7fffffff;
+        bool waited = p.shared_only != 0;
         int issued = 0;
         for (int it = 0;; ++it) {
             const int item = blockIdx.x + it * gridDim.x;
@@ -496,19 +390,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
     }
 
     // ---------------------------------------------------------------- consumers
-    using Ops = ItemOps<RW, SW, G>;
     const int ctid = tid;
     int* tok = reinterpret_cast<int*>(smem + SL::tok);
     float* wn = reinterpret_cast<float*>(smem + SL::wn);
     int* ridx = reinterpret_cast<int*>(smem + SL::ridx);
     float* rw = reinterpret_cast<float*>(smem + SL::rw);
-    uint2* xh = reinterpret_cast<uint2*>(smem + SL::xh);
-    uint4* xbf = reinterpret_cast<uint4*>(smem + SL::xb);
-    float4* red = reinterpret_cast<float4*>(smem + SL::red);
+    float* acc = reinterpret_cast<float*>(smem + SL::acc);
     __half* ahh = reinterpret_cast<__half*>(smem + SL::ah);
     __nv_bfloat16* abfh = reinterpret_cast<__nv_bfloat16*>(smem + SL::abf);
     const uint2* ah = reinterpret_cast<const uint2*>(smem + SL::ah);
     const uint2* abf = reinterpret_cast<const uint2*>(smem + SL::abf);
+    typename Ops::XF xf;
     float y[TILES_PER_WARP][4];
 #pragma unroll
     for (int j = 0; j < TILES_PER_WARP; ++j) y[j][0] = y[j][1] = y[j][2] = y[j][3] = 0.f;
@@ -516,13 +408,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
     if (small) {
         if (ctid < NTOK) tok[ctid] = ctid < p.T ? ctid : -1;
         consumer_sync();
-        build_x_frags<SL::F16, SL::BF16>(p.x, tok, xh, xbf, ctid);   // visible after the first item's barrier
+        load_x_frags(p.x, tok, warp, lane, xf);
     }
-    int n_items = 0x7fffffff;
+    int n_items = p.shared_only ? n_shared : 0x7fffffff;
     bool waited = false;
     for (int it = 0;; ++it) {
         const int item = blockIdx.x + it * gridDim.x;
-        if (item >= n_shared && !waited) {
+        if (item >= n_shared && !waited && !p.shared_only) {
             pdl_wait();
             waited = true;
             n_items = n_shared + p.R.active[E] * p.L.rg.slices;
@@ -530,7 +422,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
                 ridx[ctid] = p.R.topk_idx[ctid];
                 rw[ctid] = p.R.topk_w[ctid];
             }
-            consumer_sync();
         }
         if (item >= n_items) break;
         const int slot = it % NSLOT;
@@ -551,29 +442,34 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
         const bool routed = expert >= 0;
         const char* sbuf = smem + SL::slots + slot * SLOT_BYTES;
 
-        int ntok = NTOK, seg = 0;
-        if (!small && routed) {
-            ntok = p.R.counts[expert];
-            seg = p.R.offsets[expert];
-        } else if (!small) {
-            ntok = p.T;
-        }
-        for (int b0 = 0; b0 < ntok; b0 += NTOK) {
+        if (small) {
             if (ctid < NTOK) {
                 // routing weight of every column for this item's expert (0 if not routed)
                 float w = 0.f;
-                if (small) {
-                    if (ctid < p.T) {
-                        if (!routed) {
-                            w = 1.f;
-                        } else {
+                if (ctid < p.T) {
+                    if (!routed) {
+                        w = 1.f;
+                    } else {
 #pragma unroll
-                            for (int j = 0; j < K; ++j)
-                                if (ridx[ctid * K + j] == expert) w = rw[ctid * K + j];
-                        }
+                        for (int j = 0; j < K; ++j)
+                            if (ridx[ctid * K + j] == expert) w = rw[ctid * K + j];
                     }
-                } else {
+                }
+                wn[ctid] = w;
+            }
+            Ops::gate_up(routed, sbuf, xf, acc, warp, lane);
+            consumer_sync();
+            Ops::swiglu(routed, acc, ahh, abfh, wn, ctid);
+            consumer_sync();
+            Ops::down(routed, sbuf, ah, abf, warp, lane, y, true);
+        } else {
+            const int ntok = routed ? p.R.counts[expert] : p.T;
+            const int seg = routed ? p.R.offsets[expert] : 0;
+            for (int b0 = 0; b0 < ntok; b0 += NTOK) {
+                consumer_sync();   // the previous group is done with tok / wn
+                if (ctid < NTOK) {
                     int tk = -1;
+                    float w = 0.f;
                     if (b0 + ctid < ntok) {
                         if (!routed) {
                             tk = b0 + ctid;
@@ -585,26 +481,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
                         }
                     }
                     tok[ctid] = tk;
+                    wn[ctid] = w;
                 }
-                wn[ctid] = w;
-            }
-            if (!small) {
                 consumer_sync();
-                build_x_frags<SL::F16, SL::BF16>(p.x, tok, xh, xbf, ctid);
+                load_x_frags(p.x, tok, warp, lane, xf);
+                Ops::gate_up(routed, sbuf, xf, acc, warp, lane);
                 consumer_sync();
-            }
-            Ops::gate_up(routed, sbuf, xh, xbf, red, warp, lane);
-            consumer_sync();
-            Ops::swiglu(routed, red, ahh, abfh, wn, ctid);
-            consumer_sync();
-            if (small) {
-                Ops::down(routed, sbuf, ah, abf, warp, lane, y, true);
-            } else {
+                Ops::swiglu(routed, acc, ahh, abfh, wn, ctid);
+                consumer_sync();
                 Ops::down(routed, sbuf, ah, abf, warp, lane, y, false);
                 if (!waited) {
                     pdl_wait();   // the router zeroes `out` first
                     waited = true;
-                    n_items = n_shared + p.R.active[E] * p.L.rg.slices;
+                    if (!p.shared_only) n_items = n_shared + p.R.active[E] * p.L.rg.slices;
                 }
                 const int gr = lane >> 2, c = lane & 3;
                 const int t0 = tok[2 * c], t1 = tok[2 * c + 1];
@@ -621,9 +510,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
                     }
                 }
             }
-            consumer_sync();
         }
-        if (ctid == 0) mbar_arrive(&empty[slot]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);   // this warp is done with the slot
     }
     if (small && okflag[1] == 0) {
         if (!waited) pdl_wait();   // the router zeroes `out` first
@@ -647,20 +536,18 @@ int g_num_sms = 0;
 
 template <int RW, int SW, int G>
 cudaError_t launch_typed(const ExpertParams& p, cudaStream_t st) {
-    static_assert(blk_bytes_of(RW, G) + DSC_BYTES <= SLOT_BYTES && blk_bytes_of(SW, G) + DSC_BYTES <= SLOT_BYTES,
-                  "item does not fit a ring slot");
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(expert_decode_kernel<RW, SW, G>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SmemLayout<RW, SW>::total);
+                                             (int)SmemLayout<RW, SW, G>::total);
         if (e != cudaSuccess) return e;
         configured = true;
     }
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(g_num_sms);
     cfg.blockDim = dim3(NTHREADS);
-    cfg.dynamicSmemBytes = SmemLayout<RW, SW>::total;
+    cfg.dynamicSmemBytes = SmemLayout<RW, SW, G>::total;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -673,13 +560,13 @@ cudaError_t launch_typed(const ExpertParams& p, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_expert_decode(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
-                                 cudaStream_t st) {
+                                 bool shared_only, cudaStream_t st) {
     if (g_num_sms == 0) {
         int dev = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
     }
-    const ExpertParams p{x, T, out, L, R};
+    const ExpertParams p{x, T, out, L, R, shared_only ? 1 : 0};
     const int rw = L.rg.wtype, sw = L.sg.wtype;
     const int g = is_quant(rw) ? L.rg.group : (is_quant(sw) ? L.sg.group : 128);
 #define FOCR_CASE(A, B, GG) \

@@ -1,0 +1,15 @@
+// Internal launchers for the lm_head GEMV + argmax and the RMSNorm (see lm_head.cu, rmsnorm.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace focr {
+
+size_t lm_head_smem_bytes();
+int lm_head_grid();
+cudaError_t launch_lm_head(const uint4* codes, const float* scales, const float* x, int T, float* logits,
+                           int32_t* argmax, void* ws, cudaStream_t st);
+cudaError_t launch_rmsnorm(const float* x, const float* gamma, int T, float eps, float* out, cudaStream_t st);
+
+}  // namespace focr

@@ -166,7 +166,7 @@ void host_pack_set(const float* gate, const float* up, const float* down, const 
         }
     }
     if (is_quant(wt)) {
-        const int ngd = g.inter / g.group;
+        const int ngd = (g.inter + g.group - 1) / g.group;
         for (int grp = 0; grp < ngd; ++grp)
             for (int h = 0; h < H; ++h) dscale[(size_t)grp * H + h] = qd.s[(size_t)(h * qd.ng + grp)];
     }
@@ -203,7 +203,7 @@ void host_unpack_matrix(const uint8_t* items, const float* dscale, const ItemGeo
         }
     }
     if (which == 2 && is_quant(wt)) {
-        const int ngd = g.inter / g.group;
+        const int ngd = (g.inter + g.group - 1) / g.group;
         for (int grp = 0; grp < ngd; ++grp)
             for (int h = 0; h < H; ++h) s[(int64_t)h * ngd + grp] = dscale[(size_t)grp * H + h];
     }
@@ -220,6 +220,41 @@ void parallel_for(int n, const std::function<void(int)>& fn) {
             for (int i = next++; i < n; i = next++) fn(i);
         });
     for (auto& t : th) t.join();
+}
+
+// lm_head codes: tile r (16 rows), k-step q, lane L = 4 gr + c hold the A-fragment
+// elements e0..e7 of rows 16r+gr, 16r+gr+8 and columns 16q+2c(+1), 16q+2c+8(+9), two
+// k-steps per 16-byte lane vector, offset-binary (q + 128).
+static size_t lm_code_offset(int64_t row, int col) {
+    const int64_t r = row / 16;
+    const int rr = (int)(row % 16);
+    const int gr = rr & 7, hi = rr >> 3;
+    const int q = col / 16, kc = col % 16;
+    const int c = (kc & 7) >> 1, odd = kc & 1, up = kc >> 3;
+    const int L = 4 * gr + c;
+    const int j = odd + 2 * hi + 4 * up;   // inverse of the e0..e7 element order
+    return ((size_t)(r * (KSTEPS / 2) + q / 2) * 32 + L) * 16 + (q % 2) * 8 + j;
+}
+
+void host_pack_lm_head(const float* w, int64_t V, uint8_t* codes, float* scales) {
+    const int64_t tiles = V / 16;
+    parallel_for((int)tiles, [&](int r) {
+        std::vector<int8_t> q(16 * H);
+        host_quantize(w + (size_t)r * 16 * H, 16, H, H, 8, q.data(), scales + (size_t)r * 16);
+        for (int rr = 0; rr < 16; ++rr)
+            for (int col = 0; col < H; ++col)
+                codes[lm_code_offset((int64_t)r * 16 + rr, col)] = (uint8_t)(q[(size_t)rr * H + col] + 128);
+    });
+}
+
+void host_unpack_lm_head(const uint8_t* codes, int64_t V, int8_t* q) {
+    parallel_for((int)(V / 16), [&](int r) {
+        for (int rr = 0; rr < 16; ++rr)
+            for (int col = 0; col < H; ++col) {
+                const int64_t row = (int64_t)r * 16 + rr;
+                q[(size_t)row * H + col] = (int8_t)((int)codes[lm_code_offset(row, col)] - 128);
+            }
+    });
 }
 
 }  // namespace focr

@@ -16,3 +16,10 @@ void host_unpack_matrix(const uint8_t* items, const float* dscale, const ItemGeo
 void parallel_for(int n, const std::function<void(int)>& fn);
 
 }  // namespace focr
+
+namespace focr {
+// lm_head: int8 codes with one scale per row, fragment-order tiles of 16 rows
+// (codes: V * 1280 bytes, scales: V floats)
+void host_pack_lm_head(const float* w, int64_t V, uint8_t* codes, float* scales);
+void host_unpack_lm_head(const uint8_t* codes, int64_t V, int8_t* q);
+}  // namespace focr

@@ -37,6 +37,7 @@ struct RouterParams {
     const uint16_t* wr;
     RouteView R;
     float* out;
+    const float* resid;   // NULL: out starts at zero; else out starts as a copy of resid
 };
 
 __device__ __forceinline__ void warp_argmax(float& v, int& i) {
@@ -144,13 +145,14 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
     pdl_wait();                 // x may come from the previous kernel on the stream
     pdl_launch_dependents();    // let the expert kernel start its routing-free work
 
-    // zero the layer output (the expert kernel adds into it after this grid completes)
+    // initialise the layer output (the expert kernel adds into it after this grid completes)
     {
         const int nblk = gridDim.x;
         float4* o4 = reinterpret_cast<float4*>(p.out);
+        const float4* r4 = reinterpret_cast<const float4*>(p.resid);
         const int n4 = p.T * H / 4;
         for (int i = blockIdx.x * RT_THREADS + tid; i < n4; i += nblk * RT_THREADS)
-            o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            o4[i] = r4 ? r4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
     for (int i = tid; i < TB * KCOLS; i += RT_THREADS) {
@@ -251,8 +253,8 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
 }  // namespace
 
 cudaError_t launch_router(const float* x, int T, int /*T_ws*/, const LayerView& L, const RouteView& R, float* out,
-                          cudaStream_t st) {
-    RouterParams p{x, T, L.router, R, out};
+                          const float* resid, cudaStream_t st) {
+    RouterParams p{x, T, L.router, R, out, resid};
     const int TB = T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : 8));
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(((T + TB - 1) / TB) * RC);
