@@ -35,9 +35,10 @@ namespace focr {
 namespace {
 
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s
-constexpr uint32_t GU_SMEM_BUDGET = 180 * 1024;     // leaves room for a router CTA on the same SM
+constexpr uint32_t GU_SMEM_BUDGET = 200 * 1024;     // leaves room for a small router CTA on the same SM
 constexpr int GU_MAX_WARPS = 16;
 constexpr int DN_WARPS = 8;                         // down kernel: 8 warps, two CTAs per SM
+constexpr int DN_BFRAGS = 16 * 2 * 32;              // B fragments of one chunk (<= 16 slices x 2 steps)
 
 struct SmallParams {
     const float* x;
@@ -54,20 +55,33 @@ __device__ __forceinline__ int gu_tile_base(bool routed, int a) { return routed 
 __device__ __forceinline__ int a16_base(bool routed, int a) { return routed ? IS_MAX / 16 + a * (I / 16) : 0; }
 __device__ __forceinline__ int abf_base(bool routed, int a) { return routed ? IS_MAX / 8 + a * (I / 8) : 0; }
 
-// x of the batch in B-fragment order, fp32: xs[q][lane] = columns 16q+2c, +1, +8, +9 of
-// token n (lane = 4n + c), zero for n >= T.  Both the f16 and the bf16 hi/lo operands
-// are formed from it at use.
-__device__ __forceinline__ void build_xs(const float* x, int T, float4* xs, int nthreads) {
-    for (int i = threadIdx.x; i < KSTEPS * 32; i += nthreads) {
+// x of the batch in B-fragment order: for k-step q and lane = 4n + c, columns 16q+2c, +1,
+// +8, +9 of token n (zero for n >= T) -- as f16 pairs (xh, the quantised sets' operand)
+// and/or fp32 (xs, split into bf16 hi + lo at use by the bf16 sets).  All loads of a
+// thread are issued before its stores.
+template <int NT, bool F16, bool F32>
+__device__ __forceinline__ void build_x(const float* x, int T, uint2* xh, float4* xs) {
+    constexpr int PER = (KSTEPS * 32 + NT - 1) / NT;
+    float4 v[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        const int i = threadIdx.x + k * NT;
         const int q = i >> 5, ln = i & 31, n = ln >> 2, c = ln & 3;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (n < T) {
+        v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < KSTEPS * 32 && n < T) {
             const float* row = x + (size_t)n * H + 16 * q + 2 * c;
             const float2 lo = __ldg(reinterpret_cast<const float2*>(row));
             const float2 hi = __ldg(reinterpret_cast<const float2*>(row + 8));
-            v = make_float4(lo.x, lo.y, hi.x, hi.y);
+            v[k] = make_float4(lo.x, lo.y, hi.x, hi.y);
         }
-        xs[i] = v;
+    }
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        const int i = threadIdx.x + k * NT;
+        if (i < KSTEPS * 32) {
+            if constexpr (F16) xh[i] = make_uint2(f32x2_to_f16x2(v[k].x, v[k].y), f32x2_to_f16x2(v[k].z, v[k].w));
+            if constexpr (F32) xs[i] = v[k];
+        }
     }
 }
 
@@ -95,9 +109,14 @@ __device__ __forceinline__ float2 route_w(const RouteView& R, int T, int expert,
 // ------------------------------------------------------------------ gate/up units
 // A unit is one tile (8 gate rows over the 8 matching up rows) over QN of the 80 k-steps:
 // all of them for int4, halves for int8, quarters for bf16 -- 10 KB of codes either way.
-template <int W, int G>
+template <int W>
+constexpr int gu_parts() {   // column parts of a unit
+    return W == FOCR_W_INT4 ? 1 : (W == FOCR_W_INT8 ? 2 : 4);
+}
+
+template <int W, int G, int PARTS = gu_parts<W>()>
 struct GuUnit {
-    static constexpr int KP = W == FOCR_W_INT4 ? 1 : (W == FOCR_W_INT8 ? 2 : 4);   // column parts
+    static constexpr int KP = PARTS;
     static constexpr int QN = KSTEPS / KP;                 // k-steps per unit
     static constexpr int KPV = ksteps_per_vec(W);          // k-steps per 16-byte lane vector
     static constexpr int NV = QN / KPV;                    // lane vectors per unit (20)
@@ -112,37 +131,51 @@ template <int RW, int SW, int G>
 struct GuCfg {
     using RU = GuUnit<RW, G>;
     using SU = GuUnit<SW, G>;
+    static constexpr bool F16 = is_quant(RW) || is_quant(SW);    // x as f16 B fragments
+    static constexpr bool F32 = !is_quant(RW) || !is_quant(SW);  // x in fp32 (bf16 hi/lo split at use)
     static constexpr uint32_t BUF = ((RU::BYTES > SU::BYTES ? RU::BYTES : SU::BYTES) + 127u) & ~127u;
-    static constexpr uint32_t XS_BYTES = (uint32_t)KSTEPS * 32 * 16;
-    static constexpr int NW_FIT = (int)((GU_SMEM_BUDGET - XS_BYTES - 256u) / BUF);
+    static constexpr uint32_t xh = 0;                                           // [80][32] uint2
+    static constexpr uint32_t xs = xh + (F16 ? (uint32_t)KSTEPS * 32 * 8 : 0u);  // [80][32] float4
+    static constexpr uint32_t bufs = xs + (F32 ? (uint32_t)KSTEPS * 32 * 16 : 0u);
+    static constexpr int NW_FIT = (int)((GU_SMEM_BUDGET - bufs - 256u) / BUF);
     static constexpr int NW = NW_FIT < GU_MAX_WARPS ? NW_FIT : GU_MAX_WARPS;
-    static constexpr uint32_t bufs = XS_BYTES;
     static constexpr uint32_t bars = bufs + (uint32_t)NW * BUF;
     static constexpr uint32_t total = bars + (uint32_t)NW * 8;
+    static_assert(xs % 16 == 0 && bufs % 128 == 0 && BUF % 128 == 0 && bars % 8 == 0, "region alignment");
     static_assert(NW >= 4, "shared memory budget");
 };
 
 // [g; u] partial sums of one unit: tot[0], tot[1] = gate row gr of tokens 2c, 2c+1;
 // tot[2], tot[3] = the up row.  int4/int8 codes become exact f16 A fragments and each
 // scale group's fp32 sum is scaled; bf16 weights meet x's bf16 hi and lo parts.
-template <int W, int G>
-__device__ __forceinline__ void gu_compute(const char* buf, const float4* xs, int q0, int lane, float (&tot)[4]) {
-    using U = GuUnit<W, G>;
+template <int W, int G, int PARTS = gu_parts<W>()>
+__device__ __forceinline__ void gu_compute(const char* buf, const uint2* xh, const float4* xs, int q0, int lane,
+                                           float (&tot)[4]) {
+    using U = GuUnit<W, G, PARTS>;
     if constexpr (!is_quant(W)) {
-#pragma unroll 5
-        for (int v = 0; v < U::NV; ++v) {
-            const uint4 a = lds128(buf + (v * 32 + lane) * 16);
-            const float4 xv = lds128f(xs + (q0 + v) * 32 + lane);
-            const uint2 l = split_bf16x2(xv.x, xv.y), h = split_bf16x2(xv.z, xv.w);
-            mma16816_bf16(tot, a, l.x, h.x);   // x hi
-            mma16816_bf16(tot, a, l.y, h.y);   // x lo
+        // four independent accumulators (hi/lo x even/odd k-step) keep the MMA pipe busy
+        float acc[4][4] = {};
+#pragma unroll 4
+        for (int v = 0; v < U::NV; v += 2) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 a = lds128(buf + ((v + h) * 32 + lane) * 16);
+                const float4 xv = lds128f(xs + (q0 + v + h) * 32 + lane);
+                const uint2 l = split_bf16x2(xv.x, xv.y), hh = split_bf16x2(xv.z, xv.w);
+                mma16816_bf16(acc[2 * h], a, l.x, hh.x);       // x hi
+                mma16816_bf16(acc[2 * h + 1], a, l.y, hh.y);   // x lo
+            }
         }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) tot[r] = (acc[0][r] + acc[1][r]) + (acc[2][r] + acc[3][r]);
     } else {
-        constexpr int QPG = G / 16;          // k-steps per scale group
-        constexpr int VB = 4;                // vectors per loop step: whole scale groups
-        static_assert((VB * U::KPV) % QPG == 0 && U::NV % VB == 0, "loop step holds whole groups");
+        // each scale group's sum is built in two accumulators (even / odd k-steps; the first
+        // MMA of each starts from zero), then scaled into tot
+        constexpr int QPG = G / 16;                  // k-steps per scale group (>= 2)
+        constexpr int VB = U::NV % 4 == 0 ? 4 : 2;   // vectors per loop step: whole scale groups
+        static_assert(QPG >= 2 && (VB * U::KPV) % QPG == 0 && U::NV % VB == 0, "loop step holds whole groups");
         const float2* sc = reinterpret_cast<const float2*>(buf + U::W_BYTES) + (lane >> 2);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        float acc[2][4];
 #pragma unroll 1
         for (int v0 = 0; v0 < U::NV; v0 += VB) {
 #pragma unroll
@@ -156,15 +189,15 @@ __device__ __forceinline__ void gu_compute(const char* buf, const float4* xs, in
                     Frag4 a;
                     if constexpr (W == FOCR_W_INT4) a = dq_int4(wr[j]);
                     else a = dq_int8(wr[2 * j], wr[2 * j + 1]);
-                    const float4 xv = lds128f(xs + (q0 + ql) * 32 + lane);
-                    mma16816(acc, a, f32x2_to_f16x2(xv.x, xv.y), f32x2_to_f16x2(xv.z, xv.w));
+                    const uint2 xb = xh[(q0 + ql) * 32 + lane];
+                    if (qq % QPG < 2) mma16816_zc(acc[qq & 1], a, xb.x, xb.y);
+                    else mma16816(acc[qq & 1], a, xb.x, xb.y);
                     if ((qq + 1) % QPG == 0) {
                         const float2 s = sc[(ql / QPG) * 8];
-                        tot[0] = fmaf(acc[0], s.x, tot[0]);
-                        tot[1] = fmaf(acc[1], s.x, tot[1]);
-                        tot[2] = fmaf(acc[2], s.y, tot[2]);
-                        tot[3] = fmaf(acc[3], s.y, tot[3]);
-                        acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+                        tot[0] = fmaf(acc[0][0] + acc[1][0], s.x, tot[0]);
+                        tot[1] = fmaf(acc[0][1] + acc[1][1], s.x, tot[1]);
+                        tot[2] = fmaf(acc[0][2] + acc[1][2], s.y, tot[2]);
+                        tot[3] = fmaf(acc[0][3] + acc[1][3], s.y, tot[3]);
                     }
                 }
             }
@@ -198,20 +231,28 @@ __device__ __forceinline__ void store_a(const RouteView& R, bool routed, int a_s
     }
 }
 
-// One gate/up unit of a warp: bulk-copy its codes (and scale groups) into the warp's
-// buffer, prefetch the slice's down-projection bytes into L2 (first unit of a slice),
-// compute, and either apply SwiGLU (whole rows) or add into the tile's sums, the last of
-// the KP parts applying it.  Returns false if the copy did not complete in time.
-template <int W, int G>
-__device__ __forceinline__ bool gu_unit(const SmallParams& p, bool routed, int a_slot, int expert, int u, char* buf,
-                                        uint64_t* bar, uint32_t& phase, const float4* xs, int lane, uint64_t pol) {
-    using U = GuUnit<W, G>;
+// One gate/up unit of a warp, in two halves.  gu_issue bulk-copies its codes (and scale
+// groups) into the warp's buffer and, for the first unit of a slice, prefetches the
+// slice's down-projection bytes into L2.  gu_finish waits for the copy, computes, and
+// either applies SwiGLU (whole rows) or adds into the tile's sums, the last of the KP
+// parts applying it.  gu_finish returns false if the copy did not complete in time.
+template <int W, int G, int PARTS = gu_parts<W>()>
+__device__ __forceinline__ const uint8_t* gu_block(const SmallParams& p, bool routed, int expert, int u) {
     constexpr int S = slice_rows(W);
     const ItemGeom& g = routed ? p.L.rg : p.L.sg;
-    const int ti = u / U::KP, part = u % U::KP;   // set-local tile, column part
+    const int s = (u / PARTS) / (S / 8);
+    return (routed ? p.L.routed_items + (size_t)expert * g.slices * g.item_bytes : p.L.shared_items) +
+           (size_t)s * g.item_bytes;
+}
+
+template <int W, int G, int PARTS = gu_parts<W>()>
+__device__ __forceinline__ void gu_issue(const SmallParams& p, bool routed, int expert, int u, char* buf,
+                                         uint64_t* bar, int lane, uint64_t pol) {
+    using U = GuUnit<W, G, PARTS>;
+    constexpr int S = slice_rows(W);
+    const int ti = u / U::KP, part = u % U::KP;
     const int s = ti / (S / 8), t = ti % (S / 8);
-    const uint8_t* blk = (routed ? p.L.routed_items + (size_t)expert * g.slices * g.item_bytes : p.L.shared_items) +
-                         (size_t)s * g.item_bytes;
+    const uint8_t* blk = gu_block<W, G, PARTS>(p, routed, expert, u);
     __syncwarp();   // every lane is done with the previous unit's buffer
     if (lane == 0) {
         mbar_arrive_expect_tx(bar, U::BYTES);
@@ -222,10 +263,19 @@ __device__ __forceinline__ bool gu_unit(const SmallParams& p, bool routed, int a
     } else if (lane == 1 && t == 0 && part == 0) {
         bulk_prefetch_l2(blk + gu_w_bytes_of(W) + gu_s_bytes_of(W, G), d_w_bytes_of());
         if (is_quant(W) && (s * S) % G == 0) {
+            const ItemGeom& g = routed ? p.L.rg : p.L.sg;
             const float* dsc = routed ? p.L.routed_dscale + (size_t)expert * g.dscale_expert_floats : p.L.shared_dscale;
             bulk_prefetch_l2(dsc + (size_t)(s * S / G) * H, H * 4);
         }
     }
+}
+
+template <int W, int G>
+__device__ __forceinline__ bool gu_finish(const SmallParams& p, bool routed, int a_slot, int expert, int u,
+                                          const char* buf, uint64_t* bar, uint32_t& phase, const uint2* xh,
+                                          const float4* xs, int lane) {
+    using U = GuUnit<W, G>;
+    const int ti = u / U::KP, part = u % U::KP;
     const float2 wr = routed ? route_w(p.R, p.T, expert, lane & 3) : make_float2(1.f, 1.f);
     const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar, phase, WAIT_LIMIT_NS));
     phase ^= 1u;
@@ -235,7 +285,7 @@ __device__ __forceinline__ bool gu_unit(const SmallParams& p, bool routed, int a
         return false;
     }
     float tot[4] = {0.f, 0.f, 0.f, 0.f};
-    gu_compute<W, G>(buf, xs, part * U::QN, lane, tot);
+    gu_compute<W, G>(buf, xh, xs, part * U::QN, lane, tot);
     if constexpr (U::KP == 1) {
         store_a<W>(p.R, routed, a_slot, ti, lane, tot, wr);
     } else {
@@ -261,30 +311,36 @@ __device__ __forceinline__ bool gu_unit(const SmallParams& p, bool routed, int a
 
 // Warps are ranked across SMs first (rho = warp * grid + block) so that both the
 // shared-set units, which take the low ranks, and the routed units, which take the high
-// ranks, spread over every SM.
+// ranks, spread over every SM.  A warp's first shared unit is in flight while x is staged.
 template <int RW, int SW, int G>
 __global__ void __launch_bounds__(GuCfg<RW, SW, G>::NW * 32, 2) decode_gu_kernel(SmallParams p) {
     using C = GuCfg<RW, SW, G>;
     extern __shared__ __align__(128) char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const float4* xs = reinterpret_cast<const float4*>(smem);
+    const uint2* xh = reinterpret_cast<const uint2*>(smem + C::xh);
+    const float4* xs = reinterpret_cast<const float4*>(smem + C::xs);
     char* buf = smem + C::bufs + warp * C::BUF;
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::bars) + warp;
+    const int nwt = gridDim.x * C::NW;
+    const int rho = warp * gridDim.x + blockIdx.x;
+    const uint64_t pol = policy_evict_first();
+    const int s_units = (p.L.sg.inter / 8) * C::SU::KP;
     if (lane == 0) {
         mbar_init(bar, 1);
         fence_barrier_init();
     }
-    build_xs(p.x, p.T, reinterpret_cast<float4*>(smem), C::NW * 32);
+    __syncwarp();
+    if (rho < s_units) gu_issue<SW, G>(p, false, -1, rho, buf, bar, lane, pol);
+    build_x<C::NW * 32, C::F16, C::F32>(p.x, p.T, reinterpret_cast<uint2*>(smem + C::xh),
+                                         reinterpret_cast<float4*>(smem + C::xs));
     __syncthreads();
 
-    const int nwt = gridDim.x * C::NW;
-    const int rho = warp * gridDim.x + blockIdx.x;
-    const uint64_t pol = policy_evict_first();
     uint32_t phase = 0;
     bool ok = true;
-    const int s_units = (p.L.sg.inter / 8) * C::SU::KP;
-    for (int u = rho; ok && u < s_units; u += nwt)
-        ok = gu_unit<SW, G>(p, false, 0, -1, u, buf, bar, phase, xs, lane, pol);
+    for (int u = rho; ok && u < s_units; u += nwt) {
+        if (u != rho) gu_issue<SW, G>(p, false, -1, u, buf, bar, lane, pol);
+        ok = gu_finish<SW, G>(p, false, 0, -1, u, buf, bar, phase, xh, xs, lane);
+    }
     pdl_wait();                 // the router's selection is complete and visible
     pdl_launch_dependents();    // the down kernel may read it from now on
     if (p.shared_only || !ok) return;
@@ -292,7 +348,9 @@ __global__ void __launch_bounds__(GuCfg<RW, SW, G>::NW * 32, 2) decode_gu_kernel
     const int r_units = p.R.active[E] * per_expert;
     for (int r = nwt - 1 - rho; ok && r < r_units; r += nwt) {
         const int a = r / per_expert;
-        ok = gu_unit<RW, G>(p, true, a, p.R.active[a], r % per_expert, buf, bar, phase, xs, lane, pol);
+        const int e = p.R.active[a];
+        gu_issue<RW, G>(p, true, e, r % per_expert, buf, bar, lane, pol);
+        ok = gu_finish<RW, G>(p, true, a, e, r % per_expert, buf, bar, phase, xh, xs, lane);
     }
 }
 
@@ -303,72 +361,90 @@ __global__ void __launch_bounds__(GuCfg<RW, SW, G>::NW * 32, 2) decode_gu_kernel
 template <int W, int G>
 struct DownUnit {
     static constexpr int S = slice_rows(W);
-    static constexpr int CH = (W == FOCR_W_INT4 && G == 32) ? 8 : 16;    // slices per chunk
+    // slices per chunk (int4 g64: 14, so an expert's 28 slices make two equal chunks)
+    static constexpr int CH = W == FOCR_W_INT4 ? (G == 32 ? 8 : (G == 64 ? 14 : 16)) : 16;
     static constexpr int SPG = is_quant(W) ? (G / S < CH ? G / S : CH) : CH;   // slices per scale group
     static constexpr int NGC = CH / SPG;                                  // scale groups per chunk
     static constexpr int BPS = W == FOCR_W_INT4 ? 2 : 1;                  // B fragments (uint2) per slice
     static_assert(!is_quant(W) || (CH * S) % G == 0, "chunks hold whole scale groups");
 };
 
+// A loads (codes, and scale groups) of one unit: independent of the gate/up kernel, so a
+// warp's first unit issues them before waiting on that kernel
 template <int W, int G>
-__device__ __forceinline__ void down_unit(const uint8_t* items, const ItemGeom& g, const float* dsc, const uint2* bfr,
-                                          int chunk, int m, int T, float* out, int lane) {
+struct DownA {
+    uint2 v[DownUnit<W, G>::CH];
+    float sc[is_quant(W) ? DownUnit<W, G>::NGC : 1][2];
+    int ns;
+};
+
+template <int W, int G>
+__device__ __forceinline__ void down_load(const uint8_t* items, const ItemGeom& g, const float* dsc, int chunk, int m,
+                                          int lane, DownA<W, G>& A) {
     using D = DownUnit<W, G>;
-    constexpr int CH = D::CH;
-    const int gr = lane >> 2, c = lane & 3;
-    const int s0 = chunk * CH;
-    const int ns = min(CH, g.slices - s0);
+    const int s0 = chunk * D::CH;
+    A.ns = min(D::CH, g.slices - s0);
     const uint8_t* dw = items + (size_t)s0 * g.item_bytes + gu_w_bytes_of(W) + gu_s_bytes_of(W, G) + (m * 32 + lane) * 8;
-    uint2 v[CH];
 #pragma unroll
-    for (int j = 0; j < CH; ++j) v[j] = j < ns ? ldg_nc2(dw + (size_t)j * g.item_bytes) : make_uint2(0u, 0u);
-    float sc[is_quant(W) ? D::NGC : 1][2];
+    for (int j = 0; j < D::CH; ++j) A.v[j] = j < A.ns ? ldg_nc2(dw + (size_t)j * g.item_bytes) : make_uint2(0u, 0u);
     if constexpr (is_quant(W)) {
 #pragma unroll
         for (int jg = 0; jg < D::NGC; ++jg) {
-            sc[jg][0] = sc[jg][1] = 0.f;
-            if (jg * D::SPG < ns) {
-                const float* r = dsc + (size_t)((s0 + jg * D::SPG) * D::S / G) * H + 16 * m + gr;
-                sc[jg][0] = __ldg(r);
-                sc[jg][1] = __ldg(r + 8);
+            A.sc[jg][0] = A.sc[jg][1] = 0.f;
+            if (jg * D::SPG < A.ns) {
+                const float* r = dsc + (size_t)((s0 + jg * D::SPG) * D::S / G) * H + 16 * m + (lane >> 2);
+                A.sc[jg][0] = __ldg(r);
+                A.sc[jg][1] = __ldg(r + 8);
             }
         }
     }
+}
+
+// B fragments of a (written by the gate/up kernel), the MMAs (two independent accumulators),
+// the group scales, and the atomic adds into the output rows 16m .. 16m+15
+template <int W, int G>
+__device__ __forceinline__ void down_finish(const DownA<W, G>& A, const uint2* bsm, int m, int T, float* out,
+                                            int lane) {
+    using D = DownUnit<W, G>;
+    constexpr int CH = D::CH;
+    const int gr = lane >> 2, c = lane & 3;
     uint2 b[CH][D::BPS];
 #pragma unroll
     for (int j = 0; j < CH; ++j)
 #pragma unroll
         for (int h = 0; h < D::BPS; ++h)
-            b[j][h] = j < ns ? bfr[((s0 + j) * D::BPS + h) * 32 + lane] : make_uint2(0u, 0u);
+            b[j][h] = j < A.ns ? bsm[(j * D::BPS + h) * 32 + lane] : make_uint2(0u, 0u);
 
     float y[4] = {0.f, 0.f, 0.f, 0.f};
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[2][4] = {};
 #pragma unroll
     for (int j = 0; j < CH; ++j) {
-        if (j < ns) {
+        if (j < A.ns) {
             if constexpr (W == FOCR_W_INT4) {
-                mma16816(acc, dq_int4(v[j].x), b[j][0].x, b[j][0].y);
-                mma16816(acc, dq_int4(v[j].y), b[j][1].x, b[j][1].y);
+                mma16816(acc[0], dq_int4(A.v[j].x), b[j][0].x, b[j][0].y);
+                mma16816(acc[1], dq_int4(A.v[j].y), b[j][1].x, b[j][1].y);
             } else if constexpr (W == FOCR_W_INT8) {
-                mma16816(acc, dq_int8(v[j].x, v[j].y), b[j][0].x, b[j][0].y);
+                mma16816(acc[j & 1], dq_int8(A.v[j].x, A.v[j].y), b[j][0].x, b[j][0].y);
             } else {
-                mma1688_bf16(acc, v[j].x, v[j].y, b[j][0].x);   // a hi
-                mma1688_bf16(acc, v[j].x, v[j].y, b[j][0].y);   // a lo
+                mma1688_bf16(acc[0], A.v[j].x, A.v[j].y, b[j][0].x);   // a hi
+                mma1688_bf16(acc[1], A.v[j].x, A.v[j].y, b[j][0].y);   // a lo
             }
         }
         if constexpr (is_quant(W)) {
             if ((j + 1) % D::SPG == 0) {
                 const int jg = j / D::SPG;
-                y[0] = fmaf(acc[0], sc[jg][0], y[0]);
-                y[1] = fmaf(acc[1], sc[jg][0], y[1]);
-                y[2] = fmaf(acc[2], sc[jg][1], y[2]);
-                y[3] = fmaf(acc[3], sc[jg][1], y[3]);
-                acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+                y[0] = fmaf(acc[0][0] + acc[1][0], A.sc[jg][0], y[0]);
+                y[1] = fmaf(acc[0][1] + acc[1][1], A.sc[jg][0], y[1]);
+                y[2] = fmaf(acc[0][2] + acc[1][2], A.sc[jg][1], y[2]);
+                y[3] = fmaf(acc[0][3] + acc[1][3], A.sc[jg][1], y[3]);
+#pragma unroll
+                for (int k = 0; k < 2; ++k) acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
             }
         }
     }
     if constexpr (!is_quant(W)) {
-        y[0] = acc[0]; y[1] = acc[1]; y[2] = acc[2]; y[3] = acc[3];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) y[r] = acc[0][r] + acc[1][r];
     }
     const int row = 16 * m + gr;
     if (2 * c < T) {
@@ -381,38 +457,84 @@ __device__ __forceinline__ void down_unit(const uint8_t* items, const ItemGeom& 
     }
 }
 
-// Units: the shared set's (chunk, tile) pairs, then every selected expert's; consecutive
-// warps of a CTA take consecutive output tiles of one chunk, so they read the same a
-// fragments.
+// One step of a CTA: its 8 warps take 8 consecutive output tiles of one chunk of one set.
+// Each warp loads its A codes and scales; on the first step the CTA then waits on the
+// gate/up kernel; one thread bulk-copies the chunk's B fragments of a (contiguous in the
+// workspace) into shared memory for all eight warps.  Returns false if that copy did not
+// complete in time.
+template <int W, int G>
+__device__ __forceinline__ bool down_step(const SmallParams& p, const uint8_t* items, const ItemGeom& g,
+                                          const float* dsc, const uint2* bset, int chunk, int m, bool first,
+                                          uint2* bsm, uint64_t* bar, uint32_t& phase, int lane) {
+    using D = DownUnit<W, G>;
+    DownA<W, G> A;
+    down_load<W, G>(items, g, dsc, chunk, m, lane, A);
+    if (first) pdl_wait();
+    __syncthreads();   // the previous step's readers are done with bsm
+    if (threadIdx.x == 0) {
+        const uint32_t bytes = (uint32_t)A.ns * D::BPS * 256u;
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(bsm, bset + (size_t)chunk * D::CH * D::BPS * 32, bytes, bar, policy_evict_first());
+    }
+    // the verdict is CTA-uniform, so every warp leaves the step loop together
+    const bool ok = __syncthreads_and(mbar_wait_bounded(bar, phase, WAIT_LIMIT_NS)) != 0;
+    phase ^= 1u;
+    if (!ok) {
+        if (threadIdx.x == 0) atomicExch(&p.R.ctrl[CTRL_ERROR], DEVERR_FULL_WAIT);
+        (void)mbar_wait_bounded(bar, phase ^ 1u, WAIT_LIMIT_NS);   // never leave the copy in flight
+        return false;
+    }
+    down_finish<W, G>(A, bsm, m, p.T, p.out, lane);
+    return true;
+}
+
+// Units: the shared set's (chunk, tile) pairs, then every selected expert's, 80 output
+// tiles per chunk; the 8 warps of a CTA take 8 consecutive units, which share the chunk
+// (80, the number of units per chunk and the totals are multiples of 8, so the loop is
+// uniform over the CTA).  This grid is scheduled only after every gate/up CTA has passed
+// its own wait on the router, so the expert list is final and can be read (from L2)
+// before this grid's wait; the codes of a CTA's first step are then in flight while the
+// gate/up kernel finishes.
 template <int RW, int SW, int G>
 __global__ void __launch_bounds__(DN_WARPS * 32, 2) decode_down_kernel(SmallParams p) {
     using DR = DownUnit<RW, G>;
     using DS = DownUnit<SW, G>;
+    __shared__ __align__(128) uint2 bsm[DN_BFRAGS];
+    __shared__ uint64_t bar;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    pdl_wait();   // a fragments of the gate/up kernel (and, through it, the router's output)
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    pdl_launch_dependents();   // the next forward's router may launch; it waits for this grid
     const int nwt = gridDim.x * DN_WARPS;
-    const int gw = blockIdx.x * DN_WARPS + warp;
     const int nch_s = (p.L.sg.slices + DS::CH - 1) / DS::CH;
     const int nch_r = (p.L.rg.slices + DR::CH - 1) / DR::CH;
     const int n_s = OTILES * nch_s;
     const int per_expert = OTILES * nch_r;
-    const int total = n_s + (p.shared_only ? 0 : p.R.active[E] * per_expert);
+    const int total = n_s + (p.shared_only ? 0 : __ldcg(&p.R.active[E]) * per_expert);
     const uint2* bs = is_quant(SW) ? p.R.a16 : p.R.abf;
     const uint2* br = is_quant(RW) ? p.R.a16 : p.R.abf;
-    for (int u = gw; u < total; u += nwt) {
+    uint32_t phase = 0;
+    bool first = true, ok = true;
+    for (int base = blockIdx.x * DN_WARPS; ok && base < total; base += nwt) {
+        const int u = base + warp;
         if (u < n_s) {
-            down_unit<SW, G>(p.L.shared_items, p.L.sg, p.L.shared_dscale, bs, u / OTILES, u % OTILES, p.T, p.out, lane);
+            ok = down_step<SW, G>(p, p.L.shared_items, p.L.sg, p.L.shared_dscale, bs, u / OTILES, u % OTILES, first,
+                                  bsm, &bar, phase, lane);
         } else {
             const int r = u - n_s;
             const int a = r / per_expert, rem = r % per_expert;
-            const int e = p.R.active[a];
+            const int e = __ldcg(&p.R.active[a]);
             const ItemGeom& g = p.L.rg;
-            down_unit<RW, G>(p.L.routed_items + (size_t)e * g.slices * g.item_bytes, g,
-                             p.L.routed_dscale + (size_t)e * g.dscale_expert_floats,
-                             br + (size_t)(is_quant(RW) ? a16_base(true, a) : abf_base(true, a)) * 32, rem / OTILES,
-                             rem % OTILES, p.T, p.out, lane);
+            ok = down_step<RW, G>(p, p.L.routed_items + (size_t)e * g.slices * g.item_bytes, g,
+                                  p.L.routed_dscale + (size_t)e * g.dscale_expert_floats,
+                                  br + (size_t)(is_quant(RW) ? a16_base(true, a) : abf_base(true, a)) * 32,
+                                  rem / OTILES, rem % OTILES, first, bsm, &bar, phase, lane);
         }
+        first = false;
     }
+    if (first) pdl_wait();   // every CTA waits before exiting (keeps the chain of forwards ordered)
 }
 
 int g_sms = 0;
@@ -424,6 +546,14 @@ cudaError_t launch_small_typed(const SmallParams& p, cudaStream_t st) {
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(decode_gu_kernel<RW, SW, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)C::total);
+        if (e != cudaSuccess) return e;
+        // the whole unified L1 as shared memory for all kernels of the path, so an SM never
+        // has to change its split between consecutive kernels
+        e = cudaFuncSetAttribute(decode_gu_kernel<RW, SW, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(decode_down_kernel<RW, SW, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         configured = true;
     }

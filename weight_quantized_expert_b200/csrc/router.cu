@@ -30,6 +30,7 @@ constexpr int RC = ROUTER_KSPLIT;         // CTAs per cluster
 constexpr int KCOLS = H / RC;             // 160 columns per CTA
 constexpr int PART_COLS = KCOLS / 4;      // 40 columns per thread
 constexpr int NVEC = PART_COLS / 8;       // 5 vectors of 8 bf16
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s
 
 struct RouterParams {
     const float* x;
@@ -40,16 +41,57 @@ struct RouterParams {
     const float* resid;   // NULL: out starts at zero; else out starts as a copy of resid
 };
 
-__device__ __forceinline__ void warp_argmax(float& v, int& i) {
+// counts / offsets / active list / stable permutation of n = T*6 <= 64 entries, by one warp.
+// Lane l owns experts 2l, 2l+1 and entries l, l+32.  An entry's place within its expert's
+// segment = entries before it with the same expert: lanes holding equal experts find each
+// other with __match_any_sync, and entries 32.. add the count among entries 0..31.
+__device__ void dispatch_small(const RouterParams& p, const int* sidx, int* cnt) {
+    const int lane = threadIdx.x & 31;
+    const int n = p.T * K;
+    const unsigned lt = (1u << lane) - 1u;
+    const int ea = lane < n ? sidx[lane] : -1 - lane;            // distinct negatives never match
+    const int eb = lane + 32 < n ? sidx[lane + 32] : -1 - lane;
+    cnt[2 * lane] = 0;
+    cnt[2 * lane + 1] = 0;
+    const unsigned ma = __match_any_sync(0xffffffffu, ea);
+    const unsigned mb = __match_any_sync(0xffffffffu, eb);
+    __syncwarp();
+    if (ea >= 0 && (ma & lt) == 0) cnt[ea] = __popc(ma);         // first lane of each group
+    __syncwarp();
+    const int ra = __popc(ma & lt);
+    const int rb = (eb >= 0 ? cnt[eb] : 0) + __popc(mb & lt);    // entries 0..31 come first
+    __syncwarp();
+    if (eb >= 0 && (mb & lt) == 0) cnt[eb] += __popc(mb);
+    __syncwarp();
+    const int c0 = cnt[2 * lane], c1 = cnt[2 * lane + 1];
+    int incl = c0 + c1;
+    const int h0 = c0 > 0, h1 = c1 > 0;
+    int hincl = h0 + h1;
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, v, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, i, o);
-        if (ov > v || (ov == v && oi < i)) {
-            v = ov;
-            i = oi;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        const int hv = __shfl_up_sync(0xffffffffu, hincl, o);
+        if (lane >= o) {
+            incl += v;
+            hincl += hv;
         }
     }
+    const int ex0 = incl - c0 - c1;
+    p.R.counts[2 * lane] = c0;
+    p.R.counts[2 * lane + 1] = c1;
+    p.R.offsets[2 * lane] = ex0;
+    p.R.offsets[2 * lane + 1] = ex0 + c0;
+    if (lane == 31) p.R.offsets[E] = incl;
+    int pos = hincl - h0 - h1;
+    if (h0) p.R.active[pos++] = 2 * lane;
+    if (h1) p.R.active[pos] = 2 * lane + 1;
+    if (lane == 31) p.R.active[E] = hincl;
+    // offsets of the experts of this lane's entries, from their owning lanes
+    const int sa = ea >= 0 ? ea : 0, sb = eb >= 0 ? eb : 0;
+    const int oa0 = __shfl_sync(0xffffffffu, ex0, sa >> 1), oa1 = __shfl_sync(0xffffffffu, ex0 + c0, sa >> 1);
+    const int ob0 = __shfl_sync(0xffffffffu, ex0, sb >> 1), ob1 = __shfl_sync(0xffffffffu, ex0 + c0, sb >> 1);
+    if (ea >= 0) p.R.perm[((sa & 1) ? oa1 : oa0) + ra] = lane;
+    if (eb >= 0) p.R.perm[((sb & 1) ? ob1 : ob0) + rb] = lane + 32;
 }
 
 // counts / offsets / active list / stable permutation of the T*6 entries (idx: shared or global)
@@ -120,8 +162,10 @@ template <int TB>
 __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_kernel(RouterParams p) {
     cg::cluster_group cluster = cg::this_cluster();
     __shared__ double part_s[RC][TB][E];     // filled in CTA 0 by all CTAs of the cluster
+    __shared__ __align__(8) uint64_t pbar;   // CTA 0: completes when the seven remote partials landed
     __shared__ double xs[TB][KCOLS];
-    __shared__ float lg[TB][E];
+    __shared__ __align__(16) float lg[TB][E];
+    __shared__ float smax[TB], sden[TB];
     __shared__ int sidx[TB * K];
     __shared__ int flag;
     __shared__ int cnt[E];
@@ -138,22 +182,25 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
     // router weights are layer constants: fetch them before waiting on the previous kernel
     const int e = tid >> 2, part = tid & 3;
     const uint16_t* wrow = p.wr + (size_t)e * H + k0 + part * PART_COLS;
+    // (kept in L2 with priority: 164 KB per layer, read by every forward)
+    const uint64_t keep = policy_evict_last();
     uint4 wv[NVEC];
 #pragma unroll
-    for (int v = 0; v < NVEC; ++v) wv[v] = __ldg(reinterpret_cast<const uint4*>(wrow + 8 * v));
+    for (int v = 0; v < NVEC; ++v) wv[v] = ldg_policy(wrow + 8 * v, keep);
+
+    // CTA 0's partial-logit barrier is initialised and armed for the seven remote CTAs'
+    // bytes before any of them can write (one cluster barrier, before the wait on the
+    // previous kernel, so it is off the critical path)
+    constexpr uint32_t REMOTE_BYTES = (RC - 1) * TB * E * sizeof(double);
+    if (r == 0 && tid == 0) {
+        mbar_init(&pbar, 1);
+        mbar_arrive_expect_tx(&pbar, REMOTE_BYTES);
+        fence_barrier_init();
+    }
+    cluster.sync();
 
     pdl_wait();                 // x may come from the previous kernel on the stream
     pdl_launch_dependents();    // let the expert kernel start its routing-free work
-
-    // initialise the layer output (the expert kernel adds into it after this grid completes)
-    {
-        const int nblk = gridDim.x;
-        float4* o4 = reinterpret_cast<float4*>(p.out);
-        const float4* r4 = reinterpret_cast<const float4*>(p.resid);
-        const int n4 = p.T * H / 4;
-        for (int i = blockIdx.x * RT_THREADS + tid; i < n4; i += nblk * RT_THREADS)
-            o4[i] = r4 ? r4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
 
     for (int i = tid; i < TB * KCOLS; i += RT_THREADS) {
         const int t = i / KCOLS, c = i % KCOLS;
@@ -161,10 +208,15 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
     }
     __syncthreads();
 
-    // thread -> (expert e, quarter of the CTA's columns); products are exact in fp64
-    double acc[TB];
+    // thread -> (expert e, quarter of the CTA's columns); products are exact in fp64.  With
+    // few tokens each token's sum is split over NA interleaved chains (fixed order) so that
+    // the fp64 FMAs overlap.
+    constexpr int NA = TB >= 4 ? 1 : 4 / TB;
+    double accp[TB][NA];
 #pragma unroll
-    for (int t = 0; t < TB; ++t) acc[t] = 0.0;
+    for (int t = 0; t < TB; ++t)
+#pragma unroll
+        for (int k = 0; k < NA; ++k) accp[t][k] = 0.0;
 #pragma unroll
     for (int v = 0; v < NVEC; ++v) {
         float w[8];
@@ -176,23 +228,53 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
         for (int j = 0; j < 8; ++j) {
             const double wd = (double)w[j];
 #pragma unroll
-            for (int t = 0; t < TB; ++t) acc[t] = fma(xs[t][part * PART_COLS + 8 * v + j], wd, acc[t]);
+            for (int t = 0; t < TB; ++t)
+                accp[t][j % NA] = fma(xs[t][part * PART_COLS + 8 * v + j], wd, accp[t][j % NA]);
         }
+    }
+    double acc[TB];
+#pragma unroll
+    for (int t = 0; t < TB; ++t) {
+        acc[t] = accp[t][0];
+#pragma unroll
+        for (int k = 1; k < NA; ++k) acc[t] += accp[t][k];
     }
 #pragma unroll
     for (int t = 0; t < TB; ++t) {
         acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 1);
         acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 2);
     }
+    // partials into CTA 0: local stores there, asynchronous remote stores (completing on CTA
+    // 0's barrier) from the other seven
     if (part == 0) {
-        double* dst = cluster.map_shared_rank(&part_s[r][0][0], 0);
+        if (r == 0) {
 #pragma unroll
-        for (int t = 0; t < TB; ++t) dst[t * E + e] = acc[t];
+            for (int t = 0; t < TB; ++t) part_s[0][t][e] = acc[t];
+        } else {
+            const uint32_t rbar = mapa_shared(&pbar, 0);
+#pragma unroll
+            for (int t = 0; t < TB; ++t) st_async_f64(mapa_shared(&part_s[r][t][e], 0), acc[t], rbar);
+        }
     }
-    cluster.sync();            // partials of all eight CTAs are in CTA 0
-    if (r != 0) return;
+    if (r != 0) {
+        // CTAs 1..7 of every cluster initialise the layer output (the expert kernels add into
+        // it after this grid completes)
+        const int nw = (gridDim.x / RC) * (RC - 1), w = tb * (RC - 1) + (r - 1);
+        float4* o4 = reinterpret_cast<float4*>(p.out);
+        const float4* r4 = reinterpret_cast<const float4*>(p.resid);
+        const int n4 = p.T * H / 4;
+        for (int i = w * RT_THREADS + tid; i < n4; i += nw * RT_THREADS)
+            o4[i] = r4 ? r4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        return;
+    }
 
-    // ---- CTA 0: logits (fixed summation order), softmax, top-6
+    // ---- CTA 0: wait for the remote partials (bounded), then logits (fixed summation
+    // order), softmax, top-6
+    __syncthreads();   // CTA 0's own partials are in place
+    if (!mbar_wait_bounded(&pbar, 0, WAIT_LIMIT_NS)) {
+        if (tid == 0) atomicExch(&p.R.ctrl[CTRL_ERROR], DEVERR_FULL_WAIT);
+        (void)mbar_wait_bounded(&pbar, 0, WAIT_LIMIT_NS);   // never exit with remote stores in flight
+    }
     for (int i = tid; i < TB * E; i += RT_THREADS) {
         const int t = i / E, ee = i % E;
         if (t < nt) {
@@ -207,36 +289,63 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
     __syncthreads();
 
     const int warp = tid >> 5, lane = tid & 31;
-    if (warp < nt) {
-        const int t = warp;
-        const float v0 = lg[t][lane], v1 = lg[t][lane + 32];
-        float m = fmaxf(v0, v1);
+    // softmax statistics: one warp per token (the highest warps), two logits per lane
+    {
+        const int t = RT_THREADS / 32 - 1 - warp;
+        if (t < nt) {
+            const float v0 = lg[t][lane], v1 = lg[t][lane + 32];
+            float m = fmaxf(v0, v1);
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float den = expf(v0 - m) + expf(v1 - m);
+            for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            float den = expf(v0 - m) + expf(v1 - m);
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-        bool taken0 = false, taken1 = false;
-        for (int j = 0; j < K; ++j) {
-            // best remaining candidate of this lane (lower index first on ties)
-            float cv = -INFINITY;
-            int ci = 0x7fffffff;
-            if (!taken0) { cv = v0; ci = lane; }
-            if (!taken1 && (v1 > cv || (v1 == cv && lane + 32 < ci))) { cv = v1; ci = lane + 32; }
-            warp_argmax(cv, ci);
-            if (ci == lane) taken0 = true;
-            if (ci == lane + 32) taken1 = true;
+            for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
             if (lane == 0) {
-                sidx[t * K + j] = ci;
-                p.R.topk_idx[(size_t)(t0 + t) * K + j] = ci;
-                p.R.topk_w[(size_t)(t0 + t) * K + j] = expf(cv - m) / den;
+                smax[t] = m;
+                sden[t] = den;
             }
+        }
+    }
+    // greedy top-6 by rank: candidate c of token t is ahead of `rank` experts, counted in
+    // (logit descending, index ascending) order over the token's 64 logits (branch-free, the
+    // logits read as broadcast 16-byte vectors); the six of rank < 6 are the top-6
+    constexpr int RPT = (TB * E + RT_THREADS - 1) / RT_THREADS;   // candidates per thread
+    int rank[RPT];
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+        const int i = tid + k * RT_THREADS, t = i / E, c = i % E;
+        int rk = E;
+        if (t < nt) {
+            const float vc = lg[t][c];
+            const float4* row = reinterpret_cast<const float4*>(&lg[t][0]);
+            rk = 0;
+#pragma unroll
+            for (int q = 0; q < E / 4; ++q) {
+                const float4 f = row[q];
+                const float u[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int j = 4 * q + h;
+                    rk += (int)(u[h] > vc) | ((int)(u[h] == vc) & (int)(j < c));
+                }
+            }
+        }
+        rank[k] = rk;
+    }
+    __syncthreads();   // softmax statistics in place
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+        if (rank[k] < K) {
+            const int i = tid + k * RT_THREADS, t = i / E, c = i % E;
+            sidx[t * K + rank[k]] = c;
+            p.R.topk_idx[(size_t)(t0 + t) * K + rank[k]] = c;
+            p.R.topk_w[(size_t)(t0 + t) * K + rank[k]] = expf(lg[t][c] - smax[t]) / sden[t];
         }
     }
     __syncthreads();
 
-    if (gridDim.x == RC) {     // one token block: dispatch from shared memory
-        dispatch<true>(p, sidx, cnt, cursor, wc);
+    if (gridDim.x == RC) {     // one token block (T <= 8): one warp dispatches from shared memory
+        if (warp == 0) dispatch_small(p, sidx, cnt);
         return;
     }
     // ---- several token blocks: the last one to finish dispatches
@@ -266,6 +375,16 @@ cudaError_t launch_router(const float* x, int T, int /*T_ws*/, const LayerView& 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    static bool configured = false;   // same shared-memory carveout as the expert kernels
+    if (!configured) {
+        for (const void* f : {(const void*)router_kernel<1>, (const void*)router_kernel<2>, (const void*)router_kernel<4>,
+                              (const void*)router_kernel<8>}) {
+            const cudaError_t e =
+                cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+            if (e != cudaSuccess) return e;
+        }
+        configured = true;
+    }
     switch (TB) {
         case 1: return cudaLaunchKernelEx(&cfg, router_kernel<1>, p);
         case 2: return cudaLaunchKernelEx(&cfg, router_kernel<2>, p);
