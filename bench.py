@@ -173,6 +173,19 @@ def run_reference(args, rank, world):
         return
     from weight_quantized_expert_b200 import synth
     import oracle
+    if args.workload in synth.STEP_WORKLOADS:
+        w = synth.STEP_WORKLOADS[args.workload]
+        cpu = step_oracle_rate(w, budget_s=20.0)
+        v = cpu["value"]
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": w["T"] / v * 1e3,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic", "config": {"workload": args.workload, "tokens_per_step": w["T"],
+                                                          "kind": w["kind"]},
+                          "cpu_baseline": cpu,
+                          "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
+        return
     w = synth.WORKLOADS[args.workload]
     _, layer = synth.workload(args.workload)
     om = oracle.OracleMoE(layer)
@@ -209,6 +222,209 @@ def run_reference(args, rank, world):
                                           f"; steps capped from {args.steps} to bound the CPU run")},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ decode-step companions
+
+def step_bytes_companion(w: dict, moe_hits=None) -> int:
+    """Algorithmic bytes of one step of a companion / stack workload."""
+    from weight_quantized_expert_b200 import roofline
+    T = w["T"]
+    lm = roofline.VOCAB * roofline.H * 1 + roofline.VOCAB * 4 + T * roofline.H * 4 + T * 4
+    dense = roofline.swiglu_bytes(roofline.DENSE_I, roofline.W_INT8, 128) + T * roofline.H * 4 * 2
+    if w["kind"] == "lm_head":
+        return lm
+    if w["kind"] == "dense":
+        return dense
+    moe = sum(roofline.moe_layer_bytes(T, roofline.W_INT4, roofline.W_BF16, 64, h) for h in moe_hits)
+    norms = (1 + len(moe_hits)) * T * roofline.H * 4 * 2
+    return dense + moe + norms + lm
+
+
+def run_step_workload(args, rank, world, local_rank):
+    """lm_head GEMV + argmax, the dense layer 0, or a whole decode step (dense layer 0, 11 MoE layers with
+    residual adds, RMSNorm, lm_head + argmax) through the C ABI; same JSON contract as the layer bench."""
+    import torch
+    from weight_quantized_expert_b200 import api, synth
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.STEP_WORKLOADS[args.workload]
+    T, kind = w["T"], w["kind"]
+    head = mlp = None
+    layers = []
+    if kind in ("lm_head", "stack"):
+        head = api.focr_lm_head_pack(synth.lm_head(w["seed"]))
+    if kind in ("dense", "stack"):
+        d = synth.dense_mlp(w["seed"])
+        mlp = api.focr_dense_mlp_pack(d.gate, d.up, d.down, synth.W_INT8, 128)
+        del d
+    if kind == "stack":
+        base = api.focr_moe_pack_weights(synth.moe_layer(w["seed"], synth.W_INT4, synth.W_BF16, 64))
+        layers = [base] + [api.focr_moe_layer_clone(base) for _ in range(w["moe_layers"] - 1)]
+    pool_n = 16
+    xs = torch.from_numpy(synth.hidden(w["seed"] + 3000 + rank, pool_n * T).reshape(pool_n, T, 1280)).to(dev)
+    ws = api.new_workspace(T, dev)
+    lm_ws = torch.zeros(api.focr_lm_head_workspace_bytes(T), dtype=torch.uint8, device=dev)
+    hb = [torch.empty(T, 1280, device=dev) for _ in range(2)]
+    am = torch.empty(T, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    launches = {"lm_head": 1, "dense": 2}.get(kind, 0)
+    if kind == "stack":
+        launches = (2 + 1 + 4 * len(layers) + 1) if T <= 8 else (1 + 1 + 3 * len(layers) + 1)
+
+    def step(x, st, debug_counts=None):
+        if kind == "lm_head":
+            api.focr_lm_head_gemv(head, x, argmax=am, workspace=lm_ws, stream=st)
+            return
+        if kind == "dense":
+            api.focr_dense_mlp_forward(mlp, x, out=hb[0], workspace=ws, stream=st)
+            return
+        # h <- RMSNorm(h + FFN(h)) for the dense layer and every MoE layer; the last norm feeds lm_head
+        api.focr_dense_mlp_forward(mlp, x, out=hb[0], workspace=ws, flags=api.FWD_RESIDUAL, stream=st)
+        api.focr_rmsnorm(hb[0], eps=1e-6, out=hb[1], stream=st)
+        for li, L in enumerate(layers):
+            dbg = {"counts": debug_counts[li]} if debug_counts is not None else None
+            api.focr_moe_layer_forward(L, hb[1], out=hb[0], workspace=ws, debug=dbg, stream=st,
+                                       flags=api.FWD_RESIDUAL)
+            api.focr_rmsnorm(hb[0], eps=1e-6, out=hb[1], stream=st)
+        api.focr_lm_head_gemv(head, hb[1], argmax=am, workspace=lm_ws, stream=st)
+
+    hits = None
+    if kind == "stack":   # experts hit per layer, for the algorithmic bytes
+        counts = [torch.empty(64, dtype=torch.int32, device=dev) for _ in layers]
+        per = []
+        with torch.cuda.stream(stream):
+            for j in range(pool_n):
+                step(xs[j], stream, counts)
+                per.append([int((c > 0).sum().item()) for c in counts])
+        stream.synchronize()
+        hits = [sum(p[li] for p in per) / pool_n for li in range(len(layers))]
+    bytes_step = step_bytes_companion(w, hits)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(xs[i % pool_n], stream)
+    stream.synchronize()
+    G = 20 if kind == "stack" else 160
+    K = args.steps
+    g_main = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_main, stream=stream):
+        for i in range(G):
+            step(xs[i % pool_n], torch.cuda.current_stream())
+    n_rep = max(1, K // G)
+    K = n_rep * G
+    with torch.cuda.stream(stream):
+        g_main.replay()
+    stream.synchronize()
+    clocks = Clocks(local_rank)
+    clocks.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(n_rep):
+            g_main.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / K
+    value = T * K * world / (ms / 1e3)
+    peak, peak_kind = peaks()
+    achieved = bytes_step / (ms_step / 1e3) / 1e9
+    # end to end: pinned host x in, the step, the step's result (argmax, or the dense output) out
+    out_t = hb[0] if kind == "dense" else am
+    hx = torch.from_numpy(synth.hidden(w["seed"] + 4000, T)).pin_memory()
+    hy = torch.empty(out_t.shape, dtype=out_t.dtype).pin_memory()
+    dx = torch.empty(T, 1280, device=dev)
+    K_e2e = min(K, 200)
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            dx.copy_(hx, non_blocking=True)
+            step(dx, stream)
+            hy.copy_(out_t, non_blocking=True)
+        stream.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(K_e2e):
+            dx.copy_(hx, non_blocking=True)
+            step(dx, stream)
+            hy.copy_(out_t, non_blocking=True)
+        f1.record(stream)
+        stream.synchronize()
+    e2e = T * K_e2e * world / (f0.elapsed_time(f1) / 1e3)
+    api.focr_moe_check(ws, stream)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = step_oracle_rate(w)
+    if rank == 0:
+        desc = {"workload": args.workload, "tokens_per_step": T, "kind": kind, "seed": w["seed"],
+                "parallelism": f"replicas x{world}", "graph": f"CUDA graph replay ({G} steps per graph)"}
+        if kind == "stack":
+            desc.update(wiring="h <- RMSNorm(h + FFN(h)) per layer (eps 1e-6, gamma 1); lm_head on the last norm",
+                        moe_layers=len(layers), moe="int4 g64, bf16 router and shared expert "
+                        "(11 device copies of one packed layer)", dense="int8 g128", lm_head="int8 per-row",
+                        l2="one step streams every layer once (> 1.5 GB)")
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+                "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32", "data": "synthetic", "config": desc,
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                             "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                             "kernel": "one step of the workload (all its launches, timed together)",
+                             "algorithmic_bytes_per_step": bytes_step},
+                "cpu_baseline": cpu,
+                "e2e": {"value": e2e, "unit": UNIT, "h2d_bytes_per_step": T * 1280 * 4,
+                        "d2h_bytes_per_step": int(out_t.numel() * out_t.element_size()), "steps": K_e2e},
+                "gpu_launches": launches * K, "clocks": clk}
+        print(json.dumps(line), flush=True)
+
+
+def step_oracle_rate(w: dict, budget_s: float = 10.0):
+    """tokens/s of the CPU oracle on a bounded sample of a companion / stack workload."""
+    import oracle
+    from weight_quantized_expert_b200 import synth
+    threads = oracle.max_threads()
+    kind = w["kind"]
+    lm = oracle.OracleLMHead(synth.lm_head(w["seed"])) if kind in ("lm_head", "stack") else None
+    dn = None
+    if kind in ("dense", "stack"):
+        d = synth.dense_mlp(w["seed"])
+        dn = oracle.OracleDense(d.gate, d.up, d.down, oracle.W_INT8, 128)
+        del d
+    om = oracle.OracleMoE(synth.moe_layer(w["seed"], synth.W_INT4, synth.W_BF16, 64)) if kind == "stack" else None
+
+    def run(x):
+        if kind == "lm_head":
+            lm.forward(x, nthreads=threads)
+        elif kind == "dense":
+            dn.forward(x, nthreads=threads)
+        else:
+            h = oracle.rmsnorm(x + dn.forward(x, nthreads=threads), eps=1e-6)
+            for _ in range(w["moe_layers"]):
+                h = oracle.rmsnorm(h + om.forward(h, nthreads=threads)["out"], eps=1e-6)
+            lm.forward(h, nthreads=threads)
+
+    n = max(1, min(threads, 8)) if kind == "stack" else threads
+    pool = synth.hidden(w["seed"] + 5000, 512)
+    t0 = time.perf_counter()
+    run(pool[:n])
+    dt = time.perf_counter() - t0
+    done, total = n, dt
+    while total < budget_s and done + n <= pool.shape[0]:
+        t0 = time.perf_counter()
+        run(pool[done:done + n])
+        total += time.perf_counter() - t0
+        done += n
+    return {"value": done / total, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{done} tokens through the CPU oracle's {kind} ({'dense layer 0, 11 MoE layers, RMSNorm, lm_head' if kind == 'stack' else kind}), "
+                      f"{total:.1f} s, batches of {n} tokens (plain C, fp64, OpenMP)"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -391,7 +607,11 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_ours(args, rank, world, local_rank)
+        from weight_quantized_expert_b200 import synth
+        if args.workload in synth.STEP_WORKLOADS:
+            run_step_workload(args, rank, world, local_rank)
+        else:
+            run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch

@@ -156,7 +156,7 @@ def test_residual_moe_forward_adds_the_input():
 
 @pytest.mark.parametrize("T", [1, 4])
 def test_short_decode_stack(T):
-    """h <- h + dense(h); h <- h + MoE_a(h); h <- h + MoE_b(h); argmax(lm_head(RMSNorm(h)))."""
+    """h <- RMSNorm(h + FFN(h)) for the dense layer and two MoE layers, then argmax(lm_head(h))."""
     torch = _torch()
     dref, mlp = dense_case()
     om_a, la = moe_case(1, synth.W_INT4, synth.W_BF16, 64)
@@ -164,20 +164,41 @@ def test_short_decode_stack(T):
     href, head = lm_case()
     x = synth.hidden(95, T)
     # oracle composition (fp32 residual adds, like the device path)
-    h = x + dref.forward(x)
-    h = h + om_a.forward(h)["out"]
-    h = h + om_b.forward(h)["out"]
-    rn = oracle.rmsnorm(h, eps=1e-6)
+    h = oracle.rmsnorm(x + dref.forward(x), eps=1e-6)
+    h = oracle.rmsnorm(h + om_a.forward(h)["out"], eps=1e-6)
+    rn = oracle.rmsnorm(h + om_b.forward(h)["out"], eps=1e-6)
     r_idx, r_logits = href.forward(rn, want_logits=True, nthreads=NTHREADS)
     # device path
     ws = api.new_workspace(T)
     h0 = torch.from_numpy(x).cuda()
-    h1 = api.focr_dense_mlp_forward(mlp, h0, workspace=ws, flags=api.FWD_RESIDUAL)
-    h2 = api.focr_moe_layer_forward(la, h1, workspace=ws, flags=api.FWD_RESIDUAL)
-    h3 = api.focr_moe_layer_forward(lb, h2, workspace=ws, flags=api.FWD_RESIDUAL)
-    rg = api.focr_rmsnorm(h3, eps=1e-6)
+    g = api.focr_rmsnorm(api.focr_dense_mlp_forward(mlp, h0, workspace=ws, flags=api.FWD_RESIDUAL), eps=1e-6)
+    g = api.focr_rmsnorm(api.focr_moe_layer_forward(la, g, workspace=ws, flags=api.FWD_RESIDUAL), eps=1e-6)
+    rg = api.focr_rmsnorm(api.focr_moe_layer_forward(lb, g, workspace=ws, flags=api.FWD_RESIDUAL), eps=1e-6)
     am = api.focr_lm_head_gemv(head, rg)
     torch.cuda.synchronize()
     assert per_token_rel_err(rg.cpu().numpy(), rn).max() <= 5e-3
     scale = np.abs(r_logits).max()
     _check_argmax(am.cpu().numpy(), r_logits, 2e-2 * scale)
+
+
+def test_router_survives_non_finite_tokens():
+    """A token with NaN entries still routes to six distinct in-range experts (its outputs are NaN); the
+    finite tokens of the batch are unaffected."""
+    torch = _torch()
+    om, packed = moe_case(1, synth.W_INT4, synth.W_BF16, 64)
+    x = synth.hidden(96, 3)
+    x[1, 5] = np.nan
+    xd = torch.from_numpy(x).cuda()
+    idx = torch.empty(3, 6, dtype=torch.int32, device="cuda")
+    ws = api.new_workspace(3)
+    out = api.focr_moe_layer_forward(packed, xd, workspace=ws, debug={"topk_idx": idx})
+    torch.cuda.synchronize()
+    api.focr_moe_check(ws)
+    assert int(ws[:api.focr_moe_workspace_zero_bytes()].count_nonzero()) == 0
+    got = idx.cpu().numpy()
+    for t in range(3):
+        assert len(set(got[t].tolist())) == 6 and got[t].min() >= 0 and got[t].max() < 64
+    ref = om.forward(x[[0, 2]])
+    g = out.cpu().numpy()[[0, 2]]
+    assert np.array_equal(got[[0, 2]], ref["idx"])
+    assert per_token_rel_err(g, ref["out"]).max() <= 2e-3

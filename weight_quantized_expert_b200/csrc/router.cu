@@ -163,7 +163,10 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
     cg::cluster_group cluster = cg::this_cluster();
     __shared__ double part_s[RC][TB][E];     // filled in CTA 0 by all CTAs of the cluster
     __shared__ __align__(8) uint64_t pbar;   // CTA 0: completes when the seven remote partials landed
-    __shared__ double xs[TB][KCOLS];
+    __shared__ __align__(16) double xs[TB][KCOLS];
+    // ranking keys of the logits (CTA 0, after the GEMV): they reuse the x tile's space
+    unsigned long long (*lk)[E] = reinterpret_cast<unsigned long long (*)[E]>(&xs[0][0]);
+    static_assert(sizeof(double) * KCOLS >= sizeof(unsigned long long) * E, "key rows fit the x tile");
     __shared__ __align__(16) float lg[TB][E];
     __shared__ float smax[TB], sden[TB];
     __shared__ int sidx[TB * K];
@@ -284,6 +287,12 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
             const float l = (float)s;
             lg[t][ee] = l;
             p.R.logits[(size_t)(t0 + t) * E + ee] = l;
+            // strict total order for the top-6: order-preserving bits of the logit (-0 folded into
+            // +0, so equal logits tie), then the lower index; any logit vector, NaN included,
+            // yields six distinct in-range experts
+            uint32_t b = __float_as_uint(l + 0.0f);
+            b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+            lk[t][ee] = ((unsigned long long)b << 32) | (unsigned long long)(E - 1 - ee);
         }
     }
     __syncthreads();
@@ -307,8 +316,8 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
         }
     }
     // greedy top-6 by rank: candidate c of token t is ahead of `rank` experts, counted in
-    // (logit descending, index ascending) order over the token's 64 logits (branch-free, the
-    // logits read as broadcast 16-byte vectors); the six of rank < 6 are the top-6
+    // (logit descending, index ascending) order over the token's 64 keys (branch-free, the keys
+    // read as broadcast 16-byte vectors); the six of rank < 6 are the top-6
     constexpr int RPT = (TB * E + RT_THREADS - 1) / RT_THREADS;   // candidates per thread
     int rank[RPT];
 #pragma unroll
@@ -316,18 +325,13 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
         const int i = tid + k * RT_THREADS, t = i / E, c = i % E;
         int rk = E;
         if (t < nt) {
-            const float vc = lg[t][c];
-            const float4* row = reinterpret_cast<const float4*>(&lg[t][0]);
+            const unsigned long long kc = lk[t][c];
+            const ulonglong2* row = reinterpret_cast<const ulonglong2*>(&lk[t][0]);
             rk = 0;
 #pragma unroll
-            for (int q = 0; q < E / 4; ++q) {
-                const float4 f = row[q];
-                const float u[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int j = 4 * q + h;
-                    rk += (int)(u[h] > vc) | ((int)(u[h] == vc) & (int)(j < c));
-                }
+            for (int q = 0; q < E / 2; ++q) {
+                const ulonglong2 f = row[q];
+                rk += (int)(f.x > kc) + (int)(f.y > kc);
             }
         }
         rank[k] = rk;

@@ -7,6 +7,7 @@ once per group.  Flops count 2 per multiply-add of the dense contractions.
 from __future__ import annotations
 
 H, E, TOPK, I, IS = 1280, 64, 6, 896, 1792
+VOCAB, DENSE_I = 129280, 6848
 W_BF16, W_INT8, W_INT4 = 0, 1, 2
 
 

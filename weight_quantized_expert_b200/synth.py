@@ -187,6 +187,16 @@ WORKLOADS = {
 }
 
 
+# The decode-step companions and the stack of one decode step: dense SwiGLU layer 0 (int8 g128),
+# 11 MoE layers (int4 g64, bf16 router and shared expert), final RMSNorm, int8 lm_head + argmax.
+STEP_WORKLOADS = {
+    "lm_head_t1": dict(kind="lm_head", seed=4, T=1),
+    "dense_t1": dict(kind="dense", seed=4, T=1),
+    "stack_t1": dict(kind="stack", seed=4, T=1, moe_layers=11),
+    "stack_t32": dict(kind="stack", seed=4, T=32, moe_layers=11),
+}
+
+
 def workload(name: str):
     """Return (x [T,H] f32, MoELayerInputs) for a named workload."""
     w = WORKLOADS[name]
