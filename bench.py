@@ -74,9 +74,16 @@ def peaks():
 
 
 def sources_hash() -> str:
+    """Identity of the kernel code a profile was taken on: the CUDA/C++ sources with comments and
+    blank space removed (the sources hold no comment markers inside string literals), so a comment
+    edit keeps a profile valid and any code change invalidates it."""
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "weight_quantized_expert_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+        src = open(f, encoding="utf-8").read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(os.path.basename(f).encode())
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -149,8 +149,9 @@ size_t focr_moe_workspace_zero_bytes(void);
  * Steps, all on `stream`: router GEMV (fp64 accumulation of exact products,
  * rounded to fp32) + softmax + greedy top-6 (rank by fp32 logit, ties to the
  * lower index) + dispatch (counting sort of t*6+j by expert, stable), then the
- * grouped expert kernel (shared expert and the selected experts, dequantised in
- * registers, fp32 accumulation) which adds w * expert(x) into out.
+ * shared expert and the selected experts (codes dequantised in registers, fp32
+ * accumulation), which add w * expert(x) into out: for T <= 8 a gate/up kernel
+ * and a down kernel, for larger T one grouped expert kernel.
  */
 focr_status focr_moe_layer_forward(const focr_moe_layer* layer, const float* hidden, int32_t T, float* out,
                                    void* workspace, size_t ws_bytes, const focr_moe_route_debug* dbg,

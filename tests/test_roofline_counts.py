@@ -23,3 +23,35 @@ def test_int4_single_token_group_sweep():
 def test_prefill_all_experts():
     assert rf.moe_layer_bytes(289, rf.W_INT4, rf.W_BF16, 64, 64) == 140_748_800
     assert abs(rf.moe_layer_flops(289) - 15.96e9) / 15.96e9 < 0.01
+
+
+def test_decode_step_companions():
+    # dense layer 0, int8 g128: gate/up 6848 x 1280 codes + 6848 x 10 scales; down 1280 x 6848 codes
+    # + 1280 x 54 scales (the 54th group of each down row is the short 64-wide tail)
+    assert rf.swiglu_bytes(6848, rf.W_INT8, 128) == 2 * (8_765_440 + 273_920) + (8_765_440 + 276_480)
+    assert rf.swiglu_bytes(6848, rf.W_INT8, 128) == 27_120_640
+
+
+def test_decode_step_bench_bytes():
+    import bench
+    from weight_quantized_expert_b200 import synth
+    lm = 129_280 * 1_280 + 129_280 * 4          # int8 codes + one f32 scale per row
+    assert bench.step_bytes_companion(synth.STEP_WORKLOADS["lm_head_t1"]) == lm + 1_280 * 4 + 4
+    assert bench.step_bytes_companion(synth.STEP_WORKLOADS["dense_t1"]) == 27_120_640 + 2 * 1_280 * 4
+    # T = 1 stack: dense + 11 MoE layers of 25,548,800 B + 12 RMSNorms (in + out) + lm_head
+    got = bench.step_bytes_companion(synth.STEP_WORKLOADS["stack_t1"], [6] * 11)
+    assert got == (27_120_640 + 2 * 5_120) + 11 * 25_548_800 + 12 * 2 * 5_120 + (lm + 5_120 + 4)
+
+
+def test_profile_identity_ignores_comments_only(tmp_path, monkeypatch):
+    import shutil
+    import bench
+    src = tmp_path / "weight_quantized_expert_b200" / "csrc"
+    shutil.copytree(bench.os.path.join(bench.ROOT, "weight_quantized_expert_b200", "csrc"), src)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.sources_hash()
+    f = src / "rmsnorm.cu"
+    f.write_text("// an extra comment line\n" + f.read_text().replace("{", "{ /* inline */", 1))
+    assert bench.sources_hash() == h0
+    f.write_text(f.read_text().replace("1e-6", "2e-6") + "\nstatic int focr_extra_symbol = 1;\n")
+    assert bench.sources_hash() != h0

@@ -1,4 +1,5 @@
-// Decode path for T <= 8 tokens: two streaming kernels with no CTA-wide synchronisation.
+// Decode path for T <= 8 tokens: a gate/up kernel and a down kernel, chained behind the
+// router by programmatic dependent launch.
 //
 // Sources: frankenocr.pages.dev, "One forward pass", step 6 (64 routed experts + 2 fused
 // shared experts, top-6 without renormalisation); franken_ocr README, "Architecture"
@@ -7,27 +8,29 @@
 //
 // The batch's tokens are the 8 columns of m16n8 tensor-core fragments (tokens that did not
 // pick an expert get routing weight 0).  Both kernels read the packed item layout of
-// common.cuh straight from global memory with 16-byte loads; every warp works alone on
-// ~10 KB units.
+// common.cuh.
 //
-// decode_gu (router -> gu, programmatic dependent launch): a unit is one tile of 8
-//   intermediates (8 gate rows over 8 up rows) of the shared set or of a selected expert
-//   over a range of input columns (all 1280 for int4, halves for int8, quarters for bf16).
-//   int4/int8 codes become exact f16 A fragments, each scale group's fp32 accumulator is
-//   scaled, bf16 weights enter bf16 MMAs with x split into hi + lo.  A unit that covers the
-//   whole row applies a = silu(g) * u * w_route itself; k-split tiles add their partial
-//   sums into the workspace with vector atomics, and the warp that completes a tile
-//   (arrival counter) applies it and clears the sums and the counter.  a goes to the
-//   workspace as the B fragments of the down projection.  Shared-set units run while the
-//   router is still working; routed units start after griddepcontrol.wait.  Warps of
-//   routed units also prefetch their expert's down-projection bytes into L2.
-// decode_down (gu -> down): a unit is one output tile of 16 rows of one selected expert
-//   (all 896 intermediates) or of a quarter of the shared set; y = D a is scaled per row
-//   and group and added into the output with atomics (the router initialised it).
+// decode_gu: a unit is one tile of 8 intermediates (8 gate rows over 8 up rows) of the
+//   shared set or of a selected expert over a range of input columns (all 1280 for int4,
+//   halves for int8, quarters for bf16) -- about 10 KB of codes.  Each warp works alone: it
+//   bulk-copies a unit into its own shared-memory buffer (cp.async.bulk, own mbarrier,
+//   bounded wait), turns int4/int8 codes into exact f16 A fragments (bf16 weights enter
+//   bf16 MMAs with x split into hi + lo), scales each group's fp32 sum, and applies
+//   a = silu(g) * u * w_route to whole rows; tiles split along K add their partial sums into
+//   the workspace with vector atomics and the warp that completes a tile (arrival counter)
+//   applies it and clears the sums.  a goes to the workspace as the down projection's B
+//   fragments.  Shared-set units run while the router is still working, routed units after
+//   griddepcontrol.wait; the first unit of every slice prefetches the slice's
+//   down-projection bytes into L2.
+// decode_down: a unit is one 16-row output tile of one set (shared, or a selected expert)
+//   over a chunk of 8-16 slices.  The 8 warps of a CTA take 8 tiles of one chunk; each
+//   loads its codes and scales (the first step before waiting on decode_gu), one bulk copy
+//   stages the chunk's B fragments of a in shared memory for all of them, and y = D a is
+//   scaled per row and group and added into the output with atomics (the router initialised
+//   it).
 //
-// Precision: as the grouped expert kernel -- int4/int8 codes exact in f16 with fp32 group
-// scales and f16 activations; bf16 weights exact with bf16 hi + lo activations; fp32
-// accumulation throughout.
+// Precision: int4/int8 codes exact in f16 with fp32 group scales and f16 activations; bf16
+// weights exact with bf16 hi + lo activations; fp32 accumulation throughout.
 #include "common.cuh"
 #include "fragments.cuh"
 

@@ -10,12 +10,15 @@
 // (fp32 logit descending, index ascending).  Softmax is evaluated in fp32.
 //
 // Grid: one thread-block cluster of 8 CTAs per block of TB <= 8 tokens.  CTA r of a
-// cluster computes fp64 partial logits over input columns [160 r, 160 r + 160) and
-// writes them into CTA 0's shared memory (distributed shared memory); after one
-// cluster barrier CTA 0 sums the eight partials in a fixed order, runs softmax + top-6
-// (one warp per token) and, when the batch has a single token block, the dispatch
-// straight from shared memory.  With several token blocks each cluster publishes its
-// top-6 and the last one to finish (atomic ticket, reset after use) does the dispatch.
+// cluster computes fp64 partial logits over input columns [160 r, 160 r + 160); the seven
+// remote CTAs send theirs into CTA 0's shared memory as asynchronous stores (st.async)
+// that complete on a CTA-0 mbarrier, armed before the one cluster barrier (which precedes
+// the wait on the previous kernel), and then initialise the layer output.  CTA 0 sums the
+// eight partials in a fixed order, ranks each token's 64 experts by a strict total-order
+// key (one thread per candidate) while other warps compute the softmax statistics, and,
+// when the batch has a single token block, one warp does the dispatch from shared memory.
+// With several token blocks each cluster publishes its top-6 and the last one to finish
+// (atomic ticket, reset after use) does the dispatch.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
