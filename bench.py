@@ -146,6 +146,24 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+# ------------------------------------------------------------------ ranks (one replica per GPU)
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank runs an independent replica, the job is done when the
+    last one is.  Collective over the default process group (NCCL on GPUs, gloo in the CPU tests)."""
+    if world == 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(tokens_per_step: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job tokens/s: the tokens all ranks processed over the slowest rank's time."""
+    return tokens_per_step * steps * world / (ms / 1e3)
+
+
 # ------------------------------------------------------------------ CPU oracle timing
 
 def oracle_rate(name: str, budget_s: float, max_tokens: int | None = None):
@@ -337,13 +355,9 @@ def run_step_workload(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     ms_step = ms / K
-    value = T * K * world / (ms / 1e3)
+    value = job_rate(T, K, world, ms)
     peak, peak_kind = peaks()
     achieved = bytes_step / (ms_step / 1e3) / 1e9
     # end to end: pinned host x in, the step, the step's result (argmax, or the dense output) out
@@ -366,7 +380,7 @@ def run_step_workload(args, rank, world, local_rank):
             hy.copy_(out_t, non_blocking=True)
         f1.record(stream)
         stream.synchronize()
-    e2e = T * K_e2e * world / (f0.elapsed_time(f1) / 1e3)
+    e2e = job_rate(T, K_e2e, world, max_over_ranks(f0.elapsed_time(f1), world, dev))
     api.focr_moe_check(ws, stream)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -522,11 +536,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     # steps in the timed graph replay follow the same i % pool order
     order = [i % G for i in range(G)]
     if use_graph:
@@ -535,8 +545,7 @@ def run_ours(args, rank, world, local_rank):
     else:
         avg_bytes = sum(step_bytes[i % pool_n] for i in range(args.steps)) / args.steps
     ms_per_step = ms / args.steps
-    tokens = T * args.steps * world
-    value = tokens / (ms / 1e3)
+    value = job_rate(T, args.steps, world, ms)
     peak, peak_kind = peaks()
     achieved = avg_bytes / (ms_per_step / 1e3) / 1e9
     traffic = profiled_traffic(args.workload)
@@ -564,12 +573,8 @@ def run_ours(args, rank, world, local_rank):
             hy[i % 8].copy_(dy, non_blocking=True)
         e1.record(stream)
         stream.synchronize()
-    ms_e2e = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e_value = T * K_e2e * world / (ms_e2e / 1e3)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_rate(T, K_e2e, world, ms_e2e)
     api.focr_moe_check(ws, stream)
 
     cpu = None
