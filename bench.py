@@ -108,8 +108,8 @@ class Clocks:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv") if os.path.isdir(
-            os.path.join(ROOT, "gpurun_out")) else f"/tmp/focr_clocks_{os.getpid()}.csv"
+        import tempfile
+        self.path = os.path.join(tempfile.gettempdir(), f"focr_clocks_{os.getpid()}_gpu{index}.csv")
 
     def start(self):
         try:

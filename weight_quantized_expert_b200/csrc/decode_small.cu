@@ -479,7 +479,7 @@ __device__ __forceinline__ bool down_step(const SmallParams& p, const uint8_t* i
         mbar_arrive_expect_tx(bar, bytes);
         bulk_g2s(bsm, bset + (size_t)chunk * D::CH * D::BPS * 32, bytes, bar, policy_evict_first());
     }
-    // the verdict is CTA-uniform, so every warp leaves the step loop together
+    // the wait's outcome is made CTA-uniform, so every warp leaves the step loop together
     const bool ok = __syncthreads_and(mbar_wait_bounded(bar, phase, WAIT_LIMIT_NS)) != 0;
     phase ^= 1u;
     if (!ok) {
