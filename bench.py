@@ -73,12 +73,15 @@ def peaks():
     return PEAK_FALLBACK_GBS, "fallback"
 
 
-def sources_hash() -> str:
-    """Identity of the kernel code a profile was taken on: the CUDA/C++ sources with comments and
-    blank space removed (the sources hold no comment markers inside string literals), so a comment
-    edit keeps a profile valid and any code change invalidates it."""
+def sources_hash(files=None) -> str:
+    """Identity of the kernel code a profile was taken on: the listed CUDA/C++ sources (all of csrc/
+    when none are listed) with comments and blank space removed (the sources hold no comment markers
+    inside string literals), so a comment edit keeps a profile valid and any code change in those
+    files invalidates it."""
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "weight_quantized_expert_b200", "csrc", "*"))):
+    csrc = os.path.join(ROOT, "weight_quantized_expert_b200", "csrc")
+    paths = sorted(glob.glob(os.path.join(csrc, "*"))) if not files else sorted(os.path.join(csrc, f) for f in files)
+    for f in paths:
         src = open(f, encoding="utf-8").read()
         src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
         src = re.sub(r"//[^\n]*", " ", src)
@@ -94,7 +97,9 @@ def profiled_traffic(workload: str):
         m_w = re.search(r"^workload:\s*(\S+)", txt, re.M)
         m_t = re.search(r"^traffic_bytes_per_step:\s*(\d+)", txt, re.M)
         m_h = re.search(r"^sources_sha256:\s*(\S+)", txt, re.M)
-        if m_w and m_t and m_h and m_w.group(1) == workload and m_h.group(1) == sources_hash():
+        m_s = re.search(r"^sources:\s*(.+)$", txt, re.M)
+        files = m_s.group(1).split() if m_s else None
+        if m_w and m_t and m_h and m_w.group(1) == workload and m_h.group(1) == sources_hash(files):
             return int(m_t.group(1))
     return None
 

@@ -1,6 +1,6 @@
-// Grouped expert kernel for decode-sized batches: the shared expert and every
-// selected routed expert, SwiGLU fused, weights dequantised in registers straight
-// into 16x8x16 tensor-core fragments (f16 operands, fp32 accumulation).
+// Grouped expert kernel for batches of more than 8 tokens (batched decode, prefill): the
+// shared expert and every selected routed expert, SwiGLU fused, weights dequantised in
+// registers straight into 16x8x16 tensor-core fragments (fp32 accumulation).
 //
 // Sources: frankenocr.pages.dev, "One forward pass", step 6 (64 routed experts + 2 fused
 // shared experts, top-6 without renormalisation); franken_ocr README, "Architecture"
@@ -12,22 +12,19 @@
 // that received tokens (ascending id); CTA b of a persistent grid (one per SM) takes
 // items b, b+G, ...  A producer warp streams item blocks into a 2- or 3-slot shared-memory
 // ring with bulk async copies (cp.async.bulk + mbarrier) and publishes each item's
-// expert id next to it; 20 consumer warps compute:
+// expert id next to it.  20 consumer warps walk the item's tokens (all tokens for the
+// shared expert, the expert's segment of the dispatch permutation otherwise) in passes of
+// NG x 8 tokens, each group of 8 being the columns of one set of n8 fragments:
 //   phase 1  [g; u] = [G; U]_slice x  -- warp w covers input columns [64w, 64w + 64) of every
-//            tile with mma.sync m16n8k16 (x's fragments stay in its registers); int4/int8
-//            codes become exact f16 values and each scale group's fp32 accumulator is
-//            multiplied by its scale; bf16 weights feed bf16 MMAs as stored; the twenty
-//            column parts are summed in shared memory
-//   swiglu   a = silu(g) * u * w_route  (fp32, then f16 phase-2 B fragments)
+//            tile with mma.sync m16n8k16; each A fragment (int4/int8 codes as exact f16,
+//            bf16 weights as stored) serves every token group of the pass; each scale
+//            group's fp32 sum is scaled; the twenty column parts meet in shared memory
+//   swiglu   a = silu(g) * u * w_route  (fp32, then the phase-2 B fragments)
 //   phase 2  y = D[:, slice] a          -- warp owns 4 of the 80 output tiles
-// Tokens are the 8 columns of the n8 fragments.  With T <= 8 every item uses the same
-// columns (the batch), routed weights of tokens that did not pick the expert are 0, and
-// the layer output stays in registers across all of a CTA's items: one flush of atomics
-// at the end.  With T > 8 items walk their tokens in groups of 8 (gathered) and add every
-// group's result into the output with atomics.
-// The shared-expert slices need no routing, so they run while the router kernel is still
-// working (programmatic dependent launch); routed items start after griddepcontrol.wait,
-// and no output is added before it (the router zeroes `out`).  Every mbarrier wait is
+// and adds every token's result into its output row with atomics.  The shared-expert
+// slices need no routing, so they run while the router kernel is still working
+// (programmatic dependent launch); routed items start after griddepcontrol.wait, and no
+// output is added before it (the router initialises `out`).  Every mbarrier wait is
 // bounded in time; on expiry the kernel records an error word and stops.
 //
 // Precision: int4/int8 codes are exact in f16 and scales are applied in fp32; x and a are
@@ -47,6 +44,8 @@ constexpr int NCW = 20;                      // consumer warps
 constexpr int NCT = NCW * 32;                // consumer threads
 constexpr int NTHREADS = NCT + 32;           // + producer warp
 constexpr int NTOK = 8;                      // tokens per fragment (n8)
+constexpr int NG = 2;                        // token groups per pass
+constexpr int NTP = NG * NTOK;               // tokens per pass
 constexpr uint32_t DSC_BYTES = H * 4;        // one group's down scales
 constexpr int TILES_PER_WARP = OTILES / NCW; // 4
 constexpr int KSW = KSTEPS / NCW;            // 4 k-steps of phase 1 per warp
@@ -58,18 +57,15 @@ struct SmemLayout {
     static constexpr uint32_t item_r = blk_bytes_of(RW, G) + (is_quant(RW) ? DSC_BYTES : 0u);
     static constexpr uint32_t item_s = blk_bytes_of(SW, G) + (is_quant(SW) ? DSC_BYTES : 0u);
     static constexpr uint32_t slot_bytes = ((item_r > item_s ? item_r : item_s) + 127u) & ~127u;
-    static constexpr uint32_t rest = 4 * 4 * 32 * 4 + 2 * 32 * 8 + 32 * 8 + 2 * NTOK * 4 + 2 * NTOK * K * 4 + 16 +
-                                     2 * 3 * 8 + 16;
+    static constexpr uint32_t rest = NG * (4 * 4 * 32 * 4 + 2 * 32 * 8 + 32 * 8) + 2 * NTP * 4 + 16 + 2 * 3 * 8 + 16;
     static constexpr int nslot = 3 * slot_bytes + rest <= 232448 ? 3 : 2;
     static constexpr uint32_t slots = 0;
-    static constexpr uint32_t acc = slots + nslot * slot_bytes;         // [4 tiles][4 comps][32] f32 phase-1 sums
-    static constexpr uint32_t ah = acc + 4 * 4 * 32 * 4;                // [2][32] uint2: f16 a B frags
-    static constexpr uint32_t abf = ah + 2 * 32 * 8;                    // [32] uint2: bf16 a hi, lo frags
-    static constexpr uint32_t wn = abf + 32 * 8;                        // [NTOK] f32 route weights
-    static constexpr uint32_t tok = wn + NTOK * 4;                      // [NTOK] i32 token ids
-    static constexpr uint32_t ridx = tok + NTOK * 4;                    // [NTOK][6] i32 (T <= 8)
-    static constexpr uint32_t rw = ridx + NTOK * K * 4;                 // [NTOK][6] f32 (T <= 8)
-    static constexpr uint32_t rec = rw + NTOK * K * 4;                  // [nslot] i32 expert of the slot's item
+    static constexpr uint32_t acc = slots + nslot * slot_bytes;         // [NG][4 tiles][4 comps][32] f32 sums
+    static constexpr uint32_t ah = acc + NG * 4 * 4 * 32 * 4;           // [NG][2][32] uint2: f16 a B frags
+    static constexpr uint32_t abf = ah + NG * 2 * 32 * 8;               // [NG][32] uint2: bf16 a hi, lo frags
+    static constexpr uint32_t wn = abf + NG * 32 * 8;                   // [NTP] f32 route weights
+    static constexpr uint32_t tok = wn + NTP * 4;                       // [NTP] i32 token ids
+    static constexpr uint32_t rec = tok + NTP * 4;                      // [nslot] i32 expert of the slot's item
     static constexpr uint32_t bars = rec + 16;                          // full[nslot], empty[nslot]
     static constexpr uint32_t misc = bars + 2 * 3 * 8;
     static constexpr uint32_t total = misc + 16;
@@ -86,65 +82,74 @@ struct ExpertParams {
 };
 
 // ------------------------------------------------------------------ x fragments (registers)
-// Warp w owns k-steps 4w .. 4w+3 of phase 1 for every item, so its B fragments of x stay in
-// registers: h[j] = f16 (for int4/int8 experts), b[j] = bf16 hi (b0, b1), lo (b0, b1) (for
-// bf16 experts).  Lane (n = lane / 4, c = lane % 4) holds columns 16q+2c, +1 and 16q+2c+8,
-// +9 of token column n; tok[n] < 0 gives zeros.
-template <bool F16, bool BF16>
+// Warp w owns k-steps 4w .. 4w+3 of phase 1, so its B fragments of the pass's x stay in
+// registers, in the form the item's weights need: v[g][j] = f16 (b0, b1) for int4/int8
+// items, bf16 hi (b0, b1), lo (b0, b1) for bf16 items, for token group g.  Lane
+// (n = lane / 4, c = lane % 4) holds columns 16q+2c, +1 and 16q+2c+8, +9 of token
+// tok[8g + n]; tok < 0 gives zeros.
 struct XFrags {
-    uint32_t h[F16 ? KSW : 1][2];
-    uint32_t b[BF16 ? KSW : 1][4];
+    uint32_t v[NG][KSW][4];
 };
 
 template <bool F16, bool BF16>
-__device__ __forceinline__ void load_x_frags(const float* x, const int* tok, int warp, int lane,
-                                             XFrags<F16, BF16>& xf) {
-    const int tk = tok[lane >> 2];
-    float2 lo[KSW], hi[KSW];
+__device__ __forceinline__ void load_x_frags(const float* x, const int* tok, int warp, int lane, bool as_bf16,
+                                             XFrags& xf) {
+    float2 lo[NG][KSW], hi[NG][KSW];
 #pragma unroll
-    for (int j = 0; j < KSW; ++j) {
-        lo[j] = hi[j] = make_float2(0.f, 0.f);
-        if (tk >= 0) {
-            const float* row = x + (size_t)tk * H + 16 * (KSW * warp + j) + 2 * (lane & 3);
-            lo[j] = __ldg(reinterpret_cast<const float2*>(row));
-            hi[j] = __ldg(reinterpret_cast<const float2*>(row + 8));
+    for (int g = 0; g < NG; ++g) {
+        const int tk = tok[NTOK * g + (lane >> 2)];
+#pragma unroll
+        for (int j = 0; j < KSW; ++j) {
+            lo[g][j] = hi[g][j] = make_float2(0.f, 0.f);
+            if (tk >= 0) {
+                const float* row = x + (size_t)tk * H + 16 * (KSW * warp + j) + 2 * (lane & 3);
+                lo[g][j] = __ldg(reinterpret_cast<const float2*>(row));
+                hi[g][j] = __ldg(reinterpret_cast<const float2*>(row + 8));
+            }
         }
     }
 #pragma unroll
-    for (int j = 0; j < KSW; ++j) {
-        if constexpr (F16) {
-            xf.h[j][0] = f32x2_to_f16x2(lo[j].x, lo[j].y);
-            xf.h[j][1] = f32x2_to_f16x2(hi[j].x, hi[j].y);
+    for (int g = 0; g < NG; ++g)
+#pragma unroll
+        for (int j = 0; j < KSW; ++j) {
+            if (BF16 && (!F16 || as_bf16)) {
+                const uint2 a = split_bf16x2(lo[g][j].x, lo[g][j].y), b = split_bf16x2(hi[g][j].x, hi[g][j].y);
+                xf.v[g][j][0] = a.x;
+                xf.v[g][j][1] = b.x;
+                xf.v[g][j][2] = a.y;
+                xf.v[g][j][3] = b.y;
+            } else {
+                xf.v[g][j][0] = f32x2_to_f16x2(lo[g][j].x, lo[g][j].y);
+                xf.v[g][j][1] = f32x2_to_f16x2(hi[g][j].x, hi[g][j].y);
+                xf.v[g][j][2] = xf.v[g][j][3] = 0u;
+            }
         }
-        if constexpr (BF16) {
-            const uint2 a = split_bf16x2(lo[j].x, lo[j].y), b = split_bf16x2(hi[j].x, hi[j].y);
-            xf.b[j][0] = a.x;
-            xf.b[j][1] = b.x;
-            xf.b[j][2] = a.y;
-            xf.b[j][3] = b.y;
-        }
-    }
 }
 
 // ------------------------------------------------------------------ phase 1: gate/up
-// Every tile of the item over this warp's four k-steps.  int4/int8 codes become exact f16
-// values and the fp32 accumulator of each scale group is multiplied by its group scale
-// (the four k-steps lie in one group for g >= 64, in two for g = 32).
-template <int W, int G, bool F16, bool BF16>
-__device__ __forceinline__ void phase_gate_up(const char* slot, const XFrags<F16, BF16>& xf, float* acc_s, int warp,
-                                              int lane) {
+// Every tile of the item over this warp's four k-steps, for the pass's ng token groups.
+// int4/int8 codes become exact f16 values and the fp32 sum of each scale group is multiplied
+// by its scale (the four k-steps lie in one group for g >= 64, in two for g = 32).
+template <int W, int G>
+__device__ __forceinline__ void phase_gate_up(const char* slot, const XFrags& xf, float* acc_s, int warp, int lane,
+                                              int ng) {
     constexpr int NT = slice_rows(W) / 8;
     const int gr = lane >> 2;
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
-        float tot[4] = {0.f, 0.f, 0.f, 0.f};
+        float tot[NG][4] = {};
         if constexpr (!is_quant(W)) {
             const uint4* gw = reinterpret_cast<const uint4*>(slot) + (t * KSTEPS + KSW * warp) * 32 + lane;
 #pragma unroll
             for (int j = 0; j < KSW; ++j) {
                 const uint4 a = gw[j * 32];
-                mma16816_bf16(tot, a, xf.b[j][0], xf.b[j][1]);   // x hi
-                mma16816_bf16(tot, a, xf.b[j][2], xf.b[j][3]);   // x lo
+#pragma unroll
+                for (int g = 0; g < NG; ++g) {
+                    if (g < ng) {
+                        mma16816_bf16(tot[g], a, xf.v[g][j][0], xf.v[g][j][1]);   // x hi
+                        mma16816_bf16(tot[g], a, xf.v[g][j][2], xf.v[g][j][3]);   // x lo
+                    }
+                }
             }
         } else {
             constexpr int NGK = H / G;
@@ -159,105 +164,127 @@ __device__ __forceinline__ void phase_gate_up(const char* slot, const XFrags<F16
                 wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
             }
             const float2* gs = reinterpret_cast<const float2*>(slot + gu_w_bytes_of(W)) + t * NGK * 8 + gr;
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            constexpr int NH = G == 32 ? 2 : 1;   // scale groups among the warp's four k-steps
+            float acc[NG][NH][4] = {};
 #pragma unroll
             for (int j = 0; j < KSW; ++j) {
                 Frag4 a;
                 if constexpr (W == FOCR_W_INT4) a = dq_int4(wv[j]);
                 else a = dq_int8(wv[2 * j], wv[2 * j + 1]);
-                mma16816(acc[G == 32 ? j >> 1 : 0], a, xf.h[j][0], xf.h[j][1]);
-            }
-            constexpr int NG = G == 32 ? 2 : 1;
 #pragma unroll
-            for (int h = 0; h < NG; ++h) {
+                for (int g = 0; g < NG; ++g)
+                    if (g < ng) mma16816(acc[g][G == 32 ? j >> 1 : 0], a, xf.v[g][j][0], xf.v[g][j][1]);
+            }
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
                 const int gi = G == 32 ? 2 * warp + h : (KSW * warp * 16) / G;
                 const float2 sc = gs[gi * 8];
-                tot[0] = fmaf(acc[h][0], sc.x, tot[0]);
-                tot[1] = fmaf(acc[h][1], sc.x, tot[1]);
-                tot[2] = fmaf(acc[h][2], sc.y, tot[2]);
-                tot[3] = fmaf(acc[h][3], sc.y, tot[3]);
+#pragma unroll
+                for (int g = 0; g < NG; ++g) {
+                    tot[g][0] = fmaf(acc[g][h][0], sc.x, tot[g][0]);
+                    tot[g][1] = fmaf(acc[g][h][1], sc.x, tot[g][1]);
+                    tot[g][2] = fmaf(acc[g][h][2], sc.y, tot[g][2]);
+                    tot[g][3] = fmaf(acc[g][h][3], sc.y, tot[g][3]);
+                }
             }
         }
-        // the twenty warps' partial sums meet in shared memory ([tile][component][lane])
+        // the twenty warps' partial sums meet in shared memory ([group][tile][component][lane])
 #pragma unroll
-        for (int r = 0; r < 4; ++r) atomicAdd(acc_s + (t * 4 + r) * 32 + lane, tot[r]);
+        for (int g = 0; g < NG; ++g)
+            if (g < ng)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) atomicAdd(acc_s + ((g * 4 + t) * 4 + r) * 32 + lane, tot[g][r]);
     }
 }
 
 // ------------------------------------------------------------------ swiglu -> phase-2 B fragments
-// One thread per (tile, lane) reads the summed g and u (and clears them for the next item);
-// a = silu(g) * u * w_route goes into the phase-2 B fragments.
+// One thread per (group, tile, lane) reads the summed g and u (and clears them for the next
+// pass); a = silu(g) * u * w_route goes into the group's phase-2 B fragments.
 template <int W>
 __device__ __forceinline__ void swiglu_to_frag(float* acc_s, __half* ah, __nv_bfloat16* abf, const float* wn,
-                                               int ctid) {
+                                               int ctid, int ng) {
     constexpr int NT = slice_rows(W) / 8;
-    if (ctid >= NT * 32) return;
-    const int t = ctid >> 5, lane = ctid & 31;
+    if (ctid >= ng * NT * 32) return;
+    const int g = ctid / (NT * 32), t = (ctid >> 5) % NT, lane = ctid & 31;
     float4 s;
-    float* a4 = acc_s + t * 4 * 32 + lane;
+    float* a4 = acc_s + ((g * 4 + t) * 4) * 32 + lane;
     s.x = a4[0]; s.y = a4[32]; s.z = a4[64]; s.w = a4[96];
     a4[0] = a4[32] = a4[64] = a4[96] = 0.f;
     const int gr = lane >> 2, c = lane & 3;
-    // s.x, s.y: gate of intermediate 8t+gr for tokens 2c, 2c+1; s.z, s.w: up
-    const float a[2] = {s.x / (1.f + __expf(-s.x)) * s.z * wn[2 * c], s.y / (1.f + __expf(-s.y)) * s.w * wn[2 * c + 1]};
+    // s.x, s.y: gate of intermediate 8t+gr for tokens 2c, 2c+1 of the group; s.z, s.w: up
+    const float* w = wn + NTOK * g;
+    const float a[2] = {s.x / (1.f + __expf(-s.x)) * s.z * w[2 * c], s.y / (1.f + __expf(-s.y)) * s.w * w[2 * c + 1]};
     const int i = 8 * t + gr;                     // slice-local intermediate index = k of phase 2
     if constexpr (is_quant(W)) {
         const int q2 = i >> 4, kin = i & 15;
         const int reg = kin >> 3, half = kin & 1, cl = (kin & 7) >> 1;
+        __half* ahg = ah + g * (2 * 32 * 4);
 #pragma unroll
         for (int h = 0; h < 2; ++h)
-            ah[((q2 * 32 + 4 * (2 * c + h) + cl) * 2 + reg) * 2 + half] = __float2half_rn(a[h]);
+            ahg[((q2 * 32 + 4 * (2 * c + h) + cl) * 2 + reg) * 2 + half] = __float2half_rn(a[h]);
     } else {
         // one 16x8x8 step: lane 4n + i/2 holds k = i in half i % 2 of its hi and lo registers
+        __nv_bfloat16* abg = abf + g * (32 * 4);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const __nv_bfloat16 hi = __float2bfloat16_rn(a[h]);
             const __nv_bfloat16 lo = __float2bfloat16_rn(a[h] - __bfloat162float(hi));
             const int ln = 4 * (2 * c + h) + (i >> 1);
-            abf[(ln * 2 + 0) * 2 + (i & 1)] = hi;
-            abf[(ln * 2 + 1) * 2 + (i & 1)] = lo;
+            abg[(ln * 2 + 0) * 2 + (i & 1)] = hi;
+            abg[(ln * 2 + 1) * 2 + (i & 1)] = lo;
         }
     }
 }
 
 // ------------------------------------------------------------------ phase 2: down
+// Each of the warp's four output tiles: one A fragment (one load, one dequantisation) for
+// every token group of the pass; the down scales of the slice's group are applied in fp32.
 template <int W, int G>
 __device__ __forceinline__ void phase_down(const char* slot, const uint2* ah, const uint2* abf, int warp, int lane,
-                                           float (&y)[TILES_PER_WARP][4], bool accumulate) {
+                                           float (&y)[TILES_PER_WARP][NG][4], int ng) {
     const uint2* dw = reinterpret_cast<const uint2*>(slot + gu_w_bytes_of(W) + gu_s_bytes_of(W, G)) + warp * 32 + lane;
     const float* dsc = reinterpret_cast<const float*>(slot + blk_bytes_of(W, G)) + 16 * warp + (lane >> 2);
-    uint2 b0 = make_uint2(0u, 0u), b1 = make_uint2(0u, 0u);
-    if constexpr (is_quant(W)) b0 = ah[lane];
-    else b0 = abf[lane];
-    if constexpr (W == FOCR_W_INT4) b1 = ah[32 + lane];
+    uint2 b0[NG], b1[NG];
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        b0[g] = b1[g] = make_uint2(0u, 0u);
+        if constexpr (is_quant(W)) b0[g] = ah[g * 64 + lane];
+        else b0[g] = abf[g * 32 + lane];
+        if constexpr (W == FOCR_W_INT4) b1[g] = ah[g * 64 + 32 + lane];
+    }
 #pragma unroll
     for (int j = 0; j < TILES_PER_WARP; ++j) {
         const uint2 v = dw[j * NCW * 32];
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (W == FOCR_W_INT4) {
-            mma16816(d, dq_int4(v.x), b0.x, b0.y);
-            mma16816(d, dq_int4(v.y), b1.x, b1.y);
-        } else if constexpr (W == FOCR_W_INT8) {
-            mma16816(d, dq_int8(v.x, v.y), b0.x, b0.y);
-        } else {
-            mma1688_bf16(d, v.x, v.y, b0.x);   // a hi
-            mma1688_bf16(d, v.x, v.y, b0.y);   // a lo
-        }
         float s0 = 1.f, s1 = 1.f;
         if constexpr (is_quant(W)) {
             s0 = dsc[j * NCW * 16];
             s1 = dsc[j * NCW * 16 + 8];
         }
-        if (accumulate) {
-            y[j][0] = fmaf(d[0], s0, y[j][0]);
-            y[j][1] = fmaf(d[1], s0, y[j][1]);
-            y[j][2] = fmaf(d[2], s1, y[j][2]);
-            y[j][3] = fmaf(d[3], s1, y[j][3]);
-        } else {
-            y[j][0] = d[0] * s0;
-            y[j][1] = d[1] * s0;
-            y[j][2] = d[2] * s1;
-            y[j][3] = d[3] * s1;
+        Frag4 a0, a1;
+        if constexpr (W == FOCR_W_INT4) {
+            a0 = dq_int4(v.x);
+            a1 = dq_int4(v.y);
+        } else if constexpr (W == FOCR_W_INT8) {
+            a0 = dq_int8(v.x, v.y);
+        }
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            if (g < ng) {
+                if constexpr (W == FOCR_W_INT4) {
+                    mma16816(d, a0, b0[g].x, b0[g].y);
+                    mma16816(d, a1, b1[g].x, b1[g].y);
+                } else if constexpr (W == FOCR_W_INT8) {
+                    mma16816(d, a0, b0[g].x, b0[g].y);
+                } else {
+                    mma1688_bf16(d, v.x, v.y, b0[g].x);   // a hi
+                    mma1688_bf16(d, v.x, v.y, b0[g].y);   // a lo
+                }
+            }
+            y[j][g][0] = d[0] * s0;
+            y[j][g][1] = d[1] * s0;
+            y[j][g][2] = d[2] * s1;
+            y[j][g][3] = d[3] * s1;
         }
     }
 }
@@ -269,21 +296,21 @@ template <int RW, int SW, int G>
 struct ItemOps {
     static constexpr bool F16 = is_quant(RW) || is_quant(SW);
     static constexpr bool BF16 = !is_quant(RW) || !is_quant(SW);
-    using XF = XFrags<F16, BF16>;
+    using XF = XFrags;
     static __device__ __forceinline__ void gate_up(bool routed, const char* slot, const XF& xf, float* acc, int warp,
-                                                   int lane) {
-        if (routed) phase_gate_up<RW, G>(slot, xf, acc, warp, lane);
-        else phase_gate_up<SW, G>(slot, xf, acc, warp, lane);
+                                                   int lane, int ng) {
+        if (routed) phase_gate_up<RW, G>(slot, xf, acc, warp, lane, ng);
+        else phase_gate_up<SW, G>(slot, xf, acc, warp, lane, ng);
     }
     static __device__ __forceinline__ void swiglu(bool routed, float* acc, __half* ah, __nv_bfloat16* abf,
-                                                  const float* wn, int ctid) {
-        if (routed) swiglu_to_frag<RW>(acc, ah, abf, wn, ctid);
-        else swiglu_to_frag<SW>(acc, ah, abf, wn, ctid);
+                                                  const float* wn, int ctid, int ng) {
+        if (routed) swiglu_to_frag<RW>(acc, ah, abf, wn, ctid, ng);
+        else swiglu_to_frag<SW>(acc, ah, abf, wn, ctid, ng);
     }
     static __device__ __forceinline__ void down(bool routed, const char* slot, const uint2* ah, const uint2* abf,
-                                                int warp, int lane, float (&y)[TILES_PER_WARP][4], bool accumulate) {
-        if (routed) phase_down<RW, G>(slot, ah, abf, warp, lane, y, accumulate);
-        else phase_down<SW, G>(slot, ah, abf, warp, lane, y, accumulate);
+                                                int warp, int lane, float (&y)[TILES_PER_WARP][NG][4], int ng) {
+        if (routed) phase_down<RW, G>(slot, ah, abf, warp, lane, y, ng);
+        else phase_down<SW, G>(slot, ah, abf, warp, lane, y, ng);
     }
 };
 
@@ -300,7 +327,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
     int* rec = reinterpret_cast<int*>(smem + SL::rec);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_shared = p.L.sg.slices;
-    const bool small = p.T <= NTOK;   // one token group for every item, output kept in registers
 
     if (tid == 0) {
         for (int s = 0; s < NSLOT; ++s) {
@@ -311,7 +337,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
         okflag[0] = 1;   // consumer wait result
         okflag[1] = 0;   // abort
     }
-    for (int i = tid; i < 4 * 4 * 32; i += NTHREADS) reinterpret_cast<float*>(smem + SL::acc)[i] = 0.f;
+    for (int i = tid; i < NG * 4 * 4 * 32; i += NTHREADS) reinterpret_cast<float*>(smem + SL::acc)[i] = 0.f;
     __syncthreads();
 
     if (warp == NCW) {
@@ -393,23 +419,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
     const int ctid = tid;
     int* tok = reinterpret_cast<int*>(smem + SL::tok);
     float* wn = reinterpret_cast<float*>(smem + SL::wn);
-    int* ridx = reinterpret_cast<int*>(smem + SL::ridx);
-    float* rw = reinterpret_cast<float*>(smem + SL::rw);
     float* acc = reinterpret_cast<float*>(smem + SL::acc);
     __half* ahh = reinterpret_cast<__half*>(smem + SL::ah);
     __nv_bfloat16* abfh = reinterpret_cast<__nv_bfloat16*>(smem + SL::abf);
     const uint2* ah = reinterpret_cast<const uint2*>(smem + SL::ah);
     const uint2* abf = reinterpret_cast<const uint2*>(smem + SL::abf);
     typename Ops::XF xf;
-    float y[TILES_PER_WARP][4];
-#pragma unroll
-    for (int j = 0; j < TILES_PER_WARP; ++j) y[j][0] = y[j][1] = y[j][2] = y[j][3] = 0.f;
+    float y[TILES_PER_WARP][NG][4];
 
-    if (small) {
-        if (ctid < NTOK) tok[ctid] = ctid < p.T ? ctid : -1;
-        consumer_sync();
-        load_x_frags(p.x, tok, warp, lane, xf);
-    }
     int n_items = p.shared_only ? n_shared : 0x7fffffff;
     bool waited = false;
     for (int it = 0;; ++it) {
@@ -418,10 +435,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
             pdl_wait();
             waited = true;
             n_items = n_shared + p.R.active[E] * p.L.rg.slices;
-            if (small && ctid < p.T * K) {
-                ridx[ctid] = p.R.topk_idx[ctid];
-                rw[ctid] = p.R.topk_w[ctid];
-            }
         }
         if (item >= n_items) break;
         const int slot = it % NSLOT;
@@ -441,72 +454,54 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
         const int expert = rec[slot];
         const bool routed = expert >= 0;
         const char* sbuf = smem + SL::slots + slot * SLOT_BYTES;
-
-        if (small) {
-            if (ctid < NTOK) {
-                // routing weight of every column for this item's expert (0 if not routed)
+        const int ntok = routed ? p.R.counts[expert] : p.T;
+        const int seg = routed ? p.R.offsets[expert] : 0;
+        for (int b0 = 0; b0 < ntok; b0 += NTP) {
+            const int ng = min(NG, (ntok - b0 + NTOK - 1) / NTOK);   // token groups with tokens (CTA-uniform)
+            consumer_sync();   // the previous pass is done with tok / wn
+            if (ctid < NTP) {
+                int tk = -1;
                 float w = 0.f;
-                if (ctid < p.T) {
+                if (b0 + ctid < ntok) {
                     if (!routed) {
+                        tk = b0 + ctid;
                         w = 1.f;
                     } else {
-#pragma unroll
-                        for (int j = 0; j < K; ++j)
-                            if (ridx[ctid * K + j] == expert) w = rw[ctid * K + j];
+                        const int e = p.R.perm[seg + b0 + ctid];
+                        tk = e / K;
+                        w = p.R.topk_w[e];
                     }
                 }
+                tok[ctid] = tk;
                 wn[ctid] = w;
             }
-            Ops::gate_up(routed, sbuf, xf, acc, warp, lane);
             consumer_sync();
-            Ops::swiglu(routed, acc, ahh, abfh, wn, ctid);
+            load_x_frags<Ops::F16, Ops::BF16>(p.x, tok, warp, lane, !is_quant(routed ? RW : SW), xf);
+            Ops::gate_up(routed, sbuf, xf, acc, warp, lane, ng);
             consumer_sync();
-            Ops::down(routed, sbuf, ah, abf, warp, lane, y, true);
-        } else {
-            const int ntok = routed ? p.R.counts[expert] : p.T;
-            const int seg = routed ? p.R.offsets[expert] : 0;
-            for (int b0 = 0; b0 < ntok; b0 += NTOK) {
-                consumer_sync();   // the previous group is done with tok / wn
-                if (ctid < NTOK) {
-                    int tk = -1;
-                    float w = 0.f;
-                    if (b0 + ctid < ntok) {
-                        if (!routed) {
-                            tk = b0 + ctid;
-                            w = 1.f;
-                        } else {
-                            const int e = p.R.perm[seg + b0 + ctid];
-                            tk = e / K;
-                            w = p.R.topk_w[e];
-                        }
-                    }
-                    tok[ctid] = tk;
-                    wn[ctid] = w;
-                }
-                consumer_sync();
-                load_x_frags(p.x, tok, warp, lane, xf);
-                Ops::gate_up(routed, sbuf, xf, acc, warp, lane);
-                consumer_sync();
-                Ops::swiglu(routed, acc, ahh, abfh, wn, ctid);
-                consumer_sync();
-                Ops::down(routed, sbuf, ah, abf, warp, lane, y, false);
-                if (!waited) {
-                    pdl_wait();   // the router zeroes `out` first
-                    waited = true;
-                    if (!p.shared_only) n_items = n_shared + p.R.active[E] * p.L.rg.slices;
-                }
-                const int gr = lane >> 2, c = lane & 3;
-                const int t0 = tok[2 * c], t1 = tok[2 * c + 1];
+            Ops::swiglu(routed, acc, ahh, abfh, wn, ctid, ng);
+            consumer_sync();
+            Ops::down(routed, sbuf, ah, abf, warp, lane, y, ng);
+            if (!waited) {
+                pdl_wait();   // the router initialises `out` first
+                waited = true;
+                if (!p.shared_only) n_items = n_shared + p.R.active[E] * p.L.rg.slices;
+            }
+            const int gr = lane >> 2, c = lane & 3;
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+                if (g >= ng) break;
+                const int t0 = tok[NTOK * g + 2 * c], t1 = tok[NTOK * g + 2 * c + 1];
 #pragma unroll
                 for (int j = 0; j < TILES_PER_WARP; ++j) {
                     const int row = 16 * (warp + NCW * j) + gr;
                     if (t0 >= 0) {
-                        atomicAdd(p.out + (size_t)t0 * H + row, y[j][0]);
-                        atomicAdd(p.out + (size_t)t0 * H + row + 8, y[j][2]);
+                        atomicAdd(p.out + (size_t)t0 * H + row, y[j][g][0]);
+                        atomicAdd(p.out + (size_t)t0 * H + row + 8, y[j][g][2]);
                     }
                     if (t1 >= 0) {
-                        atomicAdd(p.out + (size_t)t1 * H + row, y[j][1]);
-                        atomicAdd(p.out + (size_t)t1 * H + row + 8, y[j][3]);
+                        atomicAdd(p.out + (size_t)t1 * H + row, y[j][g][1]);
+                        atomicAdd(p.out + (size_t)t1 * H + row + 8, y[j][g][3]);
                     }
                 }
             }
@@ -514,22 +509,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_decode_kernel(ExpertParams
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);   // this warp is done with the slot
     }
-    if (small && okflag[1] == 0) {
-        if (!waited) pdl_wait();   // the router zeroes `out` first
-        const int gr = lane >> 2, c = lane & 3;
-#pragma unroll
-        for (int j = 0; j < TILES_PER_WARP; ++j) {
-            const int row = 16 * (warp + NCW * j) + gr;
-            if (2 * c < p.T) {
-                atomicAdd(p.out + (size_t)(2 * c) * H + row, y[j][0]);
-                atomicAdd(p.out + (size_t)(2 * c) * H + row + 8, y[j][2]);
-            }
-            if (2 * c + 1 < p.T) {
-                atomicAdd(p.out + (size_t)(2 * c + 1) * H + row, y[j][1]);
-                atomicAdd(p.out + (size_t)(2 * c + 1) * H + row + 8, y[j][3]);
-            }
-        }
-    }
+    if (!waited) pdl_wait();   // every CTA waits before exiting (keeps the chain of forwards ordered)
 }
 
 int g_num_sms = 0;
@@ -561,6 +541,7 @@ cudaError_t launch_typed(const ExpertParams& p, cudaStream_t st) {
 
 cudaError_t launch_expert_decode(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
                                  bool shared_only, cudaStream_t st) {
+    if (T <= SMALL_T) return cudaErrorInvalidValue;   // batches of up to 8 tokens take the decode kernels
     if (g_num_sms == 0) {
         int dev = 0;
         cudaGetDevice(&dev);
