@@ -198,8 +198,9 @@ focr_status focr_moe_layer_forward_ex(const focr_moe_layer* layer, const float* 
  * layer 0 is a dense SwiGLU MLP): out = D (silu(G x) * (U x)) with G, U [6848, 1280] and
  * D [1280, 6848] (HOST fp32, [out, in] row-major).  Quantisation as focr_moe_pack_weights
  * (int8 with group 128 in the decode recipe; 6848 = 53 x 128 + 64, so the last group of
- * a down row has 64 elements and its own scale).  The forward runs on the grouped expert
- * kernel as a single always-on weight set.
+ * a down row has 64 elements and its own scale).  The forward runs on the MoE layer's
+ * expert kernels as a single always-on weight set (the decode kernels for T <= 8, the
+ * grouped kernel for larger T).
  */
 typedef struct focr_dense_mlp focr_dense_mlp;
 focr_status focr_dense_mlp_pack(const float* w_gate, const float* w_up, const float* w_down, int32_t wtype,
