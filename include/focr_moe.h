@@ -169,17 +169,28 @@ focr_status focr_moe_layer_forward(const focr_moe_layer* layer, const float* hid
  *   - 1 <= T <= FOCR_NOALLOC_T_MAX; a larger T is rejected with FOCR_ERR_INVALID_ARG.
  *   - hidden, out, dbg, stream: as for focr_moe_layer_forward (caller-owned buffers).
  *   - The first call on a device looks up the array's device address and zero-fills
- *     it synchronously; make that first call before any stream capture.  Every later
- *     call clears the control words asynchronously on `stream` before the forward.
+ *     it synchronously; make that first call before any stream capture.  Later calls
+ *     launch only the forward: its control words and partial sums start at zero because
+ *     every forward that completes leaves them zero.
  *   - All calls share the one array and it keeps the last call's contents: calls that
  *     overlap on the GPU (other streams, other host threads) race and give wrong
  *     results.  Serialise them on one stream.
- *   - A device wait that runs out is cleared by the next call rather than reported.
+ *   - A bounded device wait that runs out is not reported by the call itself (the call
+ *     returns before the GPU runs it): focr_moe_check_noalloc reports it.
  */
 #define FOCR_NOALLOC_T_MAX 320
-#define FOCR_NOALLOC_SCRATCH_BYTES 7332352
+#define FOCR_NOALLOC_SCRATCH_BYTES 30844160
 focr_status focr_moe_layer_forward_noalloc(const focr_moe_layer* layer, const float* hidden, int32_t T, float* out,
                                            const focr_moe_route_debug* dbg, void* stream);
+
+/*
+ * focr_moe_check_noalloc -- focr_moe_check for the allocation-free forward's fixed array on
+ * the current device: synchronises `stream` and returns FOCR_OK, or FOCR_ERR_TIMEOUT if a
+ * bounded device wait of an earlier call ran out.  In that case it also zero-fills the
+ * array's control words and partial sums (which that call may have left behind), so the
+ * next call starts clean.  Allocates nothing.
+ */
+focr_status focr_moe_check_noalloc(void* stream);
 
 /* Flags of the *_ex / dense forwards. */
 #define FOCR_FWD_RESIDUAL 1   /* out = hidden + layer(hidden) instead of layer(hidden) */

@@ -2,8 +2,10 @@
 
 Bit-exact: the canonical quantised codes and scales, router expert indices, the
 dispatch (counts, offsets, permutation).  Floating point: the layer output within a
-per-token relative error of 2e-3 (max |gpu - oracle| / max |oracle| over the 1280
-outputs of a token; fp32 accumulation), router weights within 1e-5.
+per-token relative error (max |gpu - oracle| / max |oracle| over the 1280 outputs of a
+token) of 2e-3 on the decode kernels (T <= 8: f16 activations, fp32 accumulation) and
+1e-2 on the tensor-core path (T > 8: bf16 weights and activations in tcgen05 MMAs, fp32
+accumulation), router weights within 1e-5.
 """
 import functools
 import os
@@ -17,7 +19,12 @@ from weight_quantized_expert_b200 import api, synth
 
 pytestmark = pytest.mark.gpu
 NTHREADS = max(1, (os.cpu_count() or 1))
-TOL_DECODE = 2e-3
+TOL_DECODE = 2e-3   # T <= 8
+TOL_TC = 1e-2       # T > 8, bf16 tensor-core path
+
+
+def tol_for(T):
+    return TOL_DECODE if T <= 8 else TOL_TC
 
 W4, W8, WB = synth.W_INT4, synth.W_INT8, synth.W_BF16
 LAYERS = {
@@ -53,7 +60,9 @@ def run_gpu(packed, x, ws=None):
     return r
 
 
-def assert_parity(g, r, tol=TOL_DECODE):
+def assert_parity(g, r, tol=None):
+    if tol is None:
+        tol = tol_for(g["out"].shape[0])
     np.testing.assert_array_equal(g["topk_idx"], r["idx"])
     np.testing.assert_array_max_ulp(g["logits"], r["logits"], maxulp=1)
     np.testing.assert_allclose(g["topk_w"], r["w"], rtol=1e-5, atol=1e-9)
@@ -202,7 +211,7 @@ def test_large_batch_sampled_tokens():
     sample = np.concatenate([[0, T - 1], sample])
     r = om.forward(x[sample], nthreads=NTHREADS)
     err = per_token_rel_err(g["out"][sample], r["out"])
-    assert err.max() <= TOL_DECODE
+    assert err.max() <= TOL_TC
 
 
 def test_forward_rejects_bad_arguments_on_device():

@@ -29,7 +29,7 @@ EXPORTED = (
     "focr_moe_pack_weights", "focr_moe_layer_clone", "focr_moe_layer_free", "focr_moe_layer_device_bytes",
     "focr_moe_export_sizes", "focr_moe_export_quantized", "focr_moe_workspace_bytes",
     "focr_moe_workspace_zero_bytes", "focr_moe_layer_forward",
-    "focr_moe_check", "focr_last_error", "focr_version", "focr_moe_layer_forward_noalloc",
+    "focr_moe_check", "focr_last_error", "focr_version", "focr_moe_layer_forward_noalloc", "focr_moe_check_noalloc",
     "focr_moe_layer_forward_ex", "focr_lm_head_pack", "focr_lm_head_free", "focr_lm_head_export",
     "focr_lm_head_workspace_bytes", "focr_lm_head_gemv", "focr_rmsnorm", "focr_dense_mlp_pack",
     "focr_dense_mlp_free", "focr_dense_mlp_export_quantized", "focr_dense_mlp_forward",
@@ -81,6 +81,7 @@ def lib():
                 "focr_moe_layer_forward": (i32, [P, P, i32, P, P, sz, ctypes.POINTER(RouteDebug), P]),
                 "focr_moe_check": (i32, [P, P]),
                 "focr_moe_layer_forward_noalloc": (i32, [P, P, i32, P, ctypes.POINTER(RouteDebug), P]),
+                "focr_moe_check_noalloc": (i32, [P]),
                 "focr_moe_layer_forward_ex": (i32, [P, P, i32, P, P, sz, ctypes.POINTER(RouteDebug), i32, P]),
                 "focr_lm_head_pack": (i32, [P, ctypes.POINTER(P), P]),
                 "focr_lm_head_free": (None, [P]),
@@ -225,6 +226,11 @@ def focr_moe_layer_forward_noalloc(layer: MoELayer, hidden, out=None, debug: dic
     _check(lib().focr_moe_layer_forward_noalloc(ctypes.c_void_p(layer.handle), _ptr(hidden), T, _ptr(out),
                                                 ctypes.byref(dbg) if dbg is not None else None, _stream(stream)))
     return out
+
+
+def focr_moe_check_noalloc(stream=None):
+    """Report (FocrError TIMEOUT) a device wait of an earlier allocation-free forward that ran out."""
+    _check(lib().focr_moe_check_noalloc(_stream(stream)))
 
 
 def focr_moe_check(workspace, stream=None):

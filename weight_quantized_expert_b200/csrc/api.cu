@@ -15,9 +15,17 @@ using namespace focr;
 struct focr_moe_layer {
     int32_t routed_type, shared_type, group;
     ItemGeom rg, sg;
+    TcGeom rtg, stg;      // tensor-core layout of the routed and shared sets
     uint8_t* dev = nullptr;
     size_t bytes = 0;
     size_t off_router = 0, off_ritems = 0, off_rdsc = 0, off_sitems = 0, off_sdsc = 0;
+    size_t off_tc_rgu = 0, off_tc_rdn = 0, off_tc_sgu = 0, off_tc_sdn = 0;
+    TcView tc_view() const {
+        TcView v{};
+        v.r = TcSetView{dev + off_tc_rgu, dev + off_tc_rdn, rtg};
+        v.s = TcSetView{dev + off_tc_sgu, dev + off_tc_sdn, stg};
+        return v;
+    }
     LayerView view() const {
         LayerView v{};
         v.router = reinterpret_cast<const uint16_t*>(dev + off_router);
@@ -82,6 +90,14 @@ void plan(focr_moe_layer* L) {
     o = align_up(o + (size_t)L->sg.slices * L->sg.item_bytes, 256);
     L->off_sdsc = o;
     o = align_up(o + sizeof(float) * (size_t)L->sg.dscale_expert_floats, 256);
+    L->off_tc_rgu = o;
+    o = align_up(o + (size_t)E * L->rtg.gu_bytes, 256);
+    L->off_tc_rdn = o;
+    o = align_up(o + (size_t)E * L->rtg.dn_bytes, 256);
+    L->off_tc_sgu = o;
+    o = align_up(o + L->stg.gu_bytes, 256);
+    L->off_tc_sdn = o;
+    o = align_up(o + L->stg.dn_bytes, 256);
     L->bytes = o;
 }
 
@@ -120,6 +136,8 @@ focr_status focr_moe_pack_weights(const focr_moe_weights_desc* d, focr_moe_layer
     L->group = d->group_size;
     L->rg = make_geom(d->routed_type, d->group_size, I);
     L->sg = make_geom(d->shared_type, d->group_size, IS);
+    L->rtg = make_tc_geom(d->routed_type, d->group_size, I);
+    L->stg = make_tc_geom(d->shared_type, d->group_size, IS);
     plan(L);
 
     std::vector<uint8_t> host;
@@ -133,13 +151,15 @@ focr_status focr_moe_pack_weights(const focr_moe_weights_desc* d, focr_moe_layer
     const ItemGeom rg = L->rg;
     uint8_t* ritems = host.data() + L->off_ritems;
     float* rdsc = reinterpret_cast<float*>(host.data() + L->off_rdsc);
+    uint8_t* hb = host.data();
     parallel_for(E + 1, [&](int e) {
         if (e < E) {
             host_pack_set(d->w_gate + (size_t)e * I * H, d->w_up + (size_t)e * I * H, d->w_down + (size_t)e * H * I,
-                          rg, ritems + (size_t)e * rg.slices * rg.item_bytes, rdsc + (size_t)e * rg.dscale_expert_floats);
+                          rg, ritems + (size_t)e * rg.slices * rg.item_bytes, rdsc + (size_t)e * rg.dscale_expert_floats,
+                          hb + L->off_tc_rgu + (size_t)e * L->rtg.gu_bytes, hb + L->off_tc_rdn + (size_t)e * L->rtg.dn_bytes);
         } else {
-            host_pack_set(d->ws_gate, d->ws_up, d->ws_down, L->sg, host.data() + L->off_sitems,
-                          reinterpret_cast<float*>(host.data() + L->off_sdsc));
+            host_pack_set(d->ws_gate, d->ws_up, d->ws_down, L->sg, hb + L->off_sitems,
+                          reinterpret_cast<float*>(hb + L->off_sdsc), hb + L->off_tc_sgu, hb + L->off_tc_sdn);
         }
     });
 
@@ -273,7 +293,9 @@ focr_status focr_moe_export_quantized(const focr_moe_layer* L, int32_t matrix, i
 size_t focr_moe_workspace_bytes(int32_t T_max) {
     if (T_max < 1) T_max = 1;
     if (T_max > FOCR_T_MAX) T_max = FOCR_T_MAX;
-    return ws_layout(T_max).total;
+    // sized for both the MoE layer and the dense layer (whose shared-set regions are larger)
+    const size_t a = ws_layout(T_max, IS).total, b = ws_layout(T_max, IS_MAX).total;
+    return a > b ? a : b;
 }
 
 size_t focr_moe_workspace_zero_bytes(void) { return ws_layout(1).a16; }
@@ -288,7 +310,7 @@ focr_status focr_moe_layer_forward_ex(const focr_moe_layer* L, const float* hidd
     if (!hidden || !out || !workspace) return fail(FOCR_ERR_INVALID_ARG, "hidden, out and workspace must not be NULL");
     if (!aligned(hidden, 16) || !aligned(out, 16)) return fail(FOCR_ERR_INVALID_ARG, "hidden/out must be 16-byte aligned");
     if (!aligned(workspace, 256)) return fail(FOCR_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-    const size_t need = ws_layout(T).total;
+    const size_t need = ws_layout(T, IS).total;
     if (ws_bytes < need) return fail(FOCR_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed for T=%d", ws_bytes, need, T);
     {
         const char* h0 = (const char*)hidden;
@@ -297,11 +319,17 @@ focr_status focr_moe_layer_forward_ex(const focr_moe_layer* L, const float* hidd
         if (h0 < o0 + nb && o0 < h0 + nb) return fail(FOCR_ERR_INVALID_ARG, "hidden and out overlap");
     }
     cudaStream_t st = (cudaStream_t)stream;
-    const RouteView R = route_view(workspace, T);
+    const RouteView R = route_view(workspace, T, IS);
     const LayerView V = L->view();
-    CUDA_TRY(launch_router(hidden, T, T, V, R, out, (flags & FOCR_FWD_RESIDUAL) ? hidden : nullptr, st));
-    if (T <= SMALL_T) CUDA_TRY(launch_decode_small(hidden, T, V, R, out, false, st));
-    else CUDA_TRY(launch_expert_decode(hidden, T, V, R, out, false, st));
+    const bool resid = (flags & FOCR_FWD_RESIDUAL) != 0;
+    if (T <= SMALL_T) {
+        CUDA_TRY(launch_router(hidden, T, T, V, R, out, resid ? hidden : nullptr, nullptr, st));
+        CUDA_TRY(launch_decode_small(hidden, T, V, R, out, false, st));
+    } else {
+        const TcWork W = tc_work(workspace, T, IS);
+        CUDA_TRY(launch_router(hidden, T, T, V, R, nullptr, nullptr, W.xrows, st));
+        CUDA_TRY(launch_expert_tc(hidden, T, L->tc_view(), R, W, out, resid, false, st));
+    }
     if (dbg) {
         if (dbg->logits) CUDA_TRY(cudaMemcpyAsync(dbg->logits, R.logits, sizeof(float) * T * E, cudaMemcpyDeviceToDevice, st));
         if (dbg->topk_idx) CUDA_TRY(cudaMemcpyAsync(dbg->topk_idx, R.topk_idx, sizeof(int32_t) * T * K, cudaMemcpyDeviceToDevice, st));
@@ -415,8 +443,9 @@ focr_status focr_moe_layer_forward(const focr_moe_layer* L, const float* hidden,
 struct focr_dense_mlp {
     int32_t wtype, group;
     ItemGeom g;
+    TcGeom tg;
     uint8_t* dev = nullptr;
-    size_t bytes = 0, off_items = 0, off_dsc = 0;
+    size_t bytes = 0, off_items = 0, off_dsc = 0, off_tc_gu = 0, off_tc_dn = 0;
 };
 
 focr_status focr_dense_mlp_pack(const float* w_gate, const float* w_up, const float* w_down, int32_t wtype,
@@ -431,9 +460,12 @@ focr_status focr_dense_mlp_pack(const float* w_gate, const float* w_up, const fl
     M->wtype = wtype;
     M->group = is_quant(wtype) ? group : 0;
     M->g = make_geom(wtype, group, FOCR_DENSE_INTER);
+    M->tg = make_tc_geom(wtype, group, FOCR_DENSE_INTER);
     M->off_items = 0;
     M->off_dsc = align_up((size_t)M->g.slices * M->g.item_bytes, 256);
-    M->bytes = align_up(M->off_dsc + sizeof(float) * (size_t)M->g.dscale_expert_floats, 256);
+    M->off_tc_gu = align_up(M->off_dsc + sizeof(float) * (size_t)M->g.dscale_expert_floats, 256);
+    M->off_tc_dn = align_up(M->off_tc_gu + M->tg.gu_bytes, 256);
+    M->bytes = align_up(M->off_tc_dn + M->tg.dn_bytes, 256);
     std::vector<uint8_t> host;
     try {
         host.assign(M->bytes, 0);
@@ -441,7 +473,8 @@ focr_status focr_dense_mlp_pack(const float* w_gate, const float* w_up, const fl
         delete M;
         return fail(FOCR_ERR_OOM, "host staging of %zu bytes failed", M->bytes);
     }
-    host_pack_set(w_gate, w_up, w_down, M->g, host.data(), reinterpret_cast<float*>(host.data() + M->off_dsc));
+    host_pack_set(w_gate, w_up, w_down, M->g, host.data(), reinterpret_cast<float*>(host.data() + M->off_dsc),
+                  host.data() + M->off_tc_gu, host.data() + M->off_tc_dn);
     cudaError_t e = cudaMalloc(&M->dev, M->bytes);
     if (e != cudaSuccess) {
         delete M;
@@ -509,8 +542,8 @@ focr_status focr_dense_mlp_forward(const focr_dense_mlp* M, const float* x, int3
     if (!x || !out || !workspace) return fail(FOCR_ERR_INVALID_ARG, "x, out and workspace must not be NULL");
     if (!aligned(x, 16) || !aligned(out, 16) || !aligned(workspace, 256))
         return fail(FOCR_ERR_INVALID_ARG, "misaligned x, out or workspace");
-    if (ws_bytes < ws_layout(T).total)
-        return fail(FOCR_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, ws_layout(T).total);
+    if (ws_bytes < ws_layout(T, IS_MAX).total)
+        return fail(FOCR_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, ws_layout(T, IS_MAX).total);
     const size_t nb = (size_t)T * H * sizeof(float);
     {
         const char* a = (const char*)x;
@@ -518,17 +551,24 @@ focr_status focr_dense_mlp_forward(const focr_dense_mlp* M, const float* x, int3
         if (a < b + nb && b < a + nb) return fail(FOCR_ERR_INVALID_ARG, "x and out overlap");
     }
     cudaStream_t st = (cudaStream_t)stream;
-    if (flags & FOCR_FWD_RESIDUAL) CUDA_TRY(cudaMemcpyAsync(out, x, nb, cudaMemcpyDeviceToDevice, st));
-    else CUDA_TRY(cudaMemsetAsync(out, 0, nb, st));
-    LayerView v{};
-    v.shared_items = M->dev + M->off_items;
-    v.shared_dscale = reinterpret_cast<const float*>(M->dev + M->off_dsc);
-    v.routed_items = v.shared_items;
-    v.routed_dscale = v.shared_dscale;
-    v.rg = M->g;
-    v.sg = M->g;
-    if (T <= SMALL_T) CUDA_TRY(launch_decode_small(x, T, v, route_view(workspace, T), out, true, st));
-    else CUDA_TRY(launch_expert_decode(x, T, v, route_view(workspace, T), out, true, st));
+    if (T <= SMALL_T) {
+        if (flags & FOCR_FWD_RESIDUAL) CUDA_TRY(cudaMemcpyAsync(out, x, nb, cudaMemcpyDeviceToDevice, st));
+        else CUDA_TRY(cudaMemsetAsync(out, 0, nb, st));
+        LayerView v{};
+        v.shared_items = M->dev + M->off_items;
+        v.shared_dscale = reinterpret_cast<const float*>(M->dev + M->off_dsc);
+        v.routed_items = v.shared_items;
+        v.routed_dscale = v.shared_dscale;
+        v.rg = M->g;
+        v.sg = M->g;
+        CUDA_TRY(launch_decode_small(x, T, v, route_view(workspace, T, IS_MAX), out, true, st));
+    } else {
+        TcView v{};
+        v.s = TcSetView{M->dev + M->off_tc_gu, M->dev + M->off_tc_dn, M->tg};
+        v.r = v.s;
+        CUDA_TRY(launch_expert_tc(x, T, v, route_view(workspace, T, IS_MAX), tc_work(workspace, T, IS_MAX), out,
+                                  (flags & FOCR_FWD_RESIDUAL) != 0, true, st));
+    }
     return FOCR_OK;
 }
 

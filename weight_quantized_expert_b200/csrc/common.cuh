@@ -98,6 +98,69 @@ struct LayerView {
 };
 
 // ---------------------------------------------------------------------------------------
+// Second device layout of a weight set, read by the tensor-core (tcgen05) grouped kernel
+// for batches of more than 8 tokens.  Every matrix is cut into blocks of 128 rows x 64
+// input columns (one "K-block"); a block is what one pipeline stage of the kernel stages
+// in shared memory, and the blocks of one work unit are consecutive in memory:
+//   gate/up : [tile p of 64 intermediates][20 K-blocks][block]; block row r = 16 j + 8 h + r'
+//             is gate (h = 0) or up (h = 1) row 64 p + 8 j + r' (so a gate row and its up row
+//             sit 8 TMEM lanes apart, inside one warp's quarter of the accumulator)
+//   down    : [m-tile of 128 output rows][inter / 64 K-blocks][block]; block row r is output
+//             row 128 m + r
+// Quantised blocks: codes [128 rows][RB bytes] then f32 scales [128 rows][SPK].  A row's
+// codes come in four pairs (k-core c, k-core c + 4) of 8-element k-cores (one k-core per
+// 16-byte row of the tensor core's shared-memory operand):
+//   int4 (RB = 32): pair c = 8 bytes = two 32-bit words, word 0 k-core c, word 1 k-core c+4;
+//                   element 2m of a k-core in nibble m, element 2m+1 in nibble m+4, q + 8
+//   int8 (RB = 64): pair c = 16 bytes, bytes 0-7 k-core c, bytes 8-15 k-core c+4, q + 128
+// SPK = 64 / g scales per row for g = 32 (k-cores 0-3 use the first, 4-7 the second), one
+// otherwise (for g = 128 each scale is stored with both K-blocks of its group).
+// bf16 blocks: the operand image itself, [16 row groups][8 k-cores][8 rows][8 bf16] (16 KB):
+// the K-major, unswizzled core-matrix layout tcgen05.mma reads from shared memory.
+// ---------------------------------------------------------------------------------------
+constexpr int TC_KB = 64;                  // input columns per K-block
+constexpr int TC_M = 128;                  // rows per block (the MMA's M)
+constexpr int TC_KBH = H / TC_KB;          // 20 K-blocks of a gate/up row
+constexpr int TC_MT = H / TC_M;            // 10 output tiles of a down projection
+
+__host__ __device__ constexpr int tc_spk(int G) { return G >= 64 ? 1 : 64 / G; }
+__host__ __device__ constexpr uint32_t tc_row_bytes(int wtype) { return wtype == FOCR_W_INT4 ? 32u : 64u; }
+__host__ __device__ constexpr uint32_t tc_block_bytes(int wtype, int G) {
+    return is_quant(wtype) ? (uint32_t)TC_M * tc_row_bytes(wtype) + (uint32_t)TC_M * 4u * (uint32_t)tc_spk(G)
+                           : (uint32_t)TC_M * TC_KB * 2u;
+}
+
+struct TcGeom {
+    int wtype, group, inter;
+    int tiles;            // inter / 64 gate/up tiles (= K-blocks of the down projection)
+    uint32_t blk;         // bytes of one block
+    size_t gu_bytes;      // tiles * 20 blocks
+    size_t dn_bytes;      // 10 m-tiles * tiles blocks
+};
+
+__host__ __device__ inline TcGeom make_tc_geom(int wtype, int group, int inter) {
+    TcGeom g{};
+    g.wtype = wtype;
+    g.group = is_quant(wtype) ? group : 0;
+    g.inter = inter;
+    g.tiles = inter / TC_KB;
+    g.blk = tc_block_bytes(wtype, is_quant(wtype) ? group : 64);
+    g.gu_bytes = (size_t)g.tiles * TC_KBH * g.blk;
+    g.dn_bytes = (size_t)TC_MT * g.tiles * g.blk;
+    return g;
+}
+
+struct TcSetView {
+    const uint8_t* gu;    // routed: [64 experts][gu_bytes]; shared: [gu_bytes]
+    const uint8_t* dn;    // routed: [64 experts][dn_bytes]; shared: [dn_bytes]
+    TcGeom g;
+};
+
+struct TcView {
+    TcSetView r, s;       // routed experts, shared (or dense) set
+};
+
+// ---------------------------------------------------------------------------------------
 // Workspace layout (bytes from the workspace base).  Control words first; they are
 // zero on entry and every forward returns them to zero.
 // ---------------------------------------------------------------------------------------
@@ -108,7 +171,7 @@ constexpr int MAX_TB = (FOCR_T_MAX + ROUTER_TB - 1) / ROUTER_TB;
 struct WsLayout {
     // regions that are zero on entry and that every forward leaves zero; their offsets do
     // not depend on T_max, so calls with different T may share one workspace
-    size_t ctrl;          // int32 [MAX_TB tickets][1 global ticket][1 error word][pad]
+    size_t ctrl;          // int32 [MAX_TB tickets][1 global ticket][1 error word][pad][CTRL_TC_WORDS]
     size_t gacc;          // f32 [GU_TILES][32 lanes][4]  gate/up sums of k-split tiles (T <= 8)
     size_t tcnt;          // i32 [GU_TILES]               their arrival counters
     // regions every forward writes before reading
@@ -121,6 +184,12 @@ struct WsLayout {
     size_t offsets;       // i32 [65]
     size_t active;        // i32 [64] experts with tokens, ascending; [64] = U
     size_t perm;          // i32 [T_max*6]
+    // tensor-core grouped path (T > 8 only; size 0 otherwise)
+    size_t xrows;         // bf16 [T_pad][1280]                 tokens as the MMA's B operand rows
+    size_t a_img;         // bf16 [14][TC_AROWS(T_max)][64]     routed a, operand image per K-block
+    size_t a_sh;          // bf16 [shared K-blocks][T_pad][64]  shared-set a, operand image
+    size_t y_slot;        // f32 [T_max*6][1280]                each (token, slot) expert output
+    size_t y_sh;          // f32 [parts][T_max][1280]           shared-set output, per K part
     size_t total;
 };
 
@@ -133,10 +202,23 @@ constexpr int ABF_STEPS = IS_MAX / 8 + E * (I / 8);     // k-steps of 8 intermed
 
 constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-constexpr WsLayout ws_layout(int T_max) {
+// K parts of the shared (or dense) set's down projection in the tensor-core path: the parts'
+// partial outputs are separate and summed by the combine in a fixed order
+__host__ __device__ constexpr int tc_parts(int inter) {
+    return inter / TC_KB / 7 < 1 ? 1 : (inter / TC_KB / 7 > 8 ? 8 : inter / TC_KB / 7);
+}
+__host__ __device__ constexpr int tc_kpp(int inter) {   // K-blocks per part
+    return (inter / TC_KB + tc_parts(inter) - 1) / tc_parts(inter);
+}
+// rows of the routed a image: every expert's segment is padded to a multiple of 16 rows
+__host__ __device__ constexpr size_t tc_arows(int T) { return align_up((size_t)T * K + (size_t)E * 15, 16); }
+
+// `shared_inter`: intermediate width of the shared set the call runs (1792 for the MoE
+// layer, 6848 for the dense layer); it sizes the tensor-core path's shared-set regions
+constexpr WsLayout ws_layout(int T_max, int shared_inter = IS) {
     WsLayout w{};
     size_t o = 0;
-    w.ctrl = o;      o = align_up(o + sizeof(int32_t) * (MAX_TB + 64), 256);
+    w.ctrl = o;      o = align_up(o + sizeof(int32_t) * (MAX_TB + 256), 256);
     w.gacc = o;      o = align_up(o + sizeof(float) * 4 * 32 * (size_t)GU_TILES, 256);
     w.tcnt = o;      o = align_up(o + sizeof(int32_t) * (size_t)GU_TILES, 256);
     w.a16 = o;       o = align_up(o + 8 * 32 * (size_t)A16_STEPS, 256);
@@ -148,6 +230,13 @@ constexpr WsLayout ws_layout(int T_max) {
     w.offsets = o;   o = align_up(o + sizeof(int32_t) * (E + 1), 256);
     w.active = o;    o = align_up(o + sizeof(int32_t) * (E + 1), 256);
     w.perm = o;      o = align_up(o + sizeof(int32_t) * (size_t)T_max * K, 256);
+    const bool tc = T_max > 8;
+    const size_t tpad = align_up((size_t)T_max, 16);
+    w.xrows = o;     o = align_up(o + (tc ? 2 * tpad * H : 0), 256);
+    w.a_img = o;     o = align_up(o + (tc ? (size_t)(I / TC_KB) * tc_arows(T_max) * TC_KB * 2 : 0), 256);
+    w.a_sh = o;      o = align_up(o + (tc ? (size_t)(shared_inter / TC_KB) * tpad * TC_KB * 2 : 0), 256);
+    w.y_slot = o;    o = align_up(o + (tc ? sizeof(float) * (size_t)T_max * K * H : 0), 256);
+    w.y_sh = o;      o = align_up(o + (tc ? sizeof(float) * (size_t)tc_parts(shared_inter) * T_max * H : 0), 256);
     w.total = o;
     return w;
 }
@@ -155,6 +244,14 @@ constexpr WsLayout ws_layout(int T_max) {
 // control-word indices (int32) inside ws.ctrl
 constexpr int CTRL_GLOBAL_TICKET = MAX_TB;
 constexpr int CTRL_ERROR = MAX_TB + 1;
+// counters of the tensor-core grouped kernel (reset by its last CTA)
+constexpr int CTRL_TC = MAX_TB + 8;
+constexpr int TC_WORK = 0;        // next work unit (dynamic scheduler)
+constexpr int TC_EXIT = 1;        // CTAs finished
+constexpr int TC_DN_DONE = 2;     // down-projection units finished
+constexpr int TC_DEP_R = 3;       // [64] gate/up units finished per routed expert
+constexpr int TC_DEP_S = 67;      // [8] gate/up units finished per K part of the shared set
+constexpr int TC_WORDS = 75;
 
 struct RouteView {   // device pointers into the workspace
     int32_t* ctrl;
@@ -171,8 +268,8 @@ struct RouteView {   // device pointers into the workspace
     uint2* abf;
 };
 
-inline RouteView route_view(void* ws, int T_max) {
-    WsLayout L = ws_layout(T_max);
+inline RouteView route_view(void* ws, int T_max, int shared_inter = IS) {
+    WsLayout L = ws_layout(T_max, shared_inter);
     char* b = (char*)ws;
     return RouteView{(int32_t*)(b + L.ctrl), (float*)(b + L.logits),
                      (int32_t*)(b + L.topk_idx), (float*)(b + L.topk_w), (int32_t*)(b + L.counts),
@@ -180,14 +277,40 @@ inline RouteView route_view(void* ws, int T_max) {
                      (float*)(b + L.gacc), (int32_t*)(b + L.tcnt), (uint2*)(b + L.a16), (uint2*)(b + L.abf)};
 }
 
+// workspace regions of the tensor-core grouped path
+struct TcWork {
+    uint16_t* xrows;      // bf16 bits [T_pad][1280]
+    uint16_t* a_img;      // routed a image
+    uint16_t* a_sh;       // shared a image
+    float* y_slot;
+    float* y_sh;
+    int arows;            // rows of the routed a image
+    int tpad;             // T rounded up to 16 (rows of the shared a image)
+};
+
+inline TcWork tc_work(void* ws, int T, int shared_inter) {
+    WsLayout L = ws_layout(T, shared_inter);
+    char* b = (char*)ws;
+    return TcWork{(uint16_t*)(b + L.xrows), (uint16_t*)(b + L.a_img), (uint16_t*)(b + L.a_sh),
+                  (float*)(b + L.y_slot), (float*)(b + L.y_sh), (int)tc_arows(T), (int)align_up((size_t)T, 16)};
+}
+
 // error codes a kernel may store in the error word
 constexpr int DEVERR_FULL_WAIT = 1;
 constexpr int DEVERR_EMPTY_WAIT = 2;
 
 // ------------------------------------------------------------------ launchers (per .cu)
-// resid: NULL zeroes `out` before the experts add into it; otherwise `out` starts as a copy of resid
+// out: NULL leaves the layer output alone (the tensor-core path's combine writes all of it);
+// otherwise resid NULL zeroes `out` before the experts add into it, and a non-NULL resid
+// makes `out` start as a copy of resid.  xrows (nullable): bf16 copy of x, [T][1280].
 cudaError_t launch_router(const float* x, int T, int T_ws, const LayerView& L, const RouteView& R, float* out,
-                          const float* resid, cudaStream_t st);
+                          const float* resid, uint16_t* xrows, cudaStream_t st);
+// Tensor-core grouped path (expert_tc.cu), T > 8: the shared set and the selected experts
+// as tcgen05 GEMMs, then the combine out = resid + shared + sum_j w_j expert_j (fixed
+// order).  shared_only: the dense layer (one always-on set, no routing); it then also
+// writes xrows itself.
+cudaError_t launch_expert_tc(const float* x, int T, const TcView& V, const RouteView& R, const TcWork& W,
+                             float* out, bool resid, bool shared_only, cudaStream_t st);
 cudaError_t launch_expert_decode(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
                                  bool shared_only, cudaStream_t st);
 // T <= SMALL_T: gate/up + swiglu kernel, then the down kernel (decode_small.cu)

@@ -25,9 +25,11 @@ using namespace focr;
 
 namespace {
 
-constexpr WsLayout kNoallocLayout = ws_layout(FOCR_NOALLOC_T_MAX);
+constexpr WsLayout kNoallocLayout = ws_layout(FOCR_NOALLOC_T_MAX, IS);
 static_assert(kNoallocLayout.total == FOCR_NOALLOC_SCRATCH_BYTES, "header constant out of date");
-constexpr size_t kCtrlBytes = kNoallocLayout.logits;    // control words sit before the logits
+// control words, k-split partial sums and their counters: zero before the first forward and
+// left zero by every forward that completes
+constexpr size_t kZeroBytes = kNoallocLayout.a16;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FOCR_NOALLOC_SCRATCH_BYTES];
 
@@ -72,8 +74,29 @@ extern "C" focr_status focr_moe_layer_forward_noalloc(const focr_moe_layer* laye
     void* scratch = nullptr;
     focr_status s = scratch_for_current_device(&scratch);
     if (s != FOCR_OK) return s;
-    // The array keeps the previous call's contents; the control words must start at zero.
-    cudaError_t e = cudaMemsetAsync(scratch, 0, kCtrlBytes, (cudaStream_t)stream);
-    if (e != cudaSuccess) return report_error(FOCR_ERR_CUDA, cudaGetErrorString(e));
+    // Nothing is cleared per call: the array's zero prefix is zero after the first-use fill
+    // and every forward that completes leaves it zero.  A forward whose bounded device wait
+    // ran out may leave it dirty; focr_moe_check_noalloc reports that and restores it.
     return focr_moe_layer_forward(layer, hidden, T, out, scratch, FOCR_NOALLOC_SCRATCH_BYTES, dbg, stream);
+}
+
+extern "C" focr_status focr_moe_check_noalloc(void* stream) {
+    void* scratch = nullptr;
+    focr_status s = scratch_for_current_device(&scratch);
+    if (s != FOCR_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    int32_t* err = reinterpret_cast<int32_t*>((char*)scratch + kNoallocLayout.ctrl) + CTRL_ERROR;
+    int32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, err, sizeof(v), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return report_error(FOCR_ERR_CUDA, cudaGetErrorString(e));
+    if (v == 0) return FOCR_OK;
+    // a wait ran out: the forward that set the word may have left counters and partial sums
+    // behind, so the whole zero prefix (the error word included) is cleared
+    e = cudaMemsetAsync(scratch, 0, kZeroBytes, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return report_error(FOCR_ERR_CUDA, cudaGetErrorString(e));
+    char buf[96];
+    snprintf(buf, sizeof(buf), "device wait ran out (code %d); the scratch array was cleared", v);
+    return report_error(FOCR_ERR_TIMEOUT, buf);
 }

@@ -125,13 +125,93 @@ inline size_t gu_scale_index(int ngk, int t, int gi, int gr, int mat) {
 
 }  // namespace
 
-// Pack one SwiGLU weight set (gate/up [inter, H], down [H, inter]) into item blocks.
+namespace {
+
+// One block (128 rows x 64 input columns, K-block kb) of the tensor-core layout (common.cuh).
+// row_of(r) -> (matrix, row) of block row r.
+template <class RowOf>
+void tc_block(const Quantised* const* m3, const int64_t* cols3, const TcGeom& g, int kb, RowOf&& row_of,
+              uint8_t* blk) {
+    const int wt = g.wtype;
+    std::memset(blk, 0, g.blk);
+    if (wt == FOCR_W_BF16) {
+        for (int r = 0; r < TC_M; ++r) {
+            int mat;
+            int64_t row;
+            row_of(r, mat, row);
+            const Quantised& m = *m3[mat];
+            for (int k = 0; k < TC_KB; ++k) {
+                const uint16_t v = m.b[(size_t)(row * cols3[mat] + kb * TC_KB + k)];
+                const size_t off = ((size_t)(r / 8) * 8 + k / 8) * 128 + (size_t)(r % 8) * 16 + (size_t)(k % 8) * 2;
+                std::memcpy(blk + off, &v, 2);
+            }
+        }
+        return;
+    }
+    const int spk = tc_spk(g.group);
+    const uint32_t rb = tc_row_bytes(wt);
+    float* sc = reinterpret_cast<float*>(blk + (size_t)TC_M * rb);
+    for (int r = 0; r < TC_M; ++r) {
+        int mat;
+        int64_t row;
+        row_of(r, mat, row);
+        const Quantised& m = *m3[mat];
+        const int64_t c0 = (int64_t)kb * TC_KB;
+        for (int k = 0; k < TC_KB; ++k) {
+            const int q = m.q[(size_t)(row * cols3[mat] + c0 + k)];
+            const int kc = k / 8, e = k % 8;
+            const int pair = kc & 3, word = kc >> 2;
+            if (wt == FOCR_W_INT4) {
+                const int nib = (e >> 1) + 4 * (e & 1);
+                uint8_t* wp = blk + (size_t)r * rb + pair * 8 + word * 4;
+                uint32_t w;
+                std::memcpy(&w, wp, 4);
+                w |= (uint32_t)((q + 8) & 0xF) << (4 * nib);
+                std::memcpy(wp, &w, 4);
+            } else {
+                blk[(size_t)r * rb + pair * 16 + word * 8 + e] = (uint8_t)(q + 128);
+            }
+        }
+        for (int h = 0; h < spk; ++h) {
+            const int64_t col = c0 + (int64_t)h * (TC_KB / spk);
+            sc[r * spk + h] = m.s[(size_t)(row * m.ng + col / g.group)];
+        }
+    }
+}
+
+void tc_pack(const Quantised& qg, const Quantised& qu, const Quantised& qd, const TcGeom& g, uint8_t* gu,
+             uint8_t* dn) {
+    const Quantised* m3[3] = {&qg, &qu, &qd};
+    const int64_t cols3[3] = {H, H, g.inter};
+    for (int p = 0; p < g.tiles; ++p)
+        for (int kb = 0; kb < TC_KBH; ++kb)
+            tc_block(m3, cols3, g, kb,
+                     [&](int r, int& mat, int64_t& row) {
+                         mat = (r >> 3) & 1;                      // rows 16 j + 8 h + r': h = 1 is up
+                         row = (int64_t)TC_KB * p + 8 * (r >> 4) + (r & 7);
+                     },
+                     gu + ((size_t)p * TC_KBH + kb) * g.blk);
+    for (int mt = 0; mt < TC_MT; ++mt)
+        for (int kb = 0; kb < g.tiles; ++kb)
+            tc_block(m3, cols3, g, kb,
+                     [&](int r, int& mat, int64_t& row) {
+                         mat = 2;
+                         row = (int64_t)TC_M * mt + r;
+                     },
+                     dn + ((size_t)mt * g.tiles + kb) * g.blk);
+}
+
+}  // namespace
+
+// Pack one SwiGLU weight set (gate/up [inter, H], down [H, inter]) into item blocks and, when
+// tc_gu/tc_dn are given, into the tensor-core layout as well (one quantisation for both).
 void host_pack_set(const float* gate, const float* up, const float* down, const ItemGeom& g, uint8_t* items,
-                   float* dscale) {
+                   float* dscale, uint8_t* tc_gu, uint8_t* tc_dn) {
     const int wt = g.wtype;
     const Quantised qg = quantise(gate, g.inter, H, wt, g.group);
     const Quantised qu = quantise(up, g.inter, H, wt, g.group);
     const Quantised qd = quantise(down, H, g.inter, wt, g.group);
+    if (tc_gu && tc_dn) tc_pack(qg, qu, qd, make_tc_geom(wt, g.group, g.inter), tc_gu, tc_dn);
     const Quantised* m3[3] = {&qg, &qu, &qd};
     const int64_t cols3[3] = {H, H, g.inter};
     const int ngk = is_quant(wt) ? H / g.group : 0;

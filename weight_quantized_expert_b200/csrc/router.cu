@@ -28,6 +28,12 @@ namespace cg = cooperative_groups;
 namespace focr {
 namespace {
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
 constexpr int RT_THREADS = 256;
 constexpr int RC = ROUTER_KSPLIT;         // CTAs per cluster
 constexpr int KCOLS = H / RC;             // 160 columns per CTA
@@ -40,8 +46,9 @@ struct RouterParams {
     int T;
     const uint16_t* wr;
     RouteView R;
-    float* out;
+    float* out;           // NULL: the output is not initialised here
     const float* resid;   // NULL: out starts at zero; else out starts as a copy of resid
+    uint16_t* xrows;      // NULL, or bf16 rows of x [T][1280] for the tensor-core path
 };
 
 // counts / offsets / active list / stable permutation of n = T*6 <= 64 entries, by one warp.
@@ -213,6 +220,21 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
         xs[t][c] = t < nt ? (double)p.x[(size_t)(t0 + t) * H + k0 + c] : 0.0;
     }
     __syncthreads();
+    if (p.xrows) {
+        // this CTA's 160 columns of its tokens, rounded to bf16 (the tensor-core path's B operand)
+        for (int i = tid; i < TB * (KCOLS / 8); i += RT_THREADS) {
+            const int t = i / (KCOLS / 8), kc = i % (KCOLS / 8);
+            if (t < nt) {
+                const double* v = &xs[t][kc * 8];
+                uint4 o;
+                o.x = pack_bf16x2((float)v[0], (float)v[1]);
+                o.y = pack_bf16x2((float)v[2], (float)v[3]);
+                o.z = pack_bf16x2((float)v[4], (float)v[5]);
+                o.w = pack_bf16x2((float)v[6], (float)v[7]);
+                *reinterpret_cast<uint4*>(p.xrows + (size_t)(t0 + t) * H + k0 + kc * 8) = o;
+            }
+        }
+    }
 
     // thread -> (expert e, quarter of the CTA's columns); products are exact in fp64.  With
     // few tokens each token's sum is split over NA interleaved chains (fixed order) so that
@@ -263,14 +285,16 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
         }
     }
     if (r != 0) {
-        // CTAs 1..7 of every cluster initialise the layer output (the expert kernels add into
+        // CTAs 1..7 of every cluster initialise the layer output (the decode kernels add into
         // it after this grid completes)
-        const int nw = (gridDim.x / RC) * (RC - 1), w = tb * (RC - 1) + (r - 1);
-        float4* o4 = reinterpret_cast<float4*>(p.out);
-        const float4* r4 = reinterpret_cast<const float4*>(p.resid);
-        const int n4 = p.T * H / 4;
-        for (int i = w * RT_THREADS + tid; i < n4; i += nw * RT_THREADS)
-            o4[i] = r4 ? r4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (p.out) {
+            const int nw = (gridDim.x / RC) * (RC - 1), w = tb * (RC - 1) + (r - 1);
+            float4* o4 = reinterpret_cast<float4*>(p.out);
+            const float4* r4 = reinterpret_cast<const float4*>(p.resid);
+            const int n4 = p.T * H / 4;
+            for (int i = w * RT_THREADS + tid; i < n4; i += nw * RT_THREADS)
+                o4[i] = r4 ? r4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         return;
     }
 
@@ -369,8 +393,8 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
 }  // namespace
 
 cudaError_t launch_router(const float* x, int T, int /*T_ws*/, const LayerView& L, const RouteView& R, float* out,
-                          const float* resid, cudaStream_t st) {
-    RouterParams p{x, T, L.router, R, out, resid};
+                          const float* resid, uint16_t* xrows, cudaStream_t st) {
+    RouterParams p{x, T, L.router, R, out, resid, xrows};
     const int TB = T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : 8));
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(((T + TB - 1) / TB) * RC);

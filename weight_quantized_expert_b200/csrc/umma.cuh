@@ -1,11 +1,11 @@
 // Blackwell (sm_100a) 5th-generation tensor-core primitives: tcgen05.mma with operands in shared
-// memory and the accumulator in tensor memory (TMEM), for the grouped prefill GEMM.
+// memory and the accumulator in tensor memory (TMEM), used by the tensor-core grouped expert
+// kernel (expert_tc.cu) and checked on their own by focr_tc_selftest (tcgen05_selftest.cu).
 //
-// The encodings follow the PTX forms that the CUTLASS/CuTe sm100 headers issue.  A single-tile check
-// on a B200 (bf16 A[128 x 16] and B[16 x 16] K-major without swizzle, D = A B^T in fp32, one MMA
-// committed to an mbarrier, read back with tcgen05.ld) matched an fp64 host GEMM to 5e-8, and a
-// 128 x 256 x 64 tile (four accumulating k-steps, descriptors advanced by 256 B per k-step with
-// LBO 128 B and SBO 1024 B, 256 TMEM columns read in 16-column slices) to 3e-7.
+// The encodings follow the PTX forms that the CUTLASS/CuTe sm100 headers issue.  Operands are
+// K-major without swizzle: core matrices of 8 rows x 16 bytes stored contiguously, LBO = 128 B
+// between the two core matrices of a 16-wide k-step, SBO = 1024 B between 8-row groups, and the
+// descriptors advance by 256 B per k-step inside a 64-wide K-block.
 #pragma once
 
 #include <stdint.h>
@@ -56,7 +56,8 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc), "r"(zero));
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc), "r"(zero)
+        : "memory");
 }
 
 // The mbarrier in shared memory at `bar_smem` receives one arrival once every MMA this thread
