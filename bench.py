@@ -6,9 +6,10 @@ shared expert) on a B200, through libfocr_moe.
 
 A step is one forward of the layer over one batch of synthetic tokens (router,
 softmax/top-6, dispatch, routed + shared experts, combine).  The default workload
-is a single decode token through an int4 (group 64) layer with bf16 router and
-shared expert.  Steps rotate over 16 packed copies of the layer (~2.2 GB, far
-above the 126 MB L2) and over a pool of distinct input tokens, so the weights
+is the largest single-GPU layer workload: prefill of 289 tokens (273 visual rows +
+16 prompt rows) through an int4 (group 64) layer with bf16 router and shared
+expert, where every expert is hit.  Steps rotate over packed copies of the layer
+(far above the 126 MB L2) and over a pool of distinct token batches, so the weights
 come from HBM.  Under torchrun every rank runs an independent replica (no data
 exchange: the path does not shard), and `value` sums all ranks' tokens over the
 slowest rank's time.  `--impl reference` times the CPU oracle instead.
@@ -34,15 +35,18 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer tokens/s and achieved HBM GB/s (% of B200 peak) vs CPU oracle"
 UNIT = "tokens/s"
 N_COPIES = 16
-DEFAULT_WORKLOAD = "t1_int4_g64"
-PEAK_FALLBACK_GBS = 6650.0
+DEFAULT_WORKLOAD = "prefill289_int4_g64"
+PEAK_FALLBACK_GBS = 6650.0           # profiling recipe's fallback copy bandwidth
+PEAK_FALLBACK_TFLOPS = 1590.0        # ... and cuBLAS bf16 burst throughput
+PEAK_FALLBACK_TFLOPS_SUSTAINED = 1400.0
+GRAPH_STEPS = 160                    # forwards per captured CUDA graph
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -51,26 +55,45 @@ def parse():
     return ap.parse_args()
 
 
-def describe(name: str) -> dict:
+TNAME = {0: "bf16", 1: "int8", 2: "int4"}
+
+
+def describe(name: str, world: int) -> dict:
+    """The workload's config (the same dict in both arms)."""
     from weight_quantized_expert_b200 import synth
+    if name in synth.STEP_WORKLOADS:
+        w = synth.STEP_WORKLOADS[name]
+        d = {"workload": name, "tokens_per_step": w["T"], "kind": w["kind"], "seed": w["seed"],
+             "parallelism": f"replicas x{world}"}
+        if w["kind"] == "stack":
+            d.update(wiring="h <- RMSNorm(h + FFN(h)) per layer (eps 1e-6, gamma 1); lm_head on the last norm",
+                     moe_layers=w["moe_layers"], moe="int4 g64, bf16 router and shared expert",
+                     dense="int8 g128", lm_head="int8 per-row")
+        return d
     w = synth.WORKLOADS[name]
-    tname = {0: "bf16", 1: "int8", 2: "int4"}
-    return {"workload": name, "tokens_per_step": w["T"], "routed": f"{tname[w['routed']]} g{w['group']}",
-            "shared": tname[w["shared"]] if w["shared"] == 0 else f"{tname[w['shared']]} g{w['group']}",
+    return {"workload": name, "tokens_per_step": w["T"], "routed": f"{TNAME[w['routed']]} g{w['group']}",
+            "shared": TNAME[w["shared"]] if w["shared"] == 0 else f"{TNAME[w['shared']]} g{w['group']}",
             "router": "bf16", "seed": w["seed"], "hidden": 1280, "experts": "64 routed top-6 + shared 1792",
-            "l2": f"rotated over {N_COPIES} packed layer copies (> 2 GB, L2 is 126 MB) and distinct inputs"}
+            "parallelism": f"replicas x{world}"}
 
 
-def l2_note(n_copies: int) -> str:
-    return f"rotated over {n_copies} packed layer copies (~{n_copies * 138} MB; L2 is 126 MB) and distinct inputs"
+def precision(T: int):
+    """(dtype, description) of the arithmetic the path runs for a batch of T tokens."""
+    if T > 8:
+        return "bf16", ("tcgen05 MMAs with bf16 operands (int4/int8 weights dequantised to bf16 q*s, "
+                        "activations rounded to bf16), fp32 accumulation in TMEM; router fp64")
+    return "f16", ("mma.sync with f16 operands (int4/int8 codes exact, activations rounded to f16; bf16 "
+                   "weights exact with bf16 hi+lo activations), fp32 accumulation; router fp64")
 
 
 def peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, 'measured'|'fallback')."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return float(d["hbm_gbs"]), "measured"
-    return PEAK_FALLBACK_GBS, "fallback"
+        tf = float(d.get("bf16_tflops", PEAK_FALLBACK_TFLOPS))
+        return float(d["hbm_gbs"]), tf, float(d.get("bf16_tflops_sustained", tf)), "measured"
+    return PEAK_FALLBACK_GBS, PEAK_FALLBACK_TFLOPS, PEAK_FALLBACK_TFLOPS_SUSTAINED, "fallback"
 
 
 def sources_hash(files=None) -> str:
@@ -91,7 +114,7 @@ def sources_hash(files=None) -> str:
 
 
 def profiled_traffic(workload: str):
-    """dram bytes per launch from the committed ncu summary, if it matches these sources."""
+    """DRAM bytes per step from the committed ncu summary, if it matches these sources."""
     for f in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
         txt = open(f).read()
         m_w = re.search(r"^workload:\s*(\S+)", txt, re.M)
@@ -171,87 +194,195 @@ def job_rate(tokens_per_step: int, steps: int, world: int, ms: float) -> float:
 
 # ------------------------------------------------------------------ CPU oracle timing
 
-def oracle_rate(name: str, budget_s: float, max_tokens: int | None = None):
-    """tokens/s of the CPU oracle on a bounded sample of the workload (all host cores)."""
+def _oracle_layer(name: str):
     import oracle
     from weight_quantized_expert_b200 import synth
     w = synth.WORKLOADS[name]
     _, layer = synth.workload(name)
     om = oracle.OracleMoE(layer)
     del layer
-    threads = oracle.max_threads()
     pool = synth.hidden(w["seed"] + 1000, 4096, skew=w.get("skew", False))
-    # calibrate on one token per thread, then size the sample to the budget
-    t0 = time.perf_counter()
-    om.forward(pool[:threads], nthreads=threads)
-    dt = time.perf_counter() - t0
-    per_tok = dt / threads
-    n = max(threads, int(budget_s / max(per_tok, 1e-6)))
-    if max_tokens:
-        n = min(n, max_tokens)
-    n = min(n, pool.shape[0])
-    t0 = time.perf_counter()
-    om.forward(pool[:n], nthreads=threads)
-    dt = time.perf_counter() - t0
-    return n / dt, threads, n, dt, om, pool
+    return om, pool
+
+
+def _timed_tokens(run, pool, batch: int, budget_s: float, threads: int):
+    """Run batches of `batch` tokens until about `budget_s` have passed; returns (tokens, seconds)."""
+    done, total = 0, 0.0
+    while total < budget_s and done + batch <= pool.shape[0]:
+        t0 = time.perf_counter()
+        run(pool[done:done + batch], threads)
+        total += time.perf_counter() - t0
+        done += batch
+    return done, total
+
+
+def oracle_baseline(name: str, budget_s: float = 18.0) -> dict:
+    """The CPU oracle on bounded samples of the workload's tokens: single-threaded, and with its
+    OpenMP loop over tokens on every host core (batches of the workload's own size, so a batch of
+    T tokens keeps min(T, cores) threads busy)."""
+    import oracle
+    from weight_quantized_expert_b200 import synth
+    om, pool = _oracle_layer(name)
+    T = synth.WORKLOADS[name]["T"]
+    cores = oracle.max_threads()
+
+    def run(x, th):
+        om.forward(x, nthreads=th)
+
+    n1, t1 = _timed_tokens(run, pool, 1, budget_s * 0.3, 1)
+    batch = max(T, cores)                       # enough tokens for every core
+    nall, tall = _timed_tokens(run, pool, batch, budget_s * 0.7, cores)
+    used = min(cores, batch)
+    return {"value": nall / tall, "unit": UNIT, "cores": used, "kind": "oracle",
+            "single_thread_value": n1 / t1,
+            "sample": f"{nall} tokens of workload {name} in batches of {batch} through the CPU oracle (plain C, "
+                      f"fp64, OpenMP over tokens, {used} threads) in {tall:.1f} s; single-threaded: {n1} tokens "
+                      f"in {t1:.1f} s; layer quantisation excluded"}
+
+
+def step_oracle_baseline(w: dict, budget_s: float = 12.0) -> dict:
+    """tokens/s of the CPU oracle on a bounded sample of a companion / stack workload."""
+    import oracle
+    from weight_quantized_expert_b200 import synth
+    cores = oracle.max_threads()
+    kind = w["kind"]
+    lm = oracle.OracleLMHead(synth.lm_head(w["seed"])) if kind in ("lm_head", "stack") else None
+    dn = None
+    if kind in ("dense", "stack"):
+        d = synth.dense_mlp(w["seed"])
+        dn = oracle.OracleDense(d.gate, d.up, d.down, oracle.W_INT8, 128)
+        del d
+    om = oracle.OracleMoE(synth.moe_layer(w["seed"], synth.W_INT4, synth.W_BF16, 64)) if kind == "stack" else None
+
+    def run(x, th):
+        if kind == "lm_head":
+            lm.forward(x, nthreads=th)
+        elif kind == "dense":
+            dn.forward(x, nthreads=th)
+        else:
+            h = oracle.rmsnorm(x + dn.forward(x, nthreads=th), eps=1e-6)
+            for _ in range(w["moe_layers"]):
+                h = oracle.rmsnorm(h + om.forward(h, nthreads=th)["out"], eps=1e-6)
+            lm.forward(h, nthreads=th)
+
+    pool = synth.hidden(w["seed"] + 5000, 512)
+    batch = max(1, min(cores, 8)) if kind == "stack" else cores
+    nall, tall = _timed_tokens(run, pool, batch, budget_s, cores)
+    if nall == 0:   # one batch did not fit the budget: time one anyway
+        t0 = time.perf_counter()
+        run(pool[:batch], cores)
+        nall, tall = batch, time.perf_counter() - t0
+    used = min(cores, batch)
+    what = "dense layer 0, 11 MoE layers, RMSNorm, lm_head" if kind == "stack" else kind
+    return {"value": nall / tall, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": f"{nall} tokens through the CPU oracle's {what} in batches of {batch} ({used} threads, "
+                      f"plain C, fp64, OpenMP) in {tall:.1f} s"}
 
 
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: each step is the oracle forward of one batch of the
+    workload's tokens on the host cores, steps capped so the run stays within a few minutes."""
     if rank != 0:
         return
-    from weight_quantized_expert_b200 import synth
     import oracle
+    from weight_quantized_expert_b200 import synth
+    cores = oracle.max_threads()
     if args.workload in synth.STEP_WORKLOADS:
         w = synth.STEP_WORKLOADS[args.workload]
-        cpu = step_oracle_rate(w, budget_s=20.0)
+        cpu = step_oracle_baseline(w, budget_s=60.0)
         v = cpu["value"]
+        dtype = "f64"
         print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
                           "steps": args.steps, "warmup": args.warmup, "ms_per_step": w["T"] / v * 1e3,
-                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                          "data": "synthetic", "config": {"workload": args.workload, "tokens_per_step": w["T"],
-                                                          "kind": w["kind"]},
-                          "cpu_baseline": cpu,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
+                          "data": "synthetic", "config": describe(args.workload, world), "cpu_baseline": cpu,
                           "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
               flush=True)
         return
-    w = synth.WORKLOADS[args.workload]
-    _, layer = synth.workload(args.workload)
-    om = oracle.OracleMoE(layer)
-    del layer
-    threads = oracle.max_threads()
-    T = w["T"]
-    pool = synth.hidden(w["seed"] + 1000, 4096, skew=w.get("skew", False))
-    # one step = the oracle forward of one batch of the workload's tokens (threads over tokens)
+    T = synth.WORKLOADS[args.workload]["T"]
+    om, pool = _oracle_layer(args.workload)
+    used = min(cores, T)
     t0 = time.perf_counter()
-    om.forward(pool[:T], nthreads=threads)
+    om.forward(pool[:T], nthreads=cores)
     per_step = time.perf_counter() - t0
     budget = 150.0
-    steps = args.steps
-    warm = args.warmup
+    steps, warm = args.steps, args.warmup
     if (steps + warm) * per_step > budget:
         warm = min(warm, 1)
         steps = max(1, int(budget / per_step) - warm)
+    span = pool.shape[0] - T
     for i in range(warm):
-        om.forward(pool[(i * T) % 4000:(i * T) % 4000 + T], nthreads=threads)
+        s = (i * T) % span
+        om.forward(pool[s:s + T], nthreads=cores)
     t0 = time.perf_counter()
     for i in range(steps):
-        s = (i * T) % 4000
-        om.forward(pool[s:s + T], nthreads=threads)
+        s = (i * T) % span
+        om.forward(pool[s:s + T], nthreads=cores)
     dt = time.perf_counter() - t0
     value = steps * T / dt
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": steps, "warmup": warm, "ms_per_step": dt / steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": describe(args.workload),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "config": describe(args.workload, world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                              "sample": f"{steps} steps x {T} token(s) of the workload through the CPU oracle "
-                                       f"(plain C, fp64, OpenMP over tokens)"
+                                       f"(plain C, fp64, OpenMP over the step's tokens: {used} threads)"
                                        + ("" if steps == args.steps else
                                           f"; steps capped from {args.steps} to bound the CPU run")},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ timing helpers
+
+def capture_graphs(step, K: int, stream):
+    """CUDA graphs covering exactly K steps: `full` replays of a graph of G = min(K, GRAPH_STEPS)
+    steps, then a tail graph of K mod G steps.  Every graph is replayed once here, so no graph
+    upload or first-launch work falls inside the timed region."""
+    import torch
+    G = min(K, GRAPH_STEPS)
+    graphs = []
+    g_main = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_main, stream=stream):
+        for i in range(G):
+            step(i, torch.cuda.current_stream())
+    graphs.append((g_main, K // G))
+    tail = K % G
+    if tail:
+        g_tail = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_tail, stream=stream):
+            for i in range(tail):
+                step(i, torch.cuda.current_stream())
+        graphs.append((g_tail, 1))
+    with torch.cuda.stream(stream):
+        for g, _ in graphs:
+            g.replay()
+    stream.synchronize()
+    order = [i for i in range(G)] * (K // G) + [i for i in range(tail)]
+    return graphs, order
+
+
+def timed_replay(graphs, stream, world, dev, local_rank):
+    import torch
+    clocks = Clocks(local_rank)
+    clocks.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for g, n in graphs:
+            for _ in range(n):
+                g.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    return max_over_ranks(ev0.elapsed_time(ev1), world, dev), clk
 
 
 # ------------------------------------------------------------------ decode-step companions
@@ -298,11 +429,13 @@ def run_step_workload(args, rank, world, local_rank):
     hb = [torch.empty(T, 1280, device=dev) for _ in range(2)]
     am = torch.empty(T, dtype=torch.int32, device=dev)
     stream = torch.cuda.Stream(device=dev)
-    launches = {"lm_head": 1, "dense": 2}.get(kind, 0)
+    per_dense = 2 if T <= 8 else 2            # (memset or x-rows) + expert kernel(s)
+    per_moe = 3 if T <= 8 else 2
+    launches = {"lm_head": 1, "dense": per_dense}.get(kind, 0)
     if kind == "stack":
-        launches = (2 + 1 + 4 * len(layers) + 1) if T <= 8 else (1 + 1 + 3 * len(layers) + 1)
+        launches = per_dense + 1 + (per_moe + 1) * len(layers) + 1
 
-    def step(x, st, debug_counts=None):
+    def run(x, st, debug_counts=None):
         if kind == "lm_head":
             api.focr_lm_head_gemv(head, x, argmax=am, workspace=lm_ws, stream=st)
             return
@@ -325,45 +458,21 @@ def run_step_workload(args, rank, world, local_rank):
         per = []
         with torch.cuda.stream(stream):
             for j in range(pool_n):
-                step(xs[j], stream, counts)
+                run(xs[j], stream, counts)
                 per.append([int((c > 0).sum().item()) for c in counts])
         stream.synchronize()
         hits = [sum(p[li] for p in per) / pool_n for li in range(len(layers))]
     bytes_step = step_bytes_companion(w, hits)
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            step(xs[i % pool_n], stream)
+            run(xs[i % pool_n], stream)
     stream.synchronize()
-    G = 20 if kind == "stack" else 160
     K = args.steps
-    g_main = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_main, stream=stream):
-        for i in range(G):
-            step(xs[i % pool_n], torch.cuda.current_stream())
-    n_rep = max(1, K // G)
-    K = n_rep * G
-    with torch.cuda.stream(stream):
-        g_main.replay()
-    stream.synchronize()
-    clocks = Clocks(local_rank)
-    clocks.start()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(n_rep):
-            g_main.replay()
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
-    clk = clocks.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    graphs, _ = capture_graphs(lambda i, st: run(xs[i % pool_n], st), K, stream)
+    ms, clk = timed_replay(graphs, stream, world, dev, local_rank)
     ms_step = ms / K
     value = job_rate(T, K, world, ms)
-    peak, peak_kind = peaks()
+    peak, _, _, peak_kind = peaks()
     achieved = bytes_step / (ms_step / 1e3) / 1e9
     # end to end: pinned host x in, the step, the step's result (argmax, or the dense output) out
     out_t = hb[0] if kind == "dense" else am
@@ -374,14 +483,14 @@ def run_step_workload(args, rank, world, local_rank):
     with torch.cuda.stream(stream):
         for _ in range(5):
             dx.copy_(hx, non_blocking=True)
-            step(dx, stream)
+            run(dx, stream)
             hy.copy_(out_t, non_blocking=True)
         stream.synchronize()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(stream)
         for _ in range(K_e2e):
             dx.copy_(hx, non_blocking=True)
-            step(dx, stream)
+            run(dx, stream)
             hy.copy_(out_t, non_blocking=True)
         f1.record(stream)
         stream.synchronize()
@@ -389,18 +498,16 @@ def run_step_workload(args, rank, world, local_rank):
     api.focr_moe_check(ws, stream)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = step_oracle_rate(w)
+        cpu = step_oracle_baseline(w)
     if rank == 0:
-        desc = {"workload": args.workload, "tokens_per_step": T, "kind": kind, "seed": w["seed"],
-                "parallelism": f"replicas x{world}", "graph": f"CUDA graph replay ({G} steps per graph)"}
-        if kind == "stack":
-            desc.update(wiring="h <- RMSNorm(h + FFN(h)) per layer (eps 1e-6, gamma 1); lm_head on the last norm",
-                        moe_layers=len(layers), moe="int4 g64, bf16 router and shared expert "
-                        "(11 device copies of one packed layer)", dense="int8 g128", lm_head="int8 per-row",
-                        l2="one step streams every layer once (> 1.5 GB)")
+        dtype, prec = precision(T)
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
                 "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "f32", "data": "synthetic", "config": desc,
+                "dtype": dtype, "precision": prec, "data": "synthetic", "config": describe(args.workload, world),
+                "timing": {"graph": f"CUDA graph replay ({min(K, GRAPH_STEPS)} steps per graph, every graph "
+                                    "replayed once before the timed region)",
+                           "l2": "one step streams every layer once (> 1.5 GB)" if kind == "stack" else
+                                 "inputs re-read every step"},
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                              "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
                              "kernel": "one step of the workload (all its launches, timed together)",
@@ -412,47 +519,6 @@ def run_step_workload(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
-def step_oracle_rate(w: dict, budget_s: float = 10.0):
-    """tokens/s of the CPU oracle on a bounded sample of a companion / stack workload."""
-    import oracle
-    from weight_quantized_expert_b200 import synth
-    threads = oracle.max_threads()
-    kind = w["kind"]
-    lm = oracle.OracleLMHead(synth.lm_head(w["seed"])) if kind in ("lm_head", "stack") else None
-    dn = None
-    if kind in ("dense", "stack"):
-        d = synth.dense_mlp(w["seed"])
-        dn = oracle.OracleDense(d.gate, d.up, d.down, oracle.W_INT8, 128)
-        del d
-    om = oracle.OracleMoE(synth.moe_layer(w["seed"], synth.W_INT4, synth.W_BF16, 64)) if kind == "stack" else None
-
-    def run(x):
-        if kind == "lm_head":
-            lm.forward(x, nthreads=threads)
-        elif kind == "dense":
-            dn.forward(x, nthreads=threads)
-        else:
-            h = oracle.rmsnorm(x + dn.forward(x, nthreads=threads), eps=1e-6)
-            for _ in range(w["moe_layers"]):
-                h = oracle.rmsnorm(h + om.forward(h, nthreads=threads)["out"], eps=1e-6)
-            lm.forward(h, nthreads=threads)
-
-    n = max(1, min(threads, 8)) if kind == "stack" else threads
-    pool = synth.hidden(w["seed"] + 5000, 512)
-    t0 = time.perf_counter()
-    run(pool[:n])
-    dt = time.perf_counter() - t0
-    done, total = n, dt
-    while total < budget_s and done + n <= pool.shape[0]:
-        t0 = time.perf_counter()
-        run(pool[done:done + n])
-        total += time.perf_counter() - t0
-        done += n
-    return {"value": done / total, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{done} tokens through the CPU oracle's {kind} ({'dense layer 0, 11 MoE layers, RMSNorm, lm_head' if kind == 'stack' else kind}), "
-                      f"{total:.1f} s, batches of {n} tokens (plain C, fp64, OpenMP)"}
-
-
 # ------------------------------------------------------------------ our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -462,13 +528,17 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     w = synth.WORKLOADS[args.workload]
     T = w["T"]
-    x_np, layer = synth.workload(args.workload)
+    _, layer = synth.workload(args.workload)
     base = api.focr_moe_pack_weights(layer)
     del layer
     n_copies = max(1, args.copies)
     copies = [base] + [api.focr_moe_layer_clone(base) for _ in range(n_copies - 1)]
-    pool_n = 64
-    xs_np = synth.hidden(w["seed"] + 2000 + rank, pool_n * T, skew=w.get("skew", False)).reshape(pool_n, T, 1280)
+    pool_n = 64 if T <= 64 else 16
+    if w.get("prefill"):
+        # prefill batches: the workload's own 289 rows first, then other seeded 289-row batches
+        xs_np = np.stack([synth.prefill_hidden(w["seed"] + 100 * j + rank) for j in range(pool_n)])
+    else:
+        xs_np = synth.hidden(w["seed"] + 2000 + rank, pool_n * T, skew=w.get("skew", False)).reshape(pool_n, T, 1280)
     xs = torch.from_numpy(xs_np).to(dev)
     outs = torch.empty(pool_n, T, 1280, device=dev)
     ws = api.new_workspace(T, dev)
@@ -477,7 +547,7 @@ def run_ours(args, rank, world, local_rank):
     def step(i, st=None):
         api.focr_moe_layer_forward(copies[i % n_copies], xs[i % pool_n], outs[i % pool_n], ws, stream=st)
 
-    # experts hit per step (for the algorithmic bytes): route each pool entry once
+    # experts hit per batch (for the algorithmic bytes): route each pool entry once
     hits = []
     counts = torch.empty(64, dtype=torch.int32, device=dev)
     with torch.cuda.stream(stream):
@@ -487,76 +557,42 @@ def run_ours(args, rank, world, local_rank):
     stream.synchronize()
     step_bytes = [roofline.moe_layer_bytes(T, w["routed"], w["shared"], w["group"], h) for h in hits]
 
-    # warm-up (eager), then capture the K timed steps in CUDA graphs
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             step(i, stream)
     stream.synchronize()
-    G = 160
-    graphs = []
-    use_graph = not args.eager
-    graph_error = "--eager"
-    try:
-        if not use_graph:
-            raise RuntimeError("--eager")
-        g_main = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_main, stream=stream):
-            for i in range(G):
-                step(i, torch.cuda.current_stream())
-        tail = args.steps % G
-        g_tail = None
-        if tail:
-            g_tail = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g_tail, stream=stream):
-                for i in range(tail):
-                    step(i, torch.cuda.current_stream())
-        graphs = (g_main, g_tail)
-    except Exception as exc:  # reported in the JSON line
-        use_graph = False
-        graph_error = str(exc).splitlines()[0]
-    if use_graph:
+    K = args.steps
+    if args.eager:
+        clocks = Clocks(local_rank)
+        clocks.start()
+        torch.cuda.synchronize(dev)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
-            graphs[0].replay()
-        stream.synchronize()
-
-    clocks = Clocks(local_rank)
-    clocks.start()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        if use_graph:
-            for _ in range(args.steps // G):
-                graphs[0].replay()
-            if graphs[1] is not None:
-                graphs[1].replay()
-        else:
-            for i in range(args.steps):
+            ev0.record(stream)
+            for i in range(K):
                 step(i, stream)
-        ev1.record(stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
-    clk = clocks.stop()
-    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
-    # steps in the timed graph replay follow the same i % pool order
-    order = [i % G for i in range(G)]
-    if use_graph:
-        per_graph = [step_bytes[i % pool_n] for i in order]
-        avg_bytes = sum(per_graph) / len(per_graph)
+            ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        clk = clocks.stop()
+        ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+        order = list(range(K))
+        graph_note = "eager launches"
     else:
-        avg_bytes = sum(step_bytes[i % pool_n] for i in range(args.steps)) / args.steps
-    ms_per_step = ms / args.steps
-    value = job_rate(T, args.steps, world, ms)
-    peak, peak_kind = peaks()
+        graphs, order = capture_graphs(step, K, stream)
+        ms, clk = timed_replay(graphs, stream, world, dev, local_rank)
+        graph_note = (f"CUDA graph replay ({min(K, GRAPH_STEPS)} forwards per graph, every graph replayed once "
+                      "before the timed region)")
+    avg_bytes = sum(step_bytes[i % pool_n] for i in order) / len(order)
+    ms_per_step = ms / K
+    value = job_rate(T, K, world, ms)
+    peak, tf_burst, tf_sus, peak_kind = peaks()
     achieved = avg_bytes / (ms_per_step / 1e3) / 1e9
     traffic = profiled_traffic(args.workload)
+    flops = roofline.moe_layer_flops(T)
+    tflops = flops / (ms_per_step / 1e3) / 1e12
 
     # end to end through the C ABI with host buffers: H2D of x, forward, D2H of out
-    K_e2e = min(args.steps, 2000)
+    K_e2e = min(K, 2000)
     hx = torch.from_numpy(xs_np[:8].copy()).pin_memory()
     hy = torch.empty(8, T, 1280).pin_memory()
     dx = torch.empty(T, 1280, device=dev)
@@ -584,27 +620,33 @@ def run_ours(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, threads, n, dt, _, _ = oracle_rate(args.workload, budget_s=12.0)
-        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"{n} tokens of workload {args.workload} through the CPU oracle (plain C, fp64, "
-                         f"OpenMP over tokens) in {dt:.1f} s; layer quantisation excluded"}
+        cpu = oracle_baseline(args.workload)
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        dtype, prec = precision(T)
+        kernel = ("one layer forward: router -> gate/up -> down kernels, chained by programmatic dependent "
+                  "launch (timed together)" if T <= 8 else
+                  "one layer forward: router -> tensor-core grouped expert kernel (tcgen05, TMEM), chained by "
+                  "programmatic dependent launch (timed together)")
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": traffic, "peak_kind": peak_kind, "kernel": kernel,
+                "algorithmic_bytes_per_step": avg_bytes,
+                "nominal_peak_gbs": 7700.0, "frac_of_nominal": achieved / 7700.0,
+                "tensor": {"achieved_tflops": tflops, "algorithmic_flops_per_step": flops,
+                           "peak_tflops": tf_sus, "frac": tflops / tf_sus,
+                           "peak_note": f"bf16 dense, sustained ({peak_kind}); burst {tf_burst}"}}
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                "config": dict(describe(args.workload), parallelism=f"replicas x{world}", l2=l2_note(n_copies),
-                               graph=("CUDA graph replay" if use_graph else f"eager ({graph_error})")),
-                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                             "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
-                             "kernel": ("one layer forward: router -> gate/up -> down kernels, chained by "
-                                        "programmatic dependent launch (timed together)" if T <= 8 else
-                                        "one layer forward: router -> grouped expert kernel, chained by "
-                                        "programmatic dependent launch (timed together)"),
-                             "algorithmic_bytes_per_step": avg_bytes},
+                "scaling": "weak", "vs_baseline": None, "dtype": dtype, "precision": prec, "data": "synthetic",
+                "config": describe(args.workload, world),
+                "timing": {"graph": graph_note,
+                           "l2": f"rotated over {n_copies} packed layer copies "
+                                 f"(~{n_copies * base.device_bytes // 2**20} MB; L2 is 126 MB) and {pool_n} "
+                                 "distinct token batches"},
+                "roofline": roof,
                 "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * 1280 * 4,
                         "d2h_bytes_per_step": T * 1280 * 4, "steps": K_e2e},
-                "gpu_launches": (3 if T <= 8 else 2) * args.steps,
+                "gpu_launches": (3 if T <= 8 else 2) * K,
                 "clocks": clk}
         print(json.dumps(line), flush=True)
     del copies

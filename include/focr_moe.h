@@ -179,7 +179,7 @@ focr_status focr_moe_layer_forward(const focr_moe_layer* layer, const float* hid
  *     returns before the GPU runs it): focr_moe_check_noalloc reports it.
  */
 #define FOCR_NOALLOC_T_MAX 320
-#define FOCR_NOALLOC_SCRATCH_BYTES 30844160
+#define FOCR_NOALLOC_SCRATCH_BYTES 38216960
 focr_status focr_moe_layer_forward_noalloc(const focr_moe_layer* layer, const float* hidden, int32_t T, float* out,
                                            const focr_moe_route_debug* dbg, void* stream);
 
@@ -272,6 +272,18 @@ focr_status focr_lm_head_gemv(const focr_lm_head* head, const float* x, int32_t 
  * fp32 [1280] or NULL.  Asynchronous on `stream`.
  */
 focr_status focr_rmsnorm(const float* x, const float* gamma, int32_t T, float eps, float* out, void* stream);
+
+/*
+ * focr_tc_selftest -- diagnostic: one tensor-core tile through the library's tcgen05 primitives
+ * (the ones the T > 8 grouped kernel uses), to check them against a host GEMM.
+ * D[128, n] = A[128, k] * B[n, k]^T with A, B bf16 bit patterns (DEVICE, row-major, 16-byte
+ * aligned) and D fp32 (DEVICE); the MMA reads A from shared memory (a_from_tmem = 0) or from
+ * tensor memory after tcgen05.st (a_from_tmem = 1).  n: multiple of 16 in [16, 256]; k: multiple
+ * of 64 in [64, 256].  *err (DEVICE int32) is set to 1 if the kernel's bounded wait ran out.
+ * Asynchronous on `stream`.  (A check of the hardware path, not part of the layer.)
+ */
+focr_status focr_tc_selftest(const uint16_t* a, const uint16_t* b, int32_t n, int32_t k, int32_t a_from_tmem,
+                             float* d, int32_t* err, void* stream);
 
 /* Thread-local description of the last error (empty string if none). */
 const char* focr_last_error(void);

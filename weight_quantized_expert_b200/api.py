@@ -32,7 +32,7 @@ EXPORTED = (
     "focr_moe_check", "focr_last_error", "focr_version", "focr_moe_layer_forward_noalloc", "focr_moe_check_noalloc",
     "focr_moe_layer_forward_ex", "focr_lm_head_pack", "focr_lm_head_free", "focr_lm_head_export",
     "focr_lm_head_workspace_bytes", "focr_lm_head_gemv", "focr_rmsnorm", "focr_dense_mlp_pack",
-    "focr_dense_mlp_free", "focr_dense_mlp_export_quantized", "focr_dense_mlp_forward",
+    "focr_dense_mlp_free", "focr_dense_mlp_export_quantized", "focr_dense_mlp_forward", "focr_tc_selftest",
 )
 FWD_RESIDUAL = 1
 NOALLOC_T_MAX = 320
@@ -93,6 +93,7 @@ def lib():
                 "focr_dense_mlp_free": (None, [P]),
                 "focr_dense_mlp_export_quantized": (i32, [P, i32, P, sz, P, sz]),
                 "focr_dense_mlp_forward": (i32, [P, P, i32, P, P, sz, i32, P]),
+                "focr_tc_selftest": (i32, [P, P, i32, i32, i32, P, P, P]),
                 "focr_last_error": (ctypes.c_char_p, []),
                 "focr_version": (ctypes.c_char_p, []),
             }
@@ -337,3 +338,15 @@ def focr_dense_mlp_forward(mlp: DenseMLP, x, out=None, workspace=None, flags: in
     _check(lib().focr_dense_mlp_forward(ctypes.c_void_p(mlp.handle), _ptr(x), T, _ptr(out), _ptr(workspace),
                                         workspace.numel(), int(flags), _stream(stream)))
     return out
+
+
+def focr_tc_selftest(a, b, a_from_tmem: bool, stream=None):
+    """D = a @ b.T (fp32) through the library's tcgen05 tile primitives; a [128, k], b [n, k] bf16
+    device tensors.  Returns (D, err) with err nonzero if the kernel's bounded wait ran out."""
+    import torch
+    assert a.dtype == torch.bfloat16 and b.dtype == torch.bfloat16 and a.is_cuda and b.is_cuda
+    n, k = b.shape
+    d = torch.empty(128, n, dtype=torch.float32, device=a.device)
+    err = torch.zeros(1, dtype=torch.int32, device=a.device)
+    _check(lib().focr_tc_selftest(_ptr(a), _ptr(b), n, k, int(a_from_tmem), _ptr(d), _ptr(err), _stream(stream)))
+    return d, err

@@ -323,11 +323,11 @@ focr_status focr_moe_layer_forward_ex(const focr_moe_layer* L, const float* hidd
     const LayerView V = L->view();
     const bool resid = (flags & FOCR_FWD_RESIDUAL) != 0;
     if (T <= SMALL_T) {
-        CUDA_TRY(launch_router(hidden, T, T, V, R, out, resid ? hidden : nullptr, nullptr, st));
+        CUDA_TRY(launch_router(hidden, T, T, V, R, out, resid ? hidden : nullptr, nullptr, 0, st));
         CUDA_TRY(launch_decode_small(hidden, T, V, R, out, false, st));
     } else {
         const TcWork W = tc_work(workspace, T, IS);
-        CUDA_TRY(launch_router(hidden, T, T, V, R, nullptr, nullptr, W.xrows, st));
+        CUDA_TRY(launch_router(hidden, T, T, V, R, nullptr, nullptr, W.x_img, W.tpad, st));
         CUDA_TRY(launch_expert_tc(hidden, T, L->tc_view(), R, W, out, resid, false, st));
     }
     if (dbg) {

@@ -185,7 +185,8 @@ struct WsLayout {
     size_t active;        // i32 [64] experts with tokens, ascending; [64] = U
     size_t perm;          // i32 [T_max*6]
     // tensor-core grouped path (T > 8 only; size 0 otherwise)
-    size_t xrows;         // bf16 [T_pad][1280]                 tokens as the MMA's B operand rows
+    size_t x_img;         // bf16 [20][T_pad][64]               x in token order, operand image per K-block
+    size_t x_img_r;       // bf16 [20][TC_AROWS(T_max)][64]     x in dispatch order (each expert's rows)
     size_t a_img;         // bf16 [14][TC_AROWS(T_max)][64]     routed a, operand image per K-block
     size_t a_sh;          // bf16 [shared K-blocks][T_pad][64]  shared-set a, operand image
     size_t y_slot;        // f32 [T_max*6][1280]                each (token, slot) expert output
@@ -232,7 +233,8 @@ constexpr WsLayout ws_layout(int T_max, int shared_inter = IS) {
     w.perm = o;      o = align_up(o + sizeof(int32_t) * (size_t)T_max * K, 256);
     const bool tc = T_max > 8;
     const size_t tpad = align_up((size_t)T_max, 16);
-    w.xrows = o;     o = align_up(o + (tc ? 2 * tpad * H : 0), 256);
+    w.x_img = o;     o = align_up(o + (tc ? 2 * tpad * H : 0), 256);
+    w.x_img_r = o;   o = align_up(o + (tc ? (size_t)TC_KBH * tc_arows(T_max) * TC_KB * 2 : 0), 256);
     w.a_img = o;     o = align_up(o + (tc ? (size_t)(I / TC_KB) * tc_arows(T_max) * TC_KB * 2 : 0), 256);
     w.a_sh = o;      o = align_up(o + (tc ? (size_t)(shared_inter / TC_KB) * tpad * TC_KB * 2 : 0), 256);
     w.y_slot = o;    o = align_up(o + (tc ? sizeof(float) * (size_t)T_max * K * H : 0), 256);
@@ -251,7 +253,8 @@ constexpr int TC_EXIT = 1;        // CTAs finished
 constexpr int TC_DN_DONE = 2;     // down-projection units finished
 constexpr int TC_DEP_R = 3;       // [64] gate/up units finished per routed expert
 constexpr int TC_DEP_S = 67;      // [8] gate/up units finished per K part of the shared set
-constexpr int TC_WORDS = 75;
+constexpr int TC_DEP_X = 75;      // [64] token rows of each routed expert gathered
+constexpr int TC_WORDS = 139;
 
 struct RouteView {   // device pointers into the workspace
     int32_t* ctrl;
@@ -278,8 +281,17 @@ inline RouteView route_view(void* ws, int T_max, int shared_inter = IS) {
 }
 
 // workspace regions of the tensor-core grouped path
+// Operand images (bf16, K-major core-matrix layout of the tensor core's shared-memory operand):
+// element (row r, k) of K-block kb sits at [kb][r / 8][(k % 64) / 8][r % 8][k % 8], so the rows
+// [r0, r0 + N) of one K-block (r0 a multiple of 8) are N * 128 contiguous bytes.
+__host__ __device__ inline size_t img_index(int rows, int r, int k) {
+    return ((size_t)(k / TC_KB) * rows + (size_t)(r & ~7)) * TC_KB + (size_t)((k % TC_KB) / 8) * 64 + (r & 7) * 8 +
+           (k & 7);
+}
+
 struct TcWork {
-    uint16_t* xrows;      // bf16 bits [T_pad][1280]
+    uint16_t* x_img;      // x in token order (tpad rows)
+    uint16_t* x_img_r;    // x rows in dispatch order (arows rows)
     uint16_t* a_img;      // routed a image
     uint16_t* a_sh;       // shared a image
     float* y_slot;
@@ -291,7 +303,7 @@ struct TcWork {
 inline TcWork tc_work(void* ws, int T, int shared_inter) {
     WsLayout L = ws_layout(T, shared_inter);
     char* b = (char*)ws;
-    return TcWork{(uint16_t*)(b + L.xrows), (uint16_t*)(b + L.a_img), (uint16_t*)(b + L.a_sh),
+    return TcWork{(uint16_t*)(b + L.x_img), (uint16_t*)(b + L.x_img_r), (uint16_t*)(b + L.a_img), (uint16_t*)(b + L.a_sh),
                   (float*)(b + L.y_slot), (float*)(b + L.y_sh), (int)tc_arows(T), (int)align_up((size_t)T, 16)};
 }
 
@@ -302,13 +314,13 @@ constexpr int DEVERR_EMPTY_WAIT = 2;
 // ------------------------------------------------------------------ launchers (per .cu)
 // out: NULL leaves the layer output alone (the tensor-core path's combine writes all of it);
 // otherwise resid NULL zeroes `out` before the experts add into it, and a non-NULL resid
-// makes `out` start as a copy of resid.  xrows (nullable): bf16 copy of x, [T][1280].
+// makes `out` start as a copy of resid.
 cudaError_t launch_router(const float* x, int T, int T_ws, const LayerView& L, const RouteView& R, float* out,
-                          const float* resid, uint16_t* xrows, cudaStream_t st);
+                          const float* resid, uint16_t* x_img, int img_rows, cudaStream_t st);
 // Tensor-core grouped path (expert_tc.cu), T > 8: the shared set and the selected experts
 // as tcgen05 GEMMs, then the combine out = resid + shared + sum_j w_j expert_j (fixed
 // order).  shared_only: the dense layer (one always-on set, no routing); it then also
-// writes xrows itself.
+// writes the x image itself.
 cudaError_t launch_expert_tc(const float* x, int T, const TcView& V, const RouteView& R, const TcWork& W,
                              float* out, bool resid, bool shared_only, cudaStream_t st);
 cudaError_t launch_expert_decode(const float* x, int T, const LayerView& L, const RouteView& R, float* out,

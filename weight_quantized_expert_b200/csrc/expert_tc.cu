@@ -50,21 +50,24 @@ namespace {
 constexpr int NSTG = 8;                          // stager warps
 constexpr int NEPI = 4;                          // epilogue warps
 constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_STG = 2, WARP_EPI = WARP_STG + NSTG;
-constexpr int NWARPS = WARP_EPI + NEPI;
+constexpr int WARP_COPY = WARP_EPI + NEPI;       // streams quantised blocks into the raw ring
+constexpr int WARP_BLD = WARP_COPY + 1;          // fills operand stages by copy: bf16 A, token rows, a rows
+constexpr int NWARPS = WARP_BLD + 1;
 constexpr int NTHREADS = NWARPS * 32;
 constexpr int NCH = 128;                         // tokens of one unit at most (the MMA's N)
-constexpr int NAB = 4;                           // operand stages
+constexpr int NAB = 5;                           // operand stages
+constexpr int NPAIR = NSTG / 2;                  // stager warp pairs, one operand stage each in turn
 constexpr uint32_t A_BYTES = TC_M * TC_KB * 2;   // 16 KB bf16 A block
 constexpr uint32_t B_BYTES = NCH * TC_KB * 2;    // 16 KB bf16 B block
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr uint32_t RAW_BUDGET = 72 * 1024;       // quantised blocks in flight
-constexpr int UR = 4;                            // unit descriptors in flight
+constexpr uint32_t RAW_BUDGET = 46 * 1024;       // quantised blocks in flight (plus L2 prefetch)
+constexpr int UR = 6;                            // unit descriptors in flight
 constexpr int NACC = 4;                          // TMEM accumulators of 128 columns
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s
 constexpr int DEVERR_TC_WAIT = 3;
 
-enum UnitKind { UK_GU_S = 0, UK_GU_R = 1, UK_DN_S = 2, UK_DN_R = 3, UK_END = 4 };
+enum UnitKind { UK_GU_S = 0, UK_GU_R = 1, UK_DN_S = 2, UK_DN_R = 3, UK_XG = 4, UK_END = 5 };
 
 struct Unit {
     int kind, expert, tile, part;
@@ -72,14 +75,16 @@ struct Unit {
     int ntok, N;         // tokens of the chunk, N = ntok rounded up to 16
     int c0;              // first token of the chunk: shared, a token id; routed, an index in the expert's segment
     int arow;            // first row of the chunk in the a image
-    int dep, target;     // completion counter (index into the tensor-core control words); down: value to wait for
+    int wdep, wtarget;   // counter (index into the tensor-core control words) to wait for before the B loads, -1: none
+    int ddep;            // counter this unit's completion adds to
+    int seg;             // routed: first dispatch entry of the chunk (index into the permutation)
     int ent[NCH];        // routed: dispatch entries t * 6 + j of the chunk's tokens
     float w[NCH];        // routed gate/up: their routing weights
 };
 
 struct Sched {
     int T, U, nchs, cs_s, P, KPP;
-    int n_gu_s, n_gu_r, n_dn_s, n_dn_r, total;
+    int n_xg, n_gu_s, n_gu_r, n_dn_s, n_dn_r, total;
     int e[E], n[E], off[E], poff[E], nch[E], cs[E];
     int gu_pre[E + 1], dn_pre[E + 1];
 };
@@ -192,24 +197,26 @@ __device__ __forceinline__ uint4 dq_int8_bf16(uint32_t w0, uint32_t w1, float s)
                       f32x2_to_bf16x2(f[6], f[7]));
 }
 
-// Stager warp sw (0..7) turns rows 16 sw .. 16 sw + 15 of a quantised block into the bf16 A
-// operand: lane (pair pr = lane / 8, row rr = lane % 8) writes k-cores pr and pr + 4 of rows
-// 16 sw + rr and 16 sw + 8 + rr; each warp store covers 512 contiguous bytes.
+// Warp hw (0, 1) of a stager pair turns block rows 64 hw .. 64 hw + 63 of a quantised block into
+// the bf16 A operand: lane (pr = lane / 8, rr = lane % 8) writes k-cores pr and pr + 4 of rows
+// 8 g + rr of each of the warp's eight row groups g; every warp store covers 512 contiguous bytes.
 template <int W, int G>
-__device__ __forceinline__ void dequant_block(const uint8_t* raw, char* A, int sw, int lane) {
+__device__ __forceinline__ void dequant_half(const uint8_t* raw, char* A, int hw, int lane) {
     constexpr int SPK = tc_spk(G);
     constexpr uint32_t RB = tc_row_bytes(W);
     const float* sc = reinterpret_cast<const float*>(raw + TC_M * RB);
     const int pr = lane >> 3, rr = lane & 7;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int row = 16 * sw + 8 * h + rr;
+#pragma unroll 4
+    for (int gg = 0; gg < 8; ++gg) {
+        const int g = 8 * hw + gg;          // row group
+        const int row = 8 * g + rr;
         const float s0 = sc[row * SPK], s1 = sc[row * SPK + SPK - 1];
-        char* d0 = A + (2 * sw + h) * 1024 + pr * 128 + rr * 16;
+        char* d0 = A + g * 1024 + pr * 128 + rr * 16;
         if constexpr (W == FOCR_W_INT4) {
             const uint2 c = lds64(raw + row * 32 + pr * 8);
-            sts128(d0, dq_int4_bf16(c.x, f32x2_to_bf16x2(s0, s0)));
-            sts128(d0 + 512, dq_int4_bf16(c.y, f32x2_to_bf16x2(s1, s1)));
+            const uint32_t b0 = f32x2_to_bf16x2(s0, s0);
+            sts128(d0, dq_int4_bf16(c.x, b0));
+            sts128(d0 + 512, dq_int4_bf16(c.y, SPK == 1 ? b0 : f32x2_to_bf16x2(s1, s1)));
         } else {
             const uint4 c = lds128(raw + row * 64 + pr * 16);
             sts128(d0, dq_int8_bf16(c.x, c.y, s0));
@@ -252,16 +259,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int i = 0; i < NAB; ++i) {
-            mbar_init(&ab_full[i], NSTG);
+            mbar_init(&ab_full[i], 2 + 1);   // the dequantising pair's two warps + the loader
             mbar_init(&ab_empty[i], 1);
         }
         for (int i = 0; i < NR; ++i) {
             mbar_init(&raw_full[i], 1);
-            mbar_init(&raw_empty[i], NSTG);
+            mbar_init(&raw_empty[i], 2);
         }
         for (int i = 0; i < UR; ++i) {
             mbar_init(&u_full[i], 1);
-            mbar_init(&u_empty[i], NSTG + 1 + NEPI);
+            mbar_init(&u_empty[i], NSTG + 1 + NEPI + 2);
         }
         for (int i = 0; i < NACC; ++i) {
             mbar_init(&acc_full[i], 1);
@@ -348,17 +355,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             S.nchs = (T + S.cs_s - 1) / S.cs_s;
             S.P = tc_parts(sg.inter);
             S.KPP = tc_kpp(sg.inter);
+            S.n_xg = U;
             S.n_gu_s = sg.tiles * S.nchs;
             S.n_gu_r = sgu[1];
             S.n_dn_s = TC_MT * S.P * S.nchs;
             S.n_dn_r = sdn[1];
-            S.total = S.n_gu_s + S.n_gu_r + S.n_dn_s + S.n_dn_r;
+            S.total = S.n_xg + S.n_gu_s + S.n_gu_r + S.n_dn_s + S.n_dn_r;
         }
         __syncwarp();
 
         // ------------------------------------------------------------ loader loop
-        const uint64_t pol = policy_evict_first();
-        int raw_i = 0;
         for (int k = 0;; ++k) {
             int u = 0;
             if (lane == 0) u = *abort_flag ? S.total : atomicAdd(&ctrl[TC_WORK], 1);
@@ -375,7 +381,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             int kind = UK_END;
             if (u < S.total) {
                 int v = u;
-                if (v < S.n_gu_s) {
+                if (v < S.n_xg) {
+                    // gather unit of active expert v: its token rows of x into dispatch order
+                    kind = UK_XG;
+                    if (lane == 0) {
+                        Un.expert = S.e[v];
+                        Un.tile = Un.part = 0;
+                        Un.kb0 = Un.nkb = 0;
+                        Un.c0 = 0;
+                        Un.ntok = S.n[v];
+                        Un.arow = S.poff[v];
+                        Un.seg = S.off[v];
+                        Un.wdep = -1;
+                        Un.wtarget = 0;
+                        Un.ddep = TC_DEP_X + S.e[v];
+                    }
+                } else if ((v -= S.n_xg) < S.n_gu_s) {
                     kind = UK_GU_S;
                     const int tile = v / S.nchs, ch = v % S.nchs;
                     if (lane == 0) {
@@ -387,8 +408,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                         Un.c0 = ch * S.cs_s;
                         Un.ntok = min(S.cs_s, T - Un.c0);
                         Un.arow = Un.c0;
-                        Un.dep = TC_DEP_S + Un.part;
-                        Un.target = 0;
+                        Un.wdep = -1;
+                        Un.wtarget = 0;
+                        Un.ddep = TC_DEP_S + Un.part;
                     }
                 } else if ((v -= S.n_gu_s) < S.n_gu_r) {
                     kind = UK_GU_R;
@@ -405,8 +427,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                         Un.c0 = ch * S.cs_s;
                         Un.ntok = min(S.cs_s, T - Un.c0);
                         Un.arow = Un.c0;
-                        Un.dep = TC_DEP_S + part;
-                        Un.target = Un.nkb * S.nchs * NEPI;
+                        Un.wdep = TC_DEP_S + part;
+                        Un.wtarget = Un.nkb * S.nchs * NEPI;
+                        Un.ddep = TC_DN_DONE;
                     }
                 } else {
                     v -= S.n_dn_s;
@@ -435,8 +458,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                         Un.c0 = c0;
                         Un.ntok = ntok;
                         Un.arow = S.poff[a] + c0;
-                        Un.dep = TC_DEP_R + S.e[a];
-                        Un.target = kind == UK_DN_R ? rg.tiles * nch * NEPI : 0;
+                        Un.seg = seg;
+                        // gate/up waits for the expert's gathered rows, down for all its gate/up units
+                        Un.wdep = kind == UK_DN_R ? TC_DEP_R + S.e[a] : TC_DEP_X + S.e[a];
+                        Un.wtarget = kind == UK_DN_R ? rg.tiles * nch * NEPI : NEPI;
+                        Un.ddep = kind == UK_DN_R ? TC_DN_DONE : TC_DEP_R + S.e[a];
                     }
                     for (int n = lane; n < ntok; n += 32) {
                         const int ent = p.R.perm[seg + n];
@@ -450,32 +476,117 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&u_full[slot]);
             if (kind == UK_END) break;
-            if (lane == 0) {
+            if (lane == 0 && kind != UK_XG) {
+                // the copier will stream this unit's blocks a few units from now: bring them into L2
                 const bool routed = kind == UK_GU_R || kind == UK_DN_R;
                 const int wt = routed ? RW : SW;
-                const int nkb = Un.nkb, kb0 = Un.kb0;
+                const uint32_t blk = is_quant(wt) ? (routed ? p.V.r.g.blk : p.V.s.g.blk) : A_BYTES;
+                const uint8_t* b0 = a_block(p.V, Un, Un.kb0);
+                const uint32_t bytes = (uint32_t)Un.nkb * blk;   // the unit's blocks are contiguous
+                for (uint32_t o = 0; o < bytes; o += 64u * 1024u)
+                    bulk_prefetch_l2(b0 + o, min(64u * 1024u, bytes - o));
+            }
+            if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
+        }
+    } else if (warp == WARP_COPY) {
+        // ------------------------------------------------------------ raw-ring copier (one thread)
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            int raw_i = 0;
+            for (int k = 0;; ++k) {
+                const int slot = k % UR;
+                if (!mbar_wait_bounded(&u_full[slot], (k / UR) & 1, WAIT_LIMIT_NS)) {
+                    fail(DEVERR_TC_WAIT);
+                    break;
+                }
+                const Unit& Un = units[slot];
+                const int kind = Un.kind;
+                if (kind == UK_END) {
+                    mbar_arrive(&u_empty[slot]);
+                    break;
+                }
+                const bool routed = kind == UK_GU_R || kind == UK_DN_R;
+                const int wt = routed ? RW : SW;
+                bool ok = true;
                 if (is_quant(wt)) {
                     const uint32_t blk = routed ? p.V.r.g.blk : p.V.s.g.blk;
+                    const int nkb = Un.nkb, kb0 = Un.kb0;
                     for (int kb = 0; kb < nkb; ++kb, ++raw_i) {
                         const int r = raw_i % NR;
                         if (!mbar_wait_bounded(&raw_empty[r], ((raw_i / NR) & 1) ^ 1, WAIT_LIMIT_NS)) {
-                            fail(DEVERR_TC_WAIT);
+                            ok = false;
                             break;
                         }
                         mbar_arrive_expect_tx(&raw_full[r], blk);
                         bulk_g2s(smem + SL::raw + r * SL::raw_slot, a_block(p.V, Un, kb0 + kb), blk, &raw_full[r],
                                  pol);
                     }
-                } else {
-                    for (int kb = 0; kb < nkb; ++kb) bulk_prefetch_l2(a_block(p.V, Un, kb0 + kb), A_BYTES);
                 }
+                mbar_arrive(&u_empty[slot]);
+                if (!ok) {
+                    fail(DEVERR_TC_WAIT);
+                    break;
+                }
+                if (*abort_flag) break;
             }
-            if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
-        }
-        // never leave copies in flight: the last NR issued blocks must have landed
-        if (lane == 0)
+            // never leave copies in flight: the last NR issued blocks must have landed
             for (int i = max(0, raw_i - NR); i < raw_i; ++i)
                 (void)mbar_wait_bounded(&raw_full[i % NR], (i / NR) & 1, WAIT_LIMIT_NS);
+        }
+        __syncwarp();
+    } else if (warp == WARP_BLD) {
+        // ------------------------------------------------------------ operand-stage loader (one thread)
+        // Every stage in order: the B operand (N rows of an operand image: x in token order for the
+        // shared set, x in dispatch order for routed experts, a for down projections) and, for
+        // bf16 weights, the A block, by bulk copies completing on the stage barrier.
+        if (lane == 0) {
+            int ab_i = 0;
+            for (int k = 0;; ++k) {
+                const int slot = k % UR;
+                if (!mbar_wait_bounded(&u_full[slot], (k / UR) & 1, WAIT_LIMIT_NS)) {
+                    fail(DEVERR_TC_WAIT);
+                    break;
+                }
+                const Unit& Un = units[slot];
+                const int kind = Un.kind;
+                if (kind == UK_END) {
+                    mbar_arrive(&u_empty[slot]);
+                    break;
+                }
+                const bool routed = kind == UK_GU_R || kind == UK_DN_R;
+                const bool is_gu = kind <= UK_GU_R;
+                const bool quant = is_quant(routed ? RW : SW);
+                const int N = Un.N, kb0 = Un.kb0, nkb = Un.nkb;
+                const uint16_t* img = is_gu ? (routed ? p.W.x_img_r : p.W.x_img) : (routed ? p.W.a_img : p.W.a_sh);
+                const int rows = routed ? p.W.arows : p.W.tpad;
+                const uint32_t bbytes = (uint32_t)N * 128u;
+                bool ok = true;
+                if (nkb > 0 && Un.wdep >= 0) {
+                    // the rows come from other units' epilogues: wait until they are all written
+                    ok = wait_counter(&ctrl[Un.wdep], Un.wtarget);
+                    fence_proxy_async_all();
+                }
+                for (int kb = 0; kb < nkb && ok; ++kb, ++ab_i) {
+                    const int s = ab_i % NAB;
+                    char* Ast = smem + SL::ab + s * STAGE_BYTES;
+                    if (!mbar_wait_bounded(&ab_empty[s], ((ab_i / NAB) & 1) ^ 1, WAIT_LIMIT_NS)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&ab_full[s], bbytes + (quant ? 0u : A_BYTES));
+                    if (!quant) bulk_g2s(Ast, a_block(p.V, Un, kb0 + kb), A_BYTES, &ab_full[s], policy_evict_first());
+                    bulk_g2s(Ast + A_BYTES, img + ((size_t)(kb0 + kb) * rows + Un.arow) * TC_KB, bbytes, &ab_full[s],
+                             policy_evict_last());
+                }
+                if (!ok) {
+                    fail(DEVERR_TC_WAIT);
+                    break;
+                }
+                mbar_arrive(&u_empty[slot]);
+                if (*abort_flag) break;
+            }
+        }
+        __syncwarp();
     } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------ MMA issuer (one thread)
         if (lane == 0) {
@@ -490,6 +601,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                 if (Un.kind == UK_END) {
                     mbar_arrive(&u_empty[slot]);
                     break;
+                }
+                if (Un.kind == UK_XG) {   // no MMA work
+                    mbar_arrive(&u_empty[slot]);
+                    continue;
                 }
                 const int b = acc_i % NACC;
                 if (!mbar_wait_bounded(&acc_empty[b], ((acc_i / NACC) & 1) ^ 1, WAIT_LIMIT_NS)) {
@@ -530,8 +645,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
         }
         __syncwarp();
     } else if (warp < WARP_EPI) {
-        // ------------------------------------------------------------ stagers
+        // ------------------------------------------------------------ dequantising stagers
+        // Warp pair pp = (sw / 2) takes every NPAIR-th operand stage in turn; warp hw = sw % 2 of
+        // the pair dequantises block rows 64 hw .. 64 hw + 63 of a quantised A block (for a bf16
+        // block the pair only takes its turn: the loader warp copies it).  The pair's stores are
+        // ordered before the tensor core's reads by a proxy fence, then each warp arrives.
         const int sw = warp - WARP_STG;
+        const int pp = sw >> 1, hw = sw & 1;
         int ab_i = 0, raw_i = 0;
         for (int k = 0;; ++k) {
             const int slot = k % UR;
@@ -548,82 +668,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                 break;
             }
             const bool routed = kind == UK_GU_R || kind == UK_DN_R;
-            const bool is_gu = kind <= UK_GU_R;
-            const int wt = routed ? RW : SW;
-            const int ntok = Un.ntok, N = Un.N, kb0 = Un.kb0, nkb = Un.nkb;
-            // gather rows of this lane: row-groups sw and sw + 8, k-cores pr and pr + 4
-            int trow[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int n = 8 * (sw + 8 * (i >> 1)) + (lane & 7);
-                trow[i] = -1;
-                if (is_gu && n < ntok) trow[i] = routed ? Un.ent[n] / K : Un.c0 + n;
-            }
-            const uint16_t* aimg = routed ? p.W.a_img : p.W.a_sh;
-            const int arows = routed ? p.W.arows : p.W.tpad;
+            const bool quant = is_quant(routed ? RW : SW);
+            const int nkb = Un.nkb;
             for (int kb = 0; kb < nkb && ok; ++kb, ++ab_i) {
+                const int r = raw_i;
+                if (quant) ++raw_i;
+                if (ab_i % NPAIR != pp) continue;
                 const int s = ab_i % NAB;
                 char* Ast = smem + SL::ab + s * STAGE_BYTES;
-                char* Bst = Ast + A_BYTES;
                 if (lane == 0) ok = mbar_wait_bounded(&ab_empty[s], ((ab_i / NAB) & 1) ^ 1, WAIT_LIMIT_NS);
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
-                if (sw == 0 && lane == 0) {
-                    const uint32_t bytes = (is_quant(wt) ? 0u : A_BYTES) + (is_gu ? 0u : (uint32_t)N * 128u);
-                    if (!is_gu && kb == 0) {
-                        if (!wait_counter(&ctrl[Un.dep], Un.target)) ok = false;
-                        fence_proxy_async_all();
-                    }
-                    if (ok && bytes) {
-                        mbar_expect_tx(&ab_full[s], bytes);
-                        if (!is_quant(wt))
-                            bulk_g2s(Ast, a_block(p.V, Un, kb0 + kb), A_BYTES, &ab_full[s], policy_evict_first());
-                        if (!is_gu)
-                            bulk_g2s(Bst, aimg + ((size_t)(kb0 + kb) * arows + Un.arow) * TC_KB, (uint32_t)N * 128u,
-                                     &ab_full[s], policy_evict_last());
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                if (!ok) break;
-                uint4 bv[4];
-                if (is_gu) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int kc = (lane >> 3) + 4 * (i & 1);
-                        bv[i] = make_uint4(0u, 0u, 0u, 0u);
-                        if (trow[i] >= 0)
-                            bv[i] = __ldg(reinterpret_cast<const uint4*>(p.W.xrows + (size_t)trow[i] * H +
-                                                                         (kb0 + kb) * TC_KB + kc * 8));
-                    }
-                }
-                if (is_quant(wt)) {
-                    const int r = raw_i % NR;
-                    bool rok = true;
-                    if (lane == 0) rok = mbar_wait_bounded(&raw_full[r], (raw_i / NR) & 1, WAIT_LIMIT_NS);
-                    rok = __shfl_sync(0xffffffffu, rok ? 1 : 0, 0) != 0;
-                    if (!rok) {
-                        ok = false;
-                        break;
-                    }
-                    const uint8_t* raw = reinterpret_cast<const uint8_t*>(smem + SL::raw + r * SL::raw_slot);
+                if (quant) {
+                    const int rs = r % NR;
+                    if (lane == 0) ok = mbar_wait_bounded(&raw_full[rs], (r / NR) & 1, WAIT_LIMIT_NS);
+                    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                    if (!ok) break;
+                    const uint8_t* raw = reinterpret_cast<const uint8_t*>(smem + SL::raw + rs * SL::raw_slot);
                     if (routed) {
-                        if constexpr (is_quant(RW)) dequant_block<RW, G>(raw, Ast, sw, lane);
+                        if constexpr (is_quant(RW)) dequant_half<RW, G>(raw, Ast, hw, lane);
                     } else {
-                        if constexpr (is_quant(SW)) dequant_block<SW, G>(raw, Ast, sw, lane);
+                        if constexpr (is_quant(SW)) dequant_half<SW, G>(raw, Ast, hw, lane);
                     }
+                    umma::fence_smem_to_async();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&raw_empty[r]);
-                    ++raw_i;
+                    if (lane == 0) mbar_arrive(&raw_empty[rs]);
                 }
-                if (is_gu) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int j = sw + 8 * (i >> 1), kc = (lane >> 3) + 4 * (i & 1);
-                        if (8 * j < N) sts128(Bst + j * 1024 + kc * 128 + (lane & 7) * 16, bv[i]);
-                    }
-                }
-                umma::fence_smem_to_async();
-                __syncwarp();
                 if (lane == 0) mbar_arrive(&ab_full[s]);
             }
             if (!ok) {
@@ -650,6 +720,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             if (kind == UK_END) {
                 if (lane == 0) mbar_arrive(&u_empty[slot]);
                 break;
+            }
+            if (kind == UK_XG) {
+                // the expert's token rows of x, in dispatch order, into its padded segment of the
+                // dispatch-order image: 16-byte pieces, consecutive threads writing consecutive pieces
+                const int et = (warp - WARP_EPI) * 32 + lane, n = Un.ntok, r8 = (n + 7) & ~7;
+                const int per_kb = r8 * 8;   // pieces of one K-block
+                const uint4* src = reinterpret_cast<const uint4*>(p.W.x_img);
+                uint4* dst = reinterpret_cast<uint4*>(p.W.x_img_r);
+                for (int c = et; c < TC_KBH * per_kb; c += NEPI * 32) {
+                    const int kb = c / per_kb, rem = c % per_kb;
+                    const int row = (rem >> 6) * 8 + (rem & 7), kc = (rem >> 3) & 7;
+                    if (row < n) {
+                        const int t = p.R.perm[Un.seg + row] / K;
+                        dst[img_index(p.W.arows, Un.arow + row, kb * TC_KB + kc * 8) / 8] =
+                            __ldg(src + img_index(p.W.tpad, t, kb * TC_KB + kc * 8) / 8);
+                    }
+                }
+                fence_proxy_async_all();
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) {
+                    atomicAdd(&ctrl[Un.ddep], 1);
+                    mbar_arrive(&u_empty[slot]);
+                }
+                continue;
             }
             const int b = acc_i % NACC;
             if (lane == 0) ok = mbar_wait_bounded(&acc_full[b], (acc_i / NACC) & 1, WAIT_LIMIT_NS);
@@ -678,7 +773,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                         const int n = c + (gate ? j : 8 + j);
                         if (n < ntok) {
                             const float w = routed ? Un.w[n] : 1.0f;
-                            const float a = g / (1.0f + __expf(-g)) * u * w;
+                            const float a = __fdividef(g, 1.0f + __expf(-g)) * u * w;
                             const int row = Un.arow + n;
                             col[(size_t)(row >> 3) * 512 + (row & 7) * 8] =
                                 __bfloat16_as_ushort(__float2bfloat16_rn(a));
@@ -710,7 +805,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             fence_proxy_async_all();
             __threadfence();
             __syncwarp();
-            if (lane == 0) atomicAdd(&ctrl[kind <= UK_GU_R ? Un.dep : TC_DN_DONE], 1);
+            if (lane == 0) atomicAdd(&ctrl[Un.ddep], 1);
             if (lane == 0) mbar_arrive(&u_empty[slot]);
             if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
         }
@@ -769,13 +864,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
     }
 }
 
-// fp32 -> bf16 rows of x (the dense layer has no router to write them)
-__global__ void xrows_kernel(const float* x, int n4, uint16_t* xrows) {
+// x (fp32) -> the bf16 operand image in token order (the dense layer has no router to write it)
+__global__ void x_image_kernel(const float* x, int T, int rows, uint16_t* img) {
     pdl_wait();
     pdl_launch_dependents();
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(x) + i);
-        reinterpret_cast<uint2*>(xrows)[i] = make_uint2(f32x2_to_bf16x2(v.x, v.y), f32x2_to_bf16x2(v.z, v.w));
+    const int n = T * (H / 8);   // 16-byte pieces: 8 columns of one token
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const int t = i / (H / 8), k = (i % (H / 8)) * 8;
+        const float4 a = __ldg(reinterpret_cast<const float4*>(x + (size_t)t * H + k));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(x + (size_t)t * H + k + 4));
+        reinterpret_cast<uint4*>(img)[img_index(rows, t, k) / 8] =
+            make_uint4(f32x2_to_bf16x2(a.x, a.y), f32x2_to_bf16x2(a.z, a.w), f32x2_to_bf16x2(b.x, b.y),
+                       f32x2_to_bf16x2(b.z, b.w));
     }
 }
 
@@ -824,7 +924,7 @@ cudaError_t launch_expert_tc(const float* x, int T, const TcView& V, const Route
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, xrows_kernel, x, T * (H / 4), W.xrows);
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, x_image_kernel, x, T, W.tpad, W.x_img);
         if (e != cudaSuccess) return e;
     }
     const TcParams p{x, T, out, resid ? 1 : 0, shared_only ? 1 : 0, V, R, W};

@@ -48,7 +48,8 @@ struct RouterParams {
     RouteView R;
     float* out;           // NULL: the output is not initialised here
     const float* resid;   // NULL: out starts at zero; else out starts as a copy of resid
-    uint16_t* xrows;      // NULL, or bf16 rows of x [T][1280] for the tensor-core path
+    uint16_t* x_img;      // NULL, or x in bf16 as an operand image (tensor-core path)
+    int img_rows;         // its rows (T rounded up to 16)
 };
 
 // counts / offsets / active list / stable permutation of n = T*6 <= 64 entries, by one warp.
@@ -220,7 +221,7 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
         xs[t][c] = t < nt ? (double)p.x[(size_t)(t0 + t) * H + k0 + c] : 0.0;
     }
     __syncthreads();
-    if (p.xrows) {
+    if (p.x_img) {
         // this CTA's 160 columns of its tokens, rounded to bf16 (the tensor-core path's B operand)
         for (int i = tid; i < TB * (KCOLS / 8); i += RT_THREADS) {
             const int t = i / (KCOLS / 8), kc = i % (KCOLS / 8);
@@ -231,7 +232,7 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
                 o.y = pack_bf16x2((float)v[2], (float)v[3]);
                 o.z = pack_bf16x2((float)v[4], (float)v[5]);
                 o.w = pack_bf16x2((float)v[6], (float)v[7]);
-                *reinterpret_cast<uint4*>(p.xrows + (size_t)(t0 + t) * H + k0 + kc * 8) = o;
+                *reinterpret_cast<uint4*>(p.x_img + img_index(p.img_rows, t0 + t, k0 + kc * 8)) = o;
             }
         }
     }
@@ -393,8 +394,8 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
 }  // namespace
 
 cudaError_t launch_router(const float* x, int T, int /*T_ws*/, const LayerView& L, const RouteView& R, float* out,
-                          const float* resid, uint16_t* xrows, cudaStream_t st) {
-    RouterParams p{x, T, L.router, R, out, resid, xrows};
+                          const float* resid, uint16_t* x_img, int img_rows, cudaStream_t st) {
+    RouterParams p{x, T, L.router, R, out, resid, x_img, img_rows};
     const int TB = T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : 8));
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(((T + TB - 1) / TB) * RC);
