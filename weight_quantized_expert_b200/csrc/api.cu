@@ -136,8 +136,8 @@ focr_status focr_moe_pack_weights(const focr_moe_weights_desc* d, focr_moe_layer
     L->group = d->group_size;
     L->rg = make_geom(d->routed_type, d->group_size, I);
     L->sg = make_geom(d->shared_type, d->group_size, IS);
-    L->rtg = make_tc_geom(d->routed_type, d->group_size, I);
-    L->stg = make_tc_geom(d->shared_type, d->group_size, IS);
+    L->rtg = make_tc_geom(d->routed_type, d->group_size, I, tc_tile_group(d->routed_type));
+    L->stg = make_tc_geom(d->shared_type, d->group_size, IS, 1);
     plan(L);
 
     std::vector<uint8_t> host;
@@ -156,10 +156,11 @@ focr_status focr_moe_pack_weights(const focr_moe_weights_desc* d, focr_moe_layer
         if (e < E) {
             host_pack_set(d->w_gate + (size_t)e * I * H, d->w_up + (size_t)e * I * H, d->w_down + (size_t)e * H * I,
                           rg, ritems + (size_t)e * rg.slices * rg.item_bytes, rdsc + (size_t)e * rg.dscale_expert_floats,
-                          hb + L->off_tc_rgu + (size_t)e * L->rtg.gu_bytes, hb + L->off_tc_rdn + (size_t)e * L->rtg.dn_bytes);
+                          hb + L->off_tc_rgu + (size_t)e * L->rtg.gu_bytes, hb + L->off_tc_rdn + (size_t)e * L->rtg.dn_bytes,
+                          L->rtg.grp);
         } else {
             host_pack_set(d->ws_gate, d->ws_up, d->ws_down, L->sg, hb + L->off_sitems,
-                          reinterpret_cast<float*>(hb + L->off_sdsc), hb + L->off_tc_sgu, hb + L->off_tc_sdn);
+                          reinterpret_cast<float*>(hb + L->off_sdsc), hb + L->off_tc_sgu, hb + L->off_tc_sdn, L->stg.grp);
         }
     });
 
@@ -460,7 +461,7 @@ focr_status focr_dense_mlp_pack(const float* w_gate, const float* w_up, const fl
     M->wtype = wtype;
     M->group = is_quant(wtype) ? group : 0;
     M->g = make_geom(wtype, group, FOCR_DENSE_INTER);
-    M->tg = make_tc_geom(wtype, group, FOCR_DENSE_INTER);
+    M->tg = make_tc_geom(wtype, group, FOCR_DENSE_INTER, 1);
     M->off_items = 0;
     M->off_dsc = align_up((size_t)M->g.slices * M->g.item_bytes, 256);
     M->off_tc_gu = align_up(M->off_dsc + sizeof(float) * (size_t)M->g.dscale_expert_floats, 256);
@@ -474,7 +475,7 @@ focr_status focr_dense_mlp_pack(const float* w_gate, const float* w_up, const fl
         return fail(FOCR_ERR_OOM, "host staging of %zu bytes failed", M->bytes);
     }
     host_pack_set(w_gate, w_up, w_down, M->g, host.data(), reinterpret_cast<float*>(host.data() + M->off_dsc),
-                  host.data() + M->off_tc_gu, host.data() + M->off_tc_dn);
+                  host.data() + M->off_tc_gu, host.data() + M->off_tc_dn, M->tg.grp);
     cudaError_t e = cudaMalloc(&M->dev, M->bytes);
     if (e != cudaSuccess) {
         delete M;

@@ -100,13 +100,14 @@ struct LayerView {
 // ---------------------------------------------------------------------------------------
 // Second device layout of a weight set, read by the tensor-core (tcgen05) grouped kernel
 // for batches of more than 8 tokens.  Every matrix is cut into blocks of 128 rows x 64
-// input columns (one "K-block"); a block is what one pipeline stage of the kernel stages
-// in shared memory, and the blocks of one work unit are consecutive in memory:
-//   gate/up : [tile p of 64 intermediates][20 K-blocks][block]; block row r = 16 j + 8 h + r'
-//             is gate (h = 0) or up (h = 1) row 64 p + 8 j + r' (so a gate row and its up row
-//             sit 8 TMEM lanes apart, inside one warp's quarter of the accumulator)
-//   down    : [m-tile of 128 output rows][inter / 64 K-blocks][block]; block row r is output
-//             row 128 m + r
+// input columns (one "K-block").  Tiles come in groups of `grp` (routed experts: the most tiles a
+// work unit covers, tc_tile_group; the shared set: 1); within a group the blocks of one K-block
+// are adjacent, so a unit covering several tiles streams each of its K-blocks with one copy, and
+// with grp = 1 the K-blocks of a tile are adjacent instead (tc_block_index):
+//   gate/up : tiles p of 64 intermediates x 20 K-blocks; block row r = 16 j + 8 h + r' is gate
+//             (h = 0) or up (h = 1) row 64 p + 8 j + r' (so a gate row and its up row sit 8 TMEM
+//             lanes apart, inside one warp's quarter of the accumulator)
+//   down    : m-tiles of 128 output rows x inter / 64 K-blocks; block row r is output row 128 m + r
 // Quantised blocks: codes [128 rows][RB bytes] then f32 scales [128 rows][SPK].  A row's
 // codes come in four pairs (k-core c, k-core c + 4) of 8-element k-cores (one k-core per
 // 16-byte row of the tensor core's shared-memory operand):
@@ -130,16 +131,32 @@ __host__ __device__ constexpr uint32_t tc_block_bytes(int wtype, int G) {
                            : (uint32_t)TC_M * TC_KB * 2u;
 }
 
+// Tiles of one routed work unit at most (and the routed tile group) by weight type, so that one
+// K-block of a unit's tiles is 16-18 KB: int4 4, int8 2, bf16 1.
+__host__ __device__ constexpr int tc_tile_group(int wtype) {
+    return wtype == FOCR_W_INT4 ? 4 : (wtype == FOCR_W_INT8 ? 2 : 1);
+}
+
+// Block index of (tile, K-block) in a matrix of `tiles` tiles x `nkb` K-blocks with tile groups
+// of `grp`: the group starting at tile t0 = grp * (tile / grp) holds gs = min(grp, tiles - t0)
+// tiles, stored as [K-block][tile in group] after the t0 * nkb blocks of the groups before it.
+__host__ __device__ constexpr size_t tc_block_index(int tiles, int nkb, int tile, int kb, int grp) {
+    return (size_t)(tile - tile % grp) * nkb +
+           (size_t)kb * (tiles - (tile - tile % grp) < grp ? tiles - (tile - tile % grp) : grp) + tile % grp;
+}
+
 struct TcGeom {
     int wtype, group, inter;
     int tiles;            // inter / 64 gate/up tiles (= K-blocks of the down projection)
+    int grp;              // tile group of the layout (tc_block_index)
     uint32_t blk;         // bytes of one block
     size_t gu_bytes;      // tiles * 20 blocks
     size_t dn_bytes;      // 10 m-tiles * tiles blocks
 };
 
-__host__ __device__ inline TcGeom make_tc_geom(int wtype, int group, int inter) {
+__host__ __device__ inline TcGeom make_tc_geom(int wtype, int group, int inter, int grp) {
     TcGeom g{};
+    g.grp = grp;
     g.wtype = wtype;
     g.group = is_quant(wtype) ? group : 0;
     g.inter = inter;
@@ -391,13 +408,19 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
 }
 
 // Wait for the phase with the given parity to complete; give up after ~limit_ns.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait_bounded, kept out of line so that the common case (the phase has
+// already completed) costs one try_wait and a branch in the caller's loop.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
         if (globaltimer_ns() - t0 > limit_ns) return false;
     }
+}
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    if (__builtin_expect(mbar_try_wait(bar, parity), 1)) return true;
+    return mbar_wait_slow(bar, parity, limit_ns);
 }
 
 // Bulk (non-tensor) async copy global -> own shared memory, completing on an mbarrier.

@@ -1,8 +1,8 @@
 // Tensor-core grouped expert kernel for batches of more than 8 tokens (batched decode,
 // prefill): the shared expert and every selected routed expert as tcgen05 GEMMs with the
-// accumulators in tensor memory, SwiGLU fused into the gate/up epilogue, and a combine that
-// sums each token's parts in a fixed order (no atomics on the output, so repeated calls are
-// bit-identical).
+// dequantised weights and the accumulators in tensor memory, SwiGLU fused into the gate/up
+// epilogue, and a combine that sums each token's parts in a fixed order (no atomics on the
+// output, so repeated calls are bit-identical).
 //
 // Sources: frankenocr.pages.dev, "One forward pass", step 6 (64 routed experts + 2 fused
 // shared experts, softmax top-6 without renormalisation, weighted sum of the experts); franken_ocr
@@ -10,32 +10,38 @@
 // "Four bits, one shared scale" (int4 nibble + f32 group scale; int8 and bf16 formats).
 //
 // The contraction is swapped so that the weights fill the MMA's M = 128 rows and a chunk of at
-// most 128 of an expert's tokens fills N (a multiple of 16):
-//   gate/up unit  (set, tile of 64 intermediates, token chunk): D[128 x N] = [G; U]_tile X^T over
-//                 K = 1280 (block rows interleave gate and up by 8, see the tensor-core layout
-//                 in common.cuh); the epilogue pairs each gate lane with its up lane (shuffle
-//                 by 8) and writes a = silu(g) * u * w_route as bf16 into the "a image"
-//   down unit     (set, m-tile of 128 output rows, [K part,] token chunk): D = Down_mtile a^T
-//                 over the set's intermediates (the shared set's in up to 8 K parts); the
-//                 epilogue writes fp32 rows y per (token, slot) or per (token, part)
+// most 128 of an expert's tokens fills N (a multiple of 16).  A work unit covers MT <= 4 weight
+// tiles of one set that share the unit's token chunk (MT = 128 / N rounded down to 1, 2 or 4),
+// so each K-block of token rows is loaded once for MT tiles:
+//   gate/up unit  (set, MT tiles of 64 intermediates, token chunk): D_t[128 x N] = [G; U]_t X^T over
+//                 K = 1280 (block rows interleave gate and up by 8, see the tensor-core layout in
+//                 common.cuh); the epilogue pairs each gate lane with its up lane (shuffle by 8)
+//                 and writes a = silu(g) * u * w_route as bf16 into the "a image"
+//   down unit     (set, MT m-tiles of 128 output rows, [K part,] token chunk): D_t = Down_t a^T over
+//                 the set's intermediates (the shared set's in up to 8 K parts); the epilogue
+//                 writes fp32 rows y per (token, slot) or per (token, part)
+//   gather unit   (routed expert): its token rows of x, in dispatch order, into an operand image
 //   combine       out[t] = resid + sum_parts y_shared + sum_{j<6} y_slot[t*6+j]
-// Units are handed out by a global atomic counter (largest classes first: shared gate/up,
-// routed gate/up, shared down, routed down), so a unit only ever waits on units with smaller
-// numbers, which running CTAs hold: a down unit's B load waits (bounded) for its expert's
-// gate/up units to have written their a rows.
+// Units are handed out by a global atomic counter (gathers, shared gate/up, routed gate/up, shared
+// down, routed down), so a unit only ever waits on units with smaller numbers, which running CTAs
+// hold: a unit's token-row loads wait (bounded) until the units that write those rows are done.
 //
-// Warp roles (one CTA per SM, 448 threads):
-//   warp 0      loader: takes units, publishes their descriptors, streams quantised weight
-//               blocks (codes + scales, 4.5-8.5 KB per 128 x 64 block) into a ring with bulk
-//               async copies (cp.async.bulk + mbarrier), and prefetches bf16 blocks into L2
-//   warp 1      MMA: one thread issues tcgen05.mma (kind::f16, bf16 operands, fp32 accumulate
-//               in TMEM; 4 k-steps of 16 per block) and commits stages and accumulators
-//   warps 2-9   stagers: dequantise a block (q * s rounded to bf16; int4 by the exponent-bias
-//               method, int8 through fp32) into the K-major core-matrix layout, gather the
-//               chunk's token rows of x (bf16) as the B operand, or bulk-copy bf16 blocks and
-//               a-image rows
-//   warps 10-13 epilogue: tcgen05.ld of a 128-column accumulator (four in TMEM, so the MMA
-//               runs ahead), SwiGLU or output rows, then the unit's completion counter
+// Warp roles (one CTA per SM, 640 threads):
+//   warp 0       scheduler: takes units, publishes their descriptors
+//   warp 1       MMA: one thread issues tcgen05.mma (kind::f16, A from TMEM, B from shared
+//                memory, fp32 accumulate in TMEM; 4 k-steps of 16 per 64-wide K-block), waiting
+//                once per A stage of two blocks: a single issuing thread is bound by the
+//                latency of each wait, not by the tensor pipe, at these small N
+//   warp 2       weight copier: bulk copies (cp.async.bulk + mbarrier) of super-slots of about
+//                16-18 KB (a few K-blocks of the unit's tiles) into a ~110 KB ring, so enough
+//                HBM reads are in flight to stream at full bandwidth
+//   warp 3       token-row loader: one bulk copy per K-block of N rows of an operand image
+//   warps 4-15   dequantisers, three groups of four (one warp per TMEM lane quarter): thread = one
+//                of the block's 128 rows; int4 (exponent-bias method) or int8 codes times the group
+//                scale, rounded to bf16 (q * s), written to a TMEM A stage with tcgen05.st;
+//                bf16 blocks are moved to TMEM as they are
+//   warps 16-19  epilogue: tcgen05.ld of the accumulators, SwiGLU or output rows, completion
+//                counts; gather units
 // Every wait is bounded in time (%globaltimer); on expiry the kernel records an error word,
 // stops taking work, waits (bounded) for its own copies in flight, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -47,37 +53,51 @@
 namespace focr {
 namespace {
 
-constexpr int NSTG = 8;                          // stager warps
+constexpr int NDQG = 3;                          // dequantiser groups
 constexpr int NEPI = 4;                          // epilogue warps
-constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_STG = 2, WARP_EPI = WARP_STG + NSTG;
-constexpr int WARP_COPY = WARP_EPI + NEPI;       // streams quantised blocks into the raw ring
-constexpr int WARP_BLD = WARP_COPY + 1;          // fills operand stages by copy: bf16 A, token rows, a rows
-constexpr int NWARPS = WARP_BLD + 1;
+constexpr int WARP_SCHED = 0, WARP_MMA = 1, WARP_COPY = 2, WARP_BLD = 3, WARP_DQ = 4;
+constexpr int WARP_EPI = WARP_DQ + 4 * NDQG;
+constexpr int NWARPS = WARP_EPI + NEPI;
 constexpr int NTHREADS = NWARPS * 32;
 constexpr int NCH = 128;                         // tokens of one unit at most (the MMA's N)
-constexpr int NAB = 5;                           // operand stages
-constexpr int NPAIR = NSTG / 2;                  // stager warp pairs, one operand stage each in turn
-constexpr uint32_t A_BYTES = TC_M * TC_KB * 2;   // 16 KB bf16 A block
-constexpr uint32_t B_BYTES = NCH * TC_KB * 2;    // 16 KB bf16 B block
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr uint32_t RAW_BUDGET = 46 * 1024;       // quantised blocks in flight (plus L2 prefetch)
-constexpr int UR = 6;                            // unit descriptors in flight
-constexpr int NACC = 4;                          // TMEM accumulators of 128 columns
+constexpr int NA = 4;                            // TMEM A stages (64 columns: two blocks of 128 rows x 64 bf16)
+constexpr int NACC = 2;                          // TMEM accumulators (128 columns)
 constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_A0 = NACC * 128;           // first column of the A stages
+constexpr int NB = 6;                            // token-row stages in shared memory
+constexpr uint32_t B_SLOT = NCH * TC_KB * 2;     // 16 KB
+constexpr uint32_t RAW_BUDGET = 110 * 1024;      // weight super-slots in flight
+constexpr int UR = 4;                            // unit descriptors in flight
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s
 constexpr int DEVERR_TC_WAIT = 3;
 
+static_assert(WARP_DQ % 4 == 0 && WARP_EPI % 4 == 0, "a group of four warps covers the four TMEM lane quarters");
+static_assert(TM_A0 + NA * 64 <= TMEM_COLS, "TMEM budget");
+
 enum UnitKind { UK_GU_S = 0, UK_GU_R = 1, UK_DN_S = 2, UK_DN_R = 3, UK_XG = 4, UK_END = 5 };
 
+// A stages: a unit's weight blocks (K-block kb, tile t) pass through TMEM two at a time, tiles
+// (2 i, 2 i + 1) of one K-block per stage (a single tile where mt is odd), so that the MMA issuer
+// waits once per pair of blocks.
+__device__ __forceinline__ int stages_per_kb(int mt) { return (mt + 1) >> 1; }
+
+// tiles a unit may cover for a chunk of N token rows: the MT accumulators fit 128 TMEM columns
+__device__ __forceinline__ int mt_for(int N, int cap) {
+    const int m = N <= 32 ? 4 : (N <= 64 ? 2 : 1);
+    return m < cap ? m : cap;
+}
+
 struct Unit {
-    int kind, expert, tile, part;
+    int kind, expert;
+    int tile, mt;        // first weight tile and tiles covered (gate/up: 64 intermediates; down: 128 rows)
+    int part;            // shared down: K part
     int kb0, nkb;        // K-blocks [kb0, kb0 + nkb) of the set's matrix
     int ntok, N;         // tokens of the chunk, N = ntok rounded up to 16
     int c0;              // first token of the chunk: shared, a token id; routed, an index in the expert's segment
-    int arow;            // first row of the chunk in the a image
+    int arow;            // first row of the chunk in the operand images
+    int seg;             // routed: first dispatch entry of the chunk (index into the permutation)
     int wdep, wtarget;   // counter (index into the tensor-core control words) to wait for before the B loads, -1: none
     int ddep;            // counter this unit's completion adds to
-    int seg;             // routed: first dispatch entry of the chunk (index into the permutation)
     int ent[NCH];        // routed: dispatch entries t * 6 + j of the chunk's tokens
     float w[NCH];        // routed gate/up: their routing weights
 };
@@ -104,29 +124,26 @@ __host__ __device__ constexpr uint32_t cmax(uint32_t a, uint32_t b) { return a >
 
 template <int RW, int SW, int G>
 struct TcSmem {
-    static constexpr uint32_t raw_r = is_quant(RW) ? tc_block_bytes(RW, G) : 0u;
-    static constexpr uint32_t raw_s = is_quant(SW) ? tc_block_bytes(SW, G) : 0u;
-    static constexpr uint32_t raw_slot = (cmax(cmax(raw_r, raw_s), 128u) + 127u) & ~127u;
-    static constexpr int NR = (is_quant(RW) || is_quant(SW))
-                                  ? ((int)(RAW_BUDGET / raw_slot) > 32 ? 32 : (int)(RAW_BUDGET / raw_slot))
-                                  : 2;
-    static constexpr uint32_t ab = 0;                                        // [NAB][A | B]
-    static constexpr uint32_t raw = ab + NAB * STAGE_BYTES;                  // [NR][raw_slot]
-    static constexpr uint32_t units = raw + NR * raw_slot;                   // [UR] Unit
+    static constexpr uint32_t raw_r = (uint32_t)tc_tile_group(RW) * tc_block_bytes(RW, G);
+    static constexpr uint32_t raw_s = (uint32_t)tc_tile_group(SW) * tc_block_bytes(SW, G);
+    static constexpr uint32_t raw_slot = (cmax(raw_r, raw_s) + 127u) & ~127u;
+    static constexpr int cap_r = (int)(raw_slot / tc_block_bytes(RW, G));   // blocks one super-slot holds
+    static constexpr int cap_s = (int)(raw_slot / tc_block_bytes(SW, G));
+    static constexpr int cap = cap_r > cap_s ? cap_r : cap_s;
+    static constexpr int NR = (int)(RAW_BUDGET / raw_slot);
+    static constexpr uint32_t braw = 0;                                           // [NR][raw_slot]
+    static constexpr uint32_t bstage = (braw + NR * raw_slot + 1023u) & ~1023u;   // [NB][B_SLOT]
+    static constexpr uint32_t units = bstage + NB * B_SLOT;                       // [UR] Unit
     static constexpr uint32_t sched = (units + UR * (uint32_t)sizeof(Unit) + 15u) & ~15u;
     static constexpr uint32_t bars = (sched + (uint32_t)sizeof(Sched) + 7u) & ~7u;
-    static constexpr int NBARS = 2 * NAB + 2 * NR + 2 * UR + 2 * NACC + 1;
-    static constexpr uint32_t misc = bars + 8u * NBARS;                      // tmem base, abort flag
+    static constexpr int NBARS = 2 * NR + 2 * NB + 2 * NA + 2 * UR + 2 * NACC + 1;
+    static constexpr uint32_t misc = bars + 8u * NBARS;                           // tmem base, abort flag
     static constexpr uint32_t total = misc + 16u;
+    static_assert(NR >= 4, "weight ring depth");
     static_assert(total <= 232448, "shared memory budget");
 };
 
 // ------------------------------------------------------------------ small PTX helpers
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
     int v;
@@ -135,18 +152,6 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
 }
 
 __device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
-
-__device__ __forceinline__ void sts128(void* p, uint4 v) {
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(v.x), "r"(v.y), "r"(v.z),
-                 "r"(v.w)
-                 : "memory");
-}
-
-__device__ __forceinline__ uint2 lds64(const void* p) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_u32(p)));
-    return v;
-}
 
 // Wait (bounded) until the counter reaches `target`.
 __device__ __forceinline__ bool wait_counter(const int* p, int target) {
@@ -176,62 +181,143 @@ constexpr uint32_t BF2_136 = 0x43084308u;     // (136, 136)
 
 // One k-core of int4 codes (element 2m in nibble m, 2m+1 in nibble m+4, q + 8) -> 8 bf16 q * s.
 // q = (128 + n) - 136 is exact in bf16; the product is rounded once (s2 = bf16 pair of the scale).
-__device__ __forceinline__ uint4 dq_int4_bf16(uint32_t w, uint32_t s2) {
-    uint4 r;
-    r.x = bf2_mul(bf2_sub((w & 0x000F000Fu) | BF2_MAGIC, BF2_136), s2);
-    r.y = bf2_mul(bf2_sub(((w >> 4) & 0x000F000Fu) | BF2_MAGIC, BF2_136), s2);
-    r.z = bf2_mul(bf2_sub(((w >> 8) & 0x000F000Fu) | BF2_MAGIC, BF2_136), s2);
-    r.w = bf2_mul(bf2_sub(((w >> 12) & 0x000F000Fu) | BF2_MAGIC, BF2_136), s2);
-    return r;
+__device__ __forceinline__ void dq_int4_bf16(uint32_t w, uint32_t s2, uint32_t* r) {
+    r[0] = bf2_mul(bf2_sub((w & 0x000F000Fu) | BF2_MAGIC, BF2_136), s2);
+    r[1] = bf2_mul(bf2_sub(((w >> 4) & 0x000F000Fu) | BF2_MAGIC, BF2_136), s2);
+    r[2] = bf2_mul(bf2_sub(((w >> 8) & 0x000F000Fu) | BF2_MAGIC, BF2_136), s2);
+    r[3] = bf2_mul(bf2_sub(((w >> 12) & 0x000F000Fu) | BF2_MAGIC, BF2_136), s2);
 }
 
 // One k-core of int8 codes (q + 128 in bytes 0..7) -> 8 bf16 q * s (fp32 product, one rounding).
-__device__ __forceinline__ uint4 dq_int8_bf16(uint32_t w0, uint32_t w1, float s) {
+__device__ __forceinline__ void dq_int8_bf16(uint32_t w0, uint32_t w1, float s, uint32_t* r) {
     float f[8];
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
         f[b] = (byte_to_float(w0, b) - 8388736.0f) * s;
         f[4 + b] = (byte_to_float(w1, b) - 8388736.0f) * s;
     }
-    return make_uint4(f32x2_to_bf16x2(f[0], f[1]), f32x2_to_bf16x2(f[2], f[3]), f32x2_to_bf16x2(f[4], f[5]),
-                      f32x2_to_bf16x2(f[6], f[7]));
+#pragma unroll
+    for (int m = 0; m < 4; ++m) r[m] = f32x2_to_bf16x2(f[2 * m], f[2 * m + 1]);
 }
 
-// Warp hw (0, 1) of a stager pair turns block rows 64 hw .. 64 hw + 63 of a quantised block into
-// the bf16 A operand: lane (pr = lane / 8, rr = lane % 8) writes k-cores pr and pr + 4 of rows
-// 8 g + rr of each of the warp's eight row groups g; every warp store covers 512 contiguous bytes.
+// One row of a weight block into 32 registers (32-bit column c of the TMEM A stage = elements
+// 2c, 2c + 1 of the 64-wide K-block): thread = block row `row`.
 template <int W, int G>
-__device__ __forceinline__ void dequant_half(const uint8_t* raw, char* A, int hw, int lane) {
-    constexpr int SPK = tc_spk(G);
-    constexpr uint32_t RB = tc_row_bytes(W);
-    const float* sc = reinterpret_cast<const float*>(raw + TC_M * RB);
-    const int pr = lane >> 3, rr = lane & 7;
-#pragma unroll 4
-    for (int gg = 0; gg < 8; ++gg) {
-        const int g = 8 * hw + gg;          // row group
-        const int row = 8 * g + rr;
-        const float s0 = sc[row * SPK], s1 = sc[row * SPK + SPK - 1];
-        char* d0 = A + g * 1024 + pr * 128 + rr * 16;
+__device__ __forceinline__ void block_row(const uint8_t* blk, int row, uint32_t (&r)[32]) {
+    if constexpr (W == FOCR_W_BF16) {
+        // the operand image: k-core c of row r at [(r / 8) * 8 + c][r % 8] in 16-byte pieces
+        const uint8_t* base = blk + (row >> 3) * 1024 + (row & 7) * 16;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 v = lds128(base + c * 128);
+            r[4 * c] = v.x;
+            r[4 * c + 1] = v.y;
+            r[4 * c + 2] = v.z;
+            r[4 * c + 3] = v.w;
+        }
+    } else {
+        constexpr int SPK = tc_spk(G);
+        constexpr uint32_t RB = tc_row_bytes(W);
+        const float* sc = reinterpret_cast<const float*>(blk + TC_M * RB) + row * SPK;
+        const float s0 = sc[0], s1 = sc[SPK - 1];   // k-cores 0-3, 4-7
         if constexpr (W == FOCR_W_INT4) {
-            const uint2 c = lds64(raw + row * 32 + pr * 8);
-            const uint32_t b0 = f32x2_to_bf16x2(s0, s0);
-            sts128(d0, dq_int4_bf16(c.x, b0));
-            sts128(d0 + 512, dq_int4_bf16(c.y, SPK == 1 ? b0 : f32x2_to_bf16x2(s1, s1)));
+            // pairs (c, c + 4), 8 bytes each: words k-core c, k-core c + 4
+            const uint4 p01 = lds128(blk + row * 32), p23 = lds128(blk + row * 32 + 16);
+            const uint32_t b0 = f32x2_to_bf16x2(s0, s0), b1 = SPK == 1 ? b0 : f32x2_to_bf16x2(s1, s1);
+            dq_int4_bf16(p01.x, b0, r + 0);
+            dq_int4_bf16(p01.y, b1, r + 16);
+            dq_int4_bf16(p01.z, b0, r + 4);
+            dq_int4_bf16(p01.w, b1, r + 20);
+            dq_int4_bf16(p23.x, b0, r + 8);
+            dq_int4_bf16(p23.y, b1, r + 24);
+            dq_int4_bf16(p23.z, b0, r + 12);
+            dq_int4_bf16(p23.w, b1, r + 28);
         } else {
-            const uint4 c = lds128(raw + row * 64 + pr * 16);
-            sts128(d0, dq_int8_bf16(c.x, c.y, s0));
-            sts128(d0 + 512, dq_int8_bf16(c.z, c.w, s1));
+            // pairs (c, c + 4), 16 bytes each
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 v = lds128(blk + row * 64 + c * 16);
+                dq_int8_bf16(v.x, v.y, s0, r + 4 * c);
+                dq_int8_bf16(v.z, v.w, s1, r + 4 * (c + 4));
+            }
         }
     }
 }
 
-// weight block kb (absolute) of a unit's A operand
-__device__ __forceinline__ const uint8_t* a_block(const TcView& V, const Unit& U, int kb) {
+// One row of a quantised weight block held in registers between its shared-memory load and its
+// conversion, so that both blocks of an A stage are loaded before either is converted.
+template <int W, int G>
+struct RowRaw {
+    static constexpr int NC = W == FOCR_W_INT8 ? 4 : 2;
+    uint4 c[NC];
+    float s0, s1;
+    __device__ __forceinline__ void load(const uint8_t* blk, int row) {
+        constexpr int SPK = tc_spk(G);
+        constexpr uint32_t RB = tc_row_bytes(W);
+        const float* sc = reinterpret_cast<const float*>(blk + TC_M * RB) + row * SPK;
+#pragma unroll
+        for (int i = 0; i < NC; ++i) c[i] = lds128(blk + row * RB + 16 * i);
+        s0 = sc[0];
+        s1 = sc[SPK - 1];
+    }
+    __device__ __forceinline__ void cvt(uint32_t (&r)[32]) const {
+        if constexpr (W == FOCR_W_INT4) {
+            // pairs (c, c + 4), 8 bytes each: words k-core c, k-core c + 4
+            const uint32_t b0 = f32x2_to_bf16x2(s0, s0), b1 = tc_spk(G) == 1 ? b0 : f32x2_to_bf16x2(s1, s1);
+            dq_int4_bf16(c[0].x, b0, r + 0);
+            dq_int4_bf16(c[0].y, b1, r + 16);
+            dq_int4_bf16(c[0].z, b0, r + 4);
+            dq_int4_bf16(c[0].w, b1, r + 20);
+            dq_int4_bf16(c[1].x, b0, r + 8);
+            dq_int4_bf16(c[1].y, b1, r + 24);
+            dq_int4_bf16(c[1].z, b0, r + 12);
+            dq_int4_bf16(c[1].w, b1, r + 28);
+        } else {
+            // pairs (c, c + 4), 16 bytes each
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                dq_int8_bf16(c[i].x, c[i].y, s0, r + 4 * i);
+                dq_int8_bf16(c[i].z, c[i].w, s1, r + 4 * (i + 4));
+            }
+        }
+    }
+};
+
+// This thread's row of the `nb` (1 or 2) adjacent weight blocks at `bp` (`blk` bytes apart) into
+// the two 32-column halves of a TMEM A stage at `ta` (this warp's lane quarter).  Completes with
+// tcgen05.wait::st by the caller.
+template <int W, int G>
+__device__ __forceinline__ void dq_stage(const uint8_t* bp, uint32_t blk, int nb, int row, uint32_t ta) {
+    uint32_t r[32];
+    if constexpr (W == FOCR_W_BF16) {
+        block_row<W, G>(bp, row, r);
+        umma::st32(ta, r);
+        if (nb > 1) {
+            block_row<W, G>(bp + blk, row, r);
+            umma::st32(ta + 32u, r);
+        }
+    } else {
+        RowRaw<W, G> x0, x1;
+        x0.load(bp, row);
+        if (nb > 1) x1.load(bp + blk, row);
+        x0.cvt(r);
+        umma::st32(ta, r);
+        if (nb > 1) {
+            x1.cvt(r);
+            umma::st32(ta + 32u, r);
+        }
+    }
+}
+
+// weight block kb (absolute) of tile `tile` of a unit's set
+__device__ __forceinline__ const uint8_t* w_block(const TcView& V, const Unit& U, int tile, int kb) {
     const bool routed = U.kind == UK_GU_R || U.kind == UK_DN_R;
     const TcSetView& S = routed ? V.r : V.s;
     if (U.kind <= UK_GU_R)
-        return S.gu + (routed ? (size_t)U.expert * S.g.gu_bytes : 0) + ((size_t)U.tile * TC_KBH + kb) * S.g.blk;
-    return S.dn + (routed ? (size_t)U.expert * S.g.dn_bytes : 0) + ((size_t)U.tile * S.g.tiles + kb) * S.g.blk;
+        return S.gu + (routed ? (size_t)U.expert * S.g.gu_bytes : 0) +
+               tc_block_index(S.g.tiles, TC_KBH, tile, kb, S.g.grp) * S.g.blk;
+    return S.dn + (routed ? (size_t)U.expert * S.g.dn_bytes : 0) +
+           tc_block_index(TC_MT, S.g.tiles, tile, kb, S.g.grp) * S.g.blk;
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -243,11 +329,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
     Unit* units = reinterpret_cast<Unit*>(smem + SL::units);
     Sched& S = *reinterpret_cast<Sched*>(smem + SL::sched);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL::bars);
-    uint64_t* ab_full = bars;
-    uint64_t* ab_empty = ab_full + NAB;
-    uint64_t* raw_full = ab_empty + NAB;
+    uint64_t* raw_full = bars;
     uint64_t* raw_empty = raw_full + NR;
-    uint64_t* u_full = raw_empty + NR;
+    uint64_t* b_full = raw_empty + NR;
+    uint64_t* b_empty = b_full + NB;
+    uint64_t* a_full = b_empty + NB;
+    uint64_t* a_empty = a_full + NA;
+    uint64_t* u_full = a_empty + NA;
     uint64_t* u_empty = u_full + UR;
     uint64_t* acc_full = u_empty + UR;
     uint64_t* acc_empty = acc_full + NACC;
@@ -258,17 +346,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int i = 0; i < NAB; ++i) {
-            mbar_init(&ab_full[i], 2 + 1);   // the dequantising pair's two warps + the loader
-            mbar_init(&ab_empty[i], 1);
-        }
         for (int i = 0; i < NR; ++i) {
             mbar_init(&raw_full[i], 1);
-            mbar_init(&raw_empty[i], 2);
+            mbar_init(&raw_empty[i], 4 * SL::cap);   // 4 warps per block; the copier fills in for absent blocks
+        }
+        for (int i = 0; i < NB; ++i) {
+            mbar_init(&b_full[i], 1);
+            mbar_init(&b_empty[i], 1);
+        }
+        for (int i = 0; i < NA; ++i) {
+            mbar_init(&a_full[i], 4);
+            mbar_init(&a_empty[i], 1);
         }
         for (int i = 0; i < UR; ++i) {
             mbar_init(&u_full[i], 1);
-            mbar_init(&u_empty[i], NSTG + 1 + NEPI + 2);
+            mbar_init(&u_empty[i], 4 * NDQG + NEPI + 3);   // dequantisers, epilogue, MMA, copier, loader
         }
         for (int i = 0; i < NACC; ++i) {
             mbar_init(&acc_full[i], 1);
@@ -283,42 +375,54 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
-    pdl_wait();   // routing, x rows and the output of the previous kernel are complete
+    pdl_wait();   // routing, x image and the output of the previous kernel are complete
 
     auto fail = [&](int code) {
         atomicExch(&p.R.ctrl[CTRL_ERROR], code);
         *abort_flag = 1;
     };
 
-    if (warp == WARP_LOAD) {
+    if (warp == WARP_SCHED) {
         // ------------------------------------------------------------ schedule (whole warp)
         const TcGeom& rg = p.V.r.g;
         const TcGeom& sg = p.V.s.g;
         const int T = p.T;
-        const int U = p.shared_only ? 0 : p.R.active[E];
+        // lane l owns experts l and l + 32; the active experts (with tokens) are numbered in
+        // ascending expert order, as the router's list is
+        int cnt[2], offs[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            cnt[h] = p.shared_only ? 0 : p.R.counts[lane + 32 * h];
+            offs[h] = p.shared_only ? 0 : p.R.offsets[lane + 32 * h];
+        }
+        const unsigned m0 = __ballot_sync(0xffffffffu, cnt[0] > 0), m1 = __ballot_sync(0xffffffffu, cnt[1] > 0);
+        const int U = __popc(m0) + __popc(m1);
         int pad[2], gu[2], dn[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const int a = lane + 32 * h;
+            const int e = lane + 32 * h;
+            const int a = h == 0 ? __popc(m0 & ((1u << lane) - 1u)) : __popc(m0) + __popc(m1 & ((1u << lane) - 1u));
             pad[h] = gu[h] = dn[h] = 0;
-            if (a < U) {
-                const int e = p.R.active[a];
-                const int n = p.R.counts[e];
+            if (cnt[h] > 0) {
+                const int n = cnt[h];
                 const int nch0 = (n + NCH - 1) / NCH;
                 const int cs = ((n + nch0 - 1) / nch0 + 15) & ~15;   // chunk size, a multiple of 16
                 const int nch = (n + cs - 1) / cs;
                 S.e[a] = e;
                 S.n[a] = n;
-                S.off[a] = p.R.offsets[e];
+                S.off[a] = offs[h];
                 S.nch[a] = nch;
                 S.cs[a] = cs;
                 pad[h] = (n + 15) & ~15;
-                gu[h] = rg.tiles * nch;
-                dn[h] = TC_MT * nch;
+                for (int c = 0; c < nch; ++c) {
+                    const int mt = mt_for((min(cs, n - c * cs) + 15) & ~15, tc_tile_group(RW));
+                    gu[h] += (rg.tiles + mt - 1) / mt;
+                    dn[h] += (TC_MT + mt - 1) / mt;
+                }
             }
         }
-        // exclusive prefix sums over the active experts a = lane + 32 h (padded a-image rows,
-        // gate/up units, down units)
+        // exclusive prefix sums in expert order (inactive experts add nothing), stored at the active
+        // index: padded image rows, gate/up units, down units
         int sp[2] = {pad[0], pad[1]}, sgu[2] = {gu[0], gu[1]}, sdn[2] = {dn[0], dn[1]};
 #pragma unroll
         for (int h = 0; h < 2; ++h)
@@ -338,8 +442,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
         sdn[1] += __shfl_sync(0xffffffffu, sdn[0], 31);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const int a = lane + 32 * h;
-            if (a < U) {
+            const int a = h == 0 ? __popc(m0 & ((1u << lane) - 1u)) : __popc(m0) + __popc(m1 & ((1u << lane) - 1u));
+            if (cnt[h] > 0) {
                 S.poff[a] = sp[h] - pad[h];
                 S.gu_pre[a] = sgu[h] - gu[h];
                 S.dn_pre[a] = sdn[h] - dn[h];
@@ -364,7 +468,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
         }
         __syncwarp();
 
-        // ------------------------------------------------------------ loader loop
+        // ------------------------------------------------------------ scheduler loop
         for (int k = 0;; ++k) {
             int u = 0;
             if (lane == 0) u = *abort_flag ? S.total : atomicAdd(&ctrl[TC_WORK], 1);
@@ -387,6 +491,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                     if (lane == 0) {
                         Un.expert = S.e[v];
                         Un.tile = Un.part = 0;
+                        Un.mt = 1;
                         Un.kb0 = Un.nkb = 0;
                         Un.c0 = 0;
                         Un.ntok = S.n[v];
@@ -402,6 +507,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                     if (lane == 0) {
                         Un.expert = -1;
                         Un.tile = tile;
+                        Un.mt = 1;
                         Un.part = tile / S.KPP;
                         Un.kb0 = 0;
                         Un.nkb = TC_KBH;
@@ -416,11 +522,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                     kind = UK_GU_R;
                 } else if ((v -= S.n_gu_r) < S.n_dn_s) {
                     kind = UK_DN_S;
-                    const int mt = v / (S.P * S.nchs), rem = v % (S.P * S.nchs);
+                    const int mtile = v / (S.P * S.nchs), rem = v % (S.P * S.nchs);
                     const int part = rem / S.nchs, ch = rem % S.nchs;
                     if (lane == 0) {
                         Un.expert = -1;
-                        Un.tile = mt;
+                        Un.tile = mtile;
+                        Un.mt = 1;
                         Un.part = part;
                         Un.kb0 = part * S.KPP;
                         Un.nkb = min(S.KPP, sg.tiles - Un.kb0);
@@ -436,33 +543,42 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                     kind = UK_DN_R;
                 }
                 if (kind == UK_GU_R || kind == UK_DN_R) {
-                    const int* pre = kind == UK_GU_R ? S.gu_pre : S.dn_pre;
+                    const bool g_u = kind == UK_GU_R;
+                    const int* pre = g_u ? S.gu_pre : S.dn_pre;
                     int lo = 0, hi = S.U - 1;   // last a with pre[a] <= v
                     while (lo < hi) {
                         const int mid = (lo + hi + 1) >> 1;
                         if (pre[mid] <= v) lo = mid;
                         else hi = mid - 1;
                     }
-                    const int a = lo, w = v - pre[a];
-                    const int nch = S.nch[a];
-                    const int tile = w / nch, ch = w % nch;
+                    const int a = lo;
+                    int w = v - pre[a];
+                    const int ntiles = g_u ? rg.tiles : TC_MT;
+                    int ch = 0, mt = 1;
+                    for (;; ++ch) {   // the chunk of the expert this unit falls in
+                        mt = mt_for((min(S.cs[a], S.n[a] - ch * S.cs[a]) + 15) & ~15, tc_tile_group(RW));
+                        const int per = (ntiles + mt - 1) / mt;
+                        if (w < per || ch + 1 >= S.nch[a]) break;
+                        w -= per;
+                    }
                     const int c0 = ch * S.cs[a];
                     const int ntok = min(S.cs[a], S.n[a] - c0);
                     const int seg = S.off[a] + c0;
                     if (lane == 0) {
                         Un.expert = S.e[a];
-                        Un.tile = tile;
+                        Un.tile = w * mt;
+                        Un.mt = min(mt, ntiles - w * mt);
                         Un.part = 0;
                         Un.kb0 = 0;
-                        Un.nkb = kind == UK_GU_R ? TC_KBH : rg.tiles;
+                        Un.nkb = g_u ? TC_KBH : rg.tiles;
                         Un.c0 = c0;
                         Un.ntok = ntok;
                         Un.arow = S.poff[a] + c0;
                         Un.seg = seg;
                         // gate/up waits for the expert's gathered rows, down for all its gate/up units
-                        Un.wdep = kind == UK_DN_R ? TC_DEP_R + S.e[a] : TC_DEP_X + S.e[a];
-                        Un.wtarget = kind == UK_DN_R ? rg.tiles * nch * NEPI : NEPI;
-                        Un.ddep = kind == UK_DN_R ? TC_DN_DONE : TC_DEP_R + S.e[a];
+                        Un.wdep = g_u ? TC_DEP_X + S.e[a] : TC_DEP_R + S.e[a];
+                        Un.wtarget = g_u ? NEPI : (S.gu_pre[a + 1] - S.gu_pre[a]) * NEPI;
+                        Un.ddep = g_u ? TC_DEP_R + S.e[a] : TC_DN_DONE;
                     }
                     for (int n = lane; n < ntok; n += 32) {
                         const int ent = p.R.perm[seg + n];
@@ -476,20 +592,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&u_full[slot]);
             if (kind == UK_END) break;
-            if (lane == 0 && kind != UK_XG) {
-                // the copier will stream this unit's blocks a few units from now: bring them into L2
-                const bool routed = kind == UK_GU_R || kind == UK_DN_R;
-                const int wt = routed ? RW : SW;
-                const uint32_t blk = is_quant(wt) ? (routed ? p.V.r.g.blk : p.V.s.g.blk) : A_BYTES;
-                const uint8_t* b0 = a_block(p.V, Un, Un.kb0);
-                const uint32_t bytes = (uint32_t)Un.nkb * blk;   // the unit's blocks are contiguous
-                for (uint32_t o = 0; o < bytes; o += 64u * 1024u)
-                    bulk_prefetch_l2(b0 + o, min(64u * 1024u, bytes - o));
-            }
             if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
         }
     } else if (warp == WARP_COPY) {
-        // ------------------------------------------------------------ raw-ring copier (one thread)
+        // ------------------------------------------------------------ weight copier (one thread)
+        // Per unit: super-slots of a few K-blocks x the unit's tiles, one bulk copy per K-block
+        // (or one per super-slot where the K-blocks of a single tile are adjacent).
         if (lane == 0) {
             const uint64_t pol = policy_evict_first();
             int raw_i = 0;
@@ -506,20 +614,28 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                     break;
                 }
                 const bool routed = kind == UK_GU_R || kind == UK_DN_R;
-                const int wt = routed ? RW : SW;
+                const TcGeom& gg = routed ? p.V.r.g : p.V.s.g;
+                const int mt = Un.mt, kq = max(1, (routed ? SL::cap_r : SL::cap_s) / mt);
+                const bool whole = gg.grp == 1 && mt == 1;   // K-blocks of one tile are adjacent
                 bool ok = true;
-                if (is_quant(wt)) {
-                    const uint32_t blk = routed ? p.V.r.g.blk : p.V.s.g.blk;
-                    const int nkb = Un.nkb, kb0 = Un.kb0;
-                    for (int kb = 0; kb < nkb; ++kb, ++raw_i) {
-                        const int r = raw_i % NR;
-                        if (!mbar_wait_bounded(&raw_empty[r], ((raw_i / NR) & 1) ^ 1, WAIT_LIMIT_NS)) {
-                            ok = false;
-                            break;
-                        }
-                        mbar_arrive_expect_tx(&raw_full[r], blk);
-                        bulk_g2s(smem + SL::raw + r * SL::raw_slot, a_block(p.V, Un, kb0 + kb), blk, &raw_full[r],
-                                 pol);
+                for (int kb = 0; kb < Un.nkb; kb += kq, ++raw_i) {
+                    // super-slot: K-blocks [kb, kb + nk) x the unit's mt tiles, block (j, t) at j mt + t
+                    const int nk = min(kq, Un.nkb - kb);
+                    const int r = raw_i % NR;
+                    if (!mbar_wait_bounded(&raw_empty[r], ((raw_i / NR) & 1) ^ 1, WAIT_LIMIT_NS)) {
+                        ok = false;
+                        break;
+                    }
+                    for (int i = nk * mt; i < SL::cap; ++i)   // blocks this super-slot does not hold
+                        for (int j = 0; j < 4; ++j) mbar_arrive(&raw_empty[r]);
+                    mbar_arrive_expect_tx(&raw_full[r], (uint32_t)(nk * mt) * gg.blk);
+                    char* dst = smem + SL::braw + r * SL::raw_slot;
+                    if (whole) {
+                        bulk_g2s(dst, w_block(p.V, Un, Un.tile, Un.kb0 + kb), (uint32_t)nk * gg.blk, &raw_full[r], pol);
+                    } else {
+                        for (int j = 0; j < nk; ++j)   // the unit's tiles of one K-block are adjacent
+                            bulk_g2s(dst + (size_t)j * mt * gg.blk, w_block(p.V, Un, Un.tile, Un.kb0 + kb + j),
+                                     (uint32_t)mt * gg.blk, &raw_full[r], pol);
                     }
                 }
                 mbar_arrive(&u_empty[slot]);
@@ -529,18 +645,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                 }
                 if (*abort_flag) break;
             }
-            // never leave copies in flight: the last NR issued blocks must have landed
+            // never leave copies in flight: the last NR issued super-slots must have landed
             for (int i = max(0, raw_i - NR); i < raw_i; ++i)
                 (void)mbar_wait_bounded(&raw_full[i % NR], (i / NR) & 1, WAIT_LIMIT_NS);
         }
         __syncwarp();
     } else if (warp == WARP_BLD) {
-        // ------------------------------------------------------------ operand-stage loader (one thread)
-        // Every stage in order: the B operand (N rows of an operand image: x in token order for the
-        // shared set, x in dispatch order for routed experts, a for down projections) and, for
-        // bf16 weights, the A block, by bulk copies completing on the stage barrier.
+        // ------------------------------------------------------------ token-row loader (one thread)
+        // Per K-block: N rows of an operand image (x in token order for the shared set, x in
+        // dispatch order for routed experts, a for down projections).
         if (lane == 0) {
-            int ab_i = 0;
+            int b_i = 0;
             for (int k = 0;; ++k) {
                 const int slot = k % UR;
                 if (!mbar_wait_bounded(&u_full[slot], (k / UR) & 1, WAIT_LIMIT_NS)) {
@@ -555,28 +670,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                 }
                 const bool routed = kind == UK_GU_R || kind == UK_DN_R;
                 const bool is_gu = kind <= UK_GU_R;
-                const bool quant = is_quant(routed ? RW : SW);
-                const int N = Un.N, kb0 = Un.kb0, nkb = Un.nkb;
                 const uint16_t* img = is_gu ? (routed ? p.W.x_img_r : p.W.x_img) : (routed ? p.W.a_img : p.W.a_sh);
                 const int rows = routed ? p.W.arows : p.W.tpad;
-                const uint32_t bbytes = (uint32_t)N * 128u;
+                const uint32_t bytes = (uint32_t)Un.N * 128u;
                 bool ok = true;
-                if (nkb > 0 && Un.wdep >= 0) {
+                if (Un.nkb > 0 && Un.wdep >= 0) {
                     // the rows come from other units' epilogues: wait until they are all written
                     ok = wait_counter(&ctrl[Un.wdep], Un.wtarget);
                     fence_proxy_async_all();
                 }
-                for (int kb = 0; kb < nkb && ok; ++kb, ++ab_i) {
-                    const int s = ab_i % NAB;
-                    char* Ast = smem + SL::ab + s * STAGE_BYTES;
-                    if (!mbar_wait_bounded(&ab_empty[s], ((ab_i / NAB) & 1) ^ 1, WAIT_LIMIT_NS)) {
+                for (int kb = 0; kb < Un.nkb && ok; ++kb, ++b_i) {
+                    const int s = b_i % NB;
+                    if (!mbar_wait_bounded(&b_empty[s], ((b_i / NB) & 1) ^ 1, WAIT_LIMIT_NS)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&ab_full[s], bbytes + (quant ? 0u : A_BYTES));
-                    if (!quant) bulk_g2s(Ast, a_block(p.V, Un, kb0 + kb), A_BYTES, &ab_full[s], policy_evict_first());
-                    bulk_g2s(Ast + A_BYTES, img + ((size_t)(kb0 + kb) * rows + Un.arow) * TC_KB, bbytes, &ab_full[s],
-                             policy_evict_last());
+                    mbar_arrive_expect_tx(&b_full[s], bytes);
+                    bulk_g2s(smem + SL::bstage + s * B_SLOT, img + ((size_t)(Un.kb0 + kb) * rows + Un.arow) * TC_KB,
+                             bytes, &b_full[s], policy_evict_last());
                 }
                 if (!ok) {
                     fail(DEVERR_TC_WAIT);
@@ -590,7 +701,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
     } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------ MMA issuer (one thread)
         if (lane == 0) {
-            int ab_i = 0, acc_i = 0;
+            int a_i = 0, b_i = 0, acc_i = 0;
             for (int k = 0;; ++k) {
                 const int slot = k % UR;
                 if (!mbar_wait_bounded(&u_full[slot], (k / UR) & 1, WAIT_LIMIT_NS)) {
@@ -612,23 +723,42 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                     break;
                 }
                 umma::fence_after_sync();
-                const uint32_t idesc = umma::idesc_bf16_f32(TC_M, Un.N);
-                const uint32_t d = tmem_base + (uint32_t)(b * 128);
+                const int N = Un.N, mt = Un.mt;
+                const uint32_t idesc = umma::idesc_bf16_f32(TC_M, N);
+                const uint32_t d0 = tmem_base + (uint32_t)(b * 128);
+                const int pp = stages_per_kb(mt), nst = Un.nkb * pp;
                 bool ok = true;
-                for (int kb = 0; kb < Un.nkb; ++kb, ++ab_i) {
-                    const int s = ab_i % NAB;
-                    if (!mbar_wait_bounded(&ab_full[s], (ab_i / NAB) & 1, WAIT_LIMIT_NS)) {
+                uint32_t b0 = 0;
+                for (int st = 0; st < nst; ++st, ++a_i) {
+                    const int kb = st / pp, t0 = 2 * (st % pp);
+                    const int bs = b_i % NB;
+                    if (t0 == 0) {   // first stage of a K-block: its token rows
+                        if (!mbar_wait_bounded(&b_full[bs], (b_i / NB) & 1, WAIT_LIMIT_NS)) {
+                            ok = false;
+                            break;
+                        }
+                        b0 = smem_u32(smem + SL::bstage + bs * B_SLOT);
+                    }
+                    const int as = a_i % NA;
+                    if (!mbar_wait_bounded(&a_full[as], (a_i / NA) & 1, WAIT_LIMIT_NS)) {
                         ok = false;
                         break;
                     }
                     umma::fence_after_sync();
-                    const uint32_t a0 = smem_u32(smem + SL::ab + s * STAGE_BYTES);
-                    const uint32_t b0 = a0 + A_BYTES;
+                    const uint32_t a0 = tmem_base + TM_A0 + (uint32_t)(as * 64);
 #pragma unroll
-                    for (int j = 0; j < TC_KB / 16; ++j)
-                        umma::mma_bf16(d, umma::sdesc_kmajor(a0 + 256u * j, 128u, 1024u),
-                                       umma::sdesc_kmajor(b0 + 256u * j, 128u, 1024u), idesc, kb > 0 || j > 0);
-                    umma::commit(smem_u32(&ab_empty[s]));
+                    for (int i = 0; i < 2; ++i) {
+                        if (t0 + i >= mt) break;
+#pragma unroll
+                        for (int j = 0; j < TC_KB / 16; ++j)
+                            umma::mma_bf16_ts(d0 + (uint32_t)((t0 + i) * N), a0 + 32u * i + 8u * j,
+                                              umma::sdesc_kmajor(b0 + 256u * j, 128u, 1024u), idesc, kb > 0 || j > 0);
+                    }
+                    umma::commit(smem_u32(&a_empty[as]));
+                    if (t0 + 2 >= mt) {   // last stage of the K-block: release its token rows
+                        umma::commit(smem_u32(&b_empty[bs]));
+                        ++b_i;
+                    }
                 }
                 if (!ok) {
                     fail(DEVERR_TC_WAIT);
@@ -645,14 +775,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
         }
         __syncwarp();
     } else if (warp < WARP_EPI) {
-        // ------------------------------------------------------------ dequantising stagers
-        // Warp pair pp = (sw / 2) takes every NPAIR-th operand stage in turn; warp hw = sw % 2 of
-        // the pair dequantises block rows 64 hw .. 64 hw + 63 of a quantised A block (for a bf16
-        // block the pair only takes its turn: the loader warp copies it).  The pair's stores are
-        // ordered before the tensor core's reads by a proxy fence, then each warp arrives.
-        const int sw = warp - WARP_STG;
-        const int pp = sw >> 1, hw = sw & 1;
-        int ab_i = 0, raw_i = 0;
+        // ------------------------------------------------------------ dequantisers
+        // Group dg takes every NDQG-th A stage (the unit's stages in K-block-major order, two
+        // tiles of one K-block each); warp q of the group converts block rows 32 q .. 32 q + 31
+        // (thread = row) of the stage's blocks and writes them to its TMEM columns.
+        const int dg = (warp - WARP_DQ) >> 2, q = warp & 3;
+        const int row = 32 * q + lane;
+        int a_i = 0, raw_i = 0;   // blocks and super-slots of all units so far
         for (int k = 0;; ++k) {
             const int slot = k % UR;
             bool ok = true;
@@ -668,34 +797,36 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                 break;
             }
             const bool routed = kind == UK_GU_R || kind == UK_DN_R;
-            const bool quant = is_quant(routed ? RW : SW);
-            const int nkb = Un.nkb;
-            for (int kb = 0; kb < nkb && ok; ++kb, ++ab_i) {
-                const int r = raw_i;
-                if (quant) ++raw_i;
-                if (ab_i % NPAIR != pp) continue;
-                const int s = ab_i % NAB;
-                char* Ast = smem + SL::ab + s * STAGE_BYTES;
-                if (lane == 0) ok = mbar_wait_bounded(&ab_empty[s], ((ab_i / NAB) & 1) ^ 1, WAIT_LIMIT_NS);
+            const int nkb = Un.nkb, mt = Un.mt;
+            const uint32_t blk = routed ? p.V.r.g.blk : p.V.s.g.blk;
+            const int kq = max(1, (routed ? SL::cap_r : SL::cap_s) / mt);   // K-blocks per super-slot
+            const int pp = stages_per_kb(mt), nst = nkb * pp;
+            for (int st = 0; st < nst && ok; ++st, ++a_i) {
+                if (a_i % NDQG != dg) continue;
+                const int kb = st / pp, t0 = 2 * (st % pp), nb = min(2, mt - t0);
+                const int as = a_i % NA;
+                const int ri = raw_i + kb / kq;   // the super-slot holding K-block kb of every tile
+                const int rs = ri % NR;
+                if (lane == 0) {
+                    ok = mbar_wait_bounded(&a_empty[as], ((a_i / NA) & 1) ^ 1, WAIT_LIMIT_NS) &&
+                         mbar_wait_bounded(&raw_full[rs], (ri / NR) & 1, WAIT_LIMIT_NS);
+                }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
-                if (quant) {
-                    const int rs = r % NR;
-                    if (lane == 0) ok = mbar_wait_bounded(&raw_full[rs], (r / NR) & 1, WAIT_LIMIT_NS);
-                    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                    if (!ok) break;
-                    const uint8_t* raw = reinterpret_cast<const uint8_t*>(smem + SL::raw + rs * SL::raw_slot);
-                    if (routed) {
-                        if constexpr (is_quant(RW)) dequant_half<RW, G>(raw, Ast, hw, lane);
-                    } else {
-                        if constexpr (is_quant(SW)) dequant_half<SW, G>(raw, Ast, hw, lane);
-                    }
-                    umma::fence_smem_to_async();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&raw_empty[rs]);
+                const uint8_t* bp = reinterpret_cast<const uint8_t*>(smem + SL::braw + rs * SL::raw_slot) +
+                                    (size_t)((kb % kq) * mt + t0) * blk;
+                const uint32_t ta = tmem_base + ((uint32_t)(32 * q) << 16) + TM_A0 + (uint32_t)(as * 64);
+                if (routed) dq_stage<RW, G>(bp, blk, nb, row, ta);
+                else dq_stage<SW, G>(bp, blk, nb, row, ta);
+                umma::wait_st();
+                umma::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&a_full[as]);
+                    for (int i = 0; i < nb; ++i) mbar_arrive(&raw_empty[rs]);
                 }
-                if (lane == 0) mbar_arrive(&ab_full[s]);
             }
+            raw_i += (nkb + kq - 1) / kq;
             if (!ok) {
                 if (lane == 0) fail(DEVERR_TC_WAIT);
                 break;
@@ -723,19 +854,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             }
             if (kind == UK_XG) {
                 // the expert's token rows of x, in dispatch order, into its padded segment of the
-                // dispatch-order image: 16-byte pieces, consecutive threads writing consecutive pieces
-                const int et = (warp - WARP_EPI) * 32 + lane, n = Un.ntok, r8 = (n + 7) & ~7;
-                const int per_kb = r8 * 8;   // pieces of one K-block
+                // dispatch-order image.  Thread = (row, k-core) piece column: the row's token is read
+                // once, then its 20 K-blocks' 16-byte pieces are independent loads kept in flight.
+                const int et = (warp - WARP_EPI) * 32 + lane, n = Un.ntok;
                 const uint4* src = reinterpret_cast<const uint4*>(p.W.x_img);
                 uint4* dst = reinterpret_cast<uint4*>(p.W.x_img_r);
-                for (int c = et; c < TC_KBH * per_kb; c += NEPI * 32) {
-                    const int kb = c / per_kb, rem = c % per_kb;
-                    const int row = (rem >> 6) * 8 + (rem & 7), kc = (rem >> 3) & 7;
-                    if (row < n) {
-                        const int t = p.R.perm[Un.seg + row] / K;
-                        dst[img_index(p.W.arows, Un.arow + row, kb * TC_KB + kc * 8) / 8] =
-                            __ldg(src + img_index(p.W.tpad, t, kb * TC_KB + kc * 8) / 8);
-                    }
+                for (int c = et; c < n * 8; c += NEPI * 32) {
+                    const int rr = c >> 3, kc = c & 7;
+                    const int t = p.R.perm[Un.seg + rr] / K;
+                    uint4 v[TC_KBH];
+#pragma unroll
+                    for (int kb = 0; kb < TC_KBH; ++kb) v[kb] = __ldg(src + img_index(p.W.tpad, t, kb * TC_KB + kc * 8) / 8);
+#pragma unroll
+                    for (int kb = 0; kb < TC_KBH; ++kb) dst[img_index(p.W.arows, Un.arow + rr, kb * TC_KB + kc * 8) / 8] = v[kb];
                 }
                 fence_proxy_async_all();
                 __threadfence();
@@ -755,43 +886,44 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             umma::fence_after_sync();
             const bool routed = kind == UK_GU_R || kind == UK_DN_R;
             const int ntok = Un.ntok, N = Un.N;
-            const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * 128);
-            if (kind <= UK_GU_R) {
-                const bool gate = (lane & 8) == 0;
-                const int i = TC_KB * Un.tile + 16 * q + 8 * (lane >> 4) + (lane & 7);   // intermediate
-                uint16_t* img = routed ? p.W.a_img : p.W.a_sh;
-                const int rows = routed ? p.W.arows : p.W.tpad;
-                uint16_t* col = img + (size_t)(i / TC_KB) * rows * TC_KB + ((i % TC_KB) / 8) * 64 + (i % 8);
-                for (int c = 0; c < N; c += 16) {
-                    float v[16];
-                    umma::ld16(taddr + (uint32_t)c, v);
+            for (int t = 0; t < Un.mt; ++t) {
+                const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * 128 + t * N);
+                if (kind <= UK_GU_R) {
+                    const bool gate = (lane & 8) == 0;
+                    const int i = TC_KB * (Un.tile + t) + 16 * q + 8 * (lane >> 4) + (lane & 7);   // intermediate
+                    uint16_t* img = routed ? p.W.a_img : p.W.a_sh;
+                    const int rows = routed ? p.W.arows : p.W.tpad;
+                    uint16_t* col = img + (size_t)(i / TC_KB) * rows * TC_KB + ((i % TC_KB) / 8) * 64 + (i % 8);
+                    for (int c = 0; c < N; c += 16) {
+                        float v[16];
+                        umma::ld16(taddr + (uint32_t)c, v);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float other = __shfl_xor_sync(0xffffffffu, gate ? v[8 + j] : v[j], 8);
-                        const float g = gate ? v[j] : other;
-                        const float u = gate ? other : v[8 + j];
-                        const int n = c + (gate ? j : 8 + j);
-                        if (n < ntok) {
-                            const float w = routed ? Un.w[n] : 1.0f;
-                            const float a = __fdividef(g, 1.0f + __expf(-g)) * u * w;
-                            const int row = Un.arow + n;
-                            col[(size_t)(row >> 3) * 512 + (row & 7) * 8] =
-                                __bfloat16_as_ushort(__float2bfloat16_rn(a));
+                        for (int j = 0; j < 8; ++j) {
+                            const float other = __shfl_xor_sync(0xffffffffu, gate ? v[8 + j] : v[j], 8);
+                            const float g = gate ? v[j] : other;
+                            const float u = gate ? other : v[8 + j];
+                            const int n = c + (gate ? j : 8 + j);
+                            if (n < ntok) {
+                                const float w = routed ? Un.w[n] : 1.0f;
+                                const float a = __fdividef(g, 1.0f + __expf(-g)) * u * w;
+                                const int rr = Un.arow + n;
+                                col[(size_t)(rr >> 3) * 512 + (rr & 7) * 8] = __bfloat16_as_ushort(__float2bfloat16_rn(a));
+                            }
                         }
                     }
-                }
-            } else {
-                const int m = TC_M * Un.tile + 32 * q + lane;   // output row
-                for (int c = 0; c < N; c += 16) {
-                    float v[16];
-                    umma::ld16(taddr + (uint32_t)c, v);
+                } else {
+                    const int m = TC_M * (Un.tile + t) + 32 * q + lane;   // output row
+                    for (int c = 0; c < N; c += 16) {
+                        float v[16];
+                        umma::ld16(taddr + (uint32_t)c, v);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int n = c + j;
-                        if (n < ntok) {
-                            float* dst = routed ? p.W.y_slot + (size_t)Un.ent[n] * H + m
-                                                : p.W.y_sh + ((size_t)Un.part * p.T + Un.c0 + n) * H + m;
-                            *dst = v[j];
+                        for (int j = 0; j < 16; ++j) {
+                            const int n = c + j;
+                            if (n < ntok) {
+                                float* dst = routed ? p.W.y_slot + (size_t)Un.ent[n] * H + m
+                                                    : p.W.y_sh + ((size_t)Un.part * p.T + Un.c0 + n) * H + m;
+                                *dst = v[j];
+                            }
                         }
                     }
                 }
@@ -805,8 +937,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             fence_proxy_async_all();
             __threadfence();
             __syncwarp();
-            if (lane == 0) atomicAdd(&ctrl[Un.ddep], 1);
-            if (lane == 0) mbar_arrive(&u_empty[slot]);
+            if (lane == 0) {
+                atomicAdd(&ctrl[Un.ddep], 1);
+                mbar_arrive(&u_empty[slot]);
+            }
             if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
         }
     }

@@ -190,7 +190,7 @@ void tc_pack(const Quantised& qg, const Quantised& qu, const Quantised& qd, cons
                          mat = (r >> 3) & 1;                      // rows 16 j + 8 h + r': h = 1 is up
                          row = (int64_t)TC_KB * p + 8 * (r >> 4) + (r & 7);
                      },
-                     gu + ((size_t)p * TC_KBH + kb) * g.blk);
+                     gu + tc_block_index(g.tiles, TC_KBH, p, kb, g.grp) * g.blk);
     for (int mt = 0; mt < TC_MT; ++mt)
         for (int kb = 0; kb < g.tiles; ++kb)
             tc_block(m3, cols3, g, kb,
@@ -198,20 +198,21 @@ void tc_pack(const Quantised& qg, const Quantised& qu, const Quantised& qd, cons
                          mat = 2;
                          row = (int64_t)TC_M * mt + r;
                      },
-                     dn + ((size_t)mt * g.tiles + kb) * g.blk);
+                     dn + tc_block_index(TC_MT, g.tiles, mt, kb, g.grp) * g.blk);
 }
 
 }  // namespace
 
 // Pack one SwiGLU weight set (gate/up [inter, H], down [H, inter]) into item blocks and, when
-// tc_gu/tc_dn are given, into the tensor-core layout as well (one quantisation for both).
+// tc_gu/tc_dn are given, into the tensor-core layout with tile groups of tc_grp as well (one
+// quantisation for both).
 void host_pack_set(const float* gate, const float* up, const float* down, const ItemGeom& g, uint8_t* items,
-                   float* dscale, uint8_t* tc_gu, uint8_t* tc_dn) {
+                   float* dscale, uint8_t* tc_gu, uint8_t* tc_dn, int tc_grp) {
     const int wt = g.wtype;
     const Quantised qg = quantise(gate, g.inter, H, wt, g.group);
     const Quantised qu = quantise(up, g.inter, H, wt, g.group);
     const Quantised qd = quantise(down, H, g.inter, wt, g.group);
-    if (tc_gu && tc_dn) tc_pack(qg, qu, qd, make_tc_geom(wt, g.group, g.inter), tc_gu, tc_dn);
+    if (tc_gu && tc_dn) tc_pack(qg, qu, qd, make_tc_geom(wt, g.group, g.inter, tc_grp), tc_gu, tc_dn);
     const Quantised* m3[3] = {&qg, &qu, &qd};
     const int64_t cols3[3] = {H, H, g.inter};
     const int ngk = is_quant(wt) ? H / g.group : 0;

@@ -10,7 +10,7 @@ namespace focr {
 uint16_t host_f32_to_bf16(float f);
 void host_quantize(const float* w, int64_t rows, int64_t cols, int group, int bits, int8_t* q, float* s);
 void host_pack_set(const float* gate, const float* up, const float* down, const ItemGeom& g, uint8_t* items,
-                   float* dscale, uint8_t* tc_gu = nullptr, uint8_t* tc_dn = nullptr);
+                   float* dscale, uint8_t* tc_gu = nullptr, uint8_t* tc_dn = nullptr, int tc_grp = 1);
 void host_unpack_matrix(const uint8_t* items, const float* dscale, const ItemGeom& g, int which, int8_t* q,
                         uint16_t* b16, float* s);
 void parallel_for(int n, const std::function<void(int)>& fn);
