@@ -271,7 +271,9 @@ constexpr int TC_DN_DONE = 2;     // down-projection units finished
 constexpr int TC_DEP_R = 3;       // [64] gate/up units finished per routed expert
 constexpr int TC_DEP_S = 67;      // [8] gate/up units finished per K part of the shared set
 constexpr int TC_DEP_X = 75;      // [64] token rows of each routed expert gathered
-constexpr int TC_WORDS = 139;
+constexpr int TC_CNT = 139;       // [64] assignments per routed expert, added by the router
+constexpr int TC_WORDS = 203;
+static_assert(CTRL_TC + TC_WORDS <= MAX_TB + 256, "control words fit the ctrl region");
 
 struct RouteView {   // device pointers into the workspace
     int32_t* ctrl;

@@ -388,15 +388,40 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
         const TcGeom& sg = p.V.s.g;
         const int T = p.T;
         // lane l owns experts l and l + 32; the active experts (with tokens) are numbered in
-        // ascending expert order, as the router's list is
+        // ascending expert order.  The router left per-expert assignment counts; each expert's
+        // segment of the dispatch order starts at the exclusive prefix sum of the counts.
         int cnt[2], offs[2];
 #pragma unroll
+        for (int h = 0; h < 2; ++h) cnt[h] = p.shared_only ? 0 : __ldcg(&ctrl[TC_CNT + lane + 32 * h]);
+#pragma unroll
         for (int h = 0; h < 2; ++h) {
-            cnt[h] = p.shared_only ? 0 : p.R.counts[lane + 32 * h];
-            offs[h] = p.shared_only ? 0 : p.R.offsets[lane + 32 * h];
+            int incl = cnt[h];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            offs[h] = incl - cnt[h];
         }
+        offs[1] += __shfl_sync(0xffffffffu, offs[0] + cnt[0], 31);
         const unsigned m0 = __ballot_sync(0xffffffffu, cnt[0] > 0), m1 = __ballot_sync(0xffffffffu, cnt[1] > 0);
         const int U = __popc(m0) + __popc(m1);
+        if (blockIdx.x == 0 && !p.shared_only) {
+            // the routing summary for callers: counts, segment offsets, experts with tokens
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int e = lane + 32 * h;
+                p.R.counts[e] = cnt[h];
+                p.R.offsets[e] = offs[h];
+                if (cnt[h] > 0)
+                    p.R.active[h == 0 ? __popc(m0 & ((1u << lane) - 1u))
+                                      : __popc(m0) + __popc(m1 & ((1u << lane) - 1u))] = e;
+            }
+            if (lane == 31) {
+                p.R.offsets[E] = offs[1] + cnt[1];
+                p.R.active[E] = U;
+            }
+        }
         int pad[2], gu[2], dn[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -580,10 +605,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                         Un.wtarget = g_u ? NEPI : (S.gu_pre[a + 1] - S.gu_pre[a]) * NEPI;
                         Un.ddep = g_u ? TC_DEP_R + S.e[a] : TC_DN_DONE;
                     }
-                    for (int n = lane; n < ntok; n += 32) {
-                        const int ent = p.R.perm[seg + n];
-                        Un.ent[n] = ent;
-                        Un.w[n] = p.R.topk_w[ent];
+                    // the expert's permutation segment is written by its gather unit
+                    bool dep = true;
+                    if (lane == 0) dep = wait_counter(&ctrl[TC_DEP_X + S.e[a]], NEPI);
+                    if (!__shfl_sync(0xffffffffu, dep ? 1 : 0, 0)) {
+                        if (lane == 0) fail(DEVERR_TC_WAIT);
+                        kind = UK_END;
+                    } else {
+                        for (int n = lane; n < ntok; n += 32) {
+                            const int ent = __ldcg(&p.R.perm[seg + n]);
+                            Un.ent[n] = ent;
+                            Un.w[n] = __ldcg(&p.R.topk_w[ent]);
+                        }
                     }
                 }
                 if (lane == 0) Un.N = (Un.ntok + 15) & ~15;
@@ -857,11 +890,48 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                 // dispatch-order image.  Thread = (row, k-core) piece column: the row's token is read
                 // once, then its 20 K-blocks' 16-byte pieces are independent loads kept in flight.
                 const int et = (warp - WARP_EPI) * 32 + lane, n = Un.ntok;
+                {
+                    // the expert's segment of the dispatch order: its entries t * 6 + j in
+                    // ascending order.  Every epilogue warp scans all entries and writes the whole
+                    // segment (the same values), so that it can read back the rows it gathers
+                    // without waiting for the other warps.
+                    const int e = Un.expert, ntot = p.T * K;
+                    const int4* idx4 = reinterpret_cast<const int4*>(p.R.topk_idx);
+                    int base = 0;
+                    for (int b0 = 0; b0 < ntot; b0 += 32 * 4 * 8) {
+                        int4 v[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int i = b0 + (j * 32 + lane) * 4;
+                            v[j] = i < ntot ? __ldcg(idx4 + i / 4) : make_int4(-1, -1, -1, -1);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int i = b0 + (j * 32 + lane) * 4;
+                            const int mk = (int)(v[j].x == e && i < ntot) | ((int)(v[j].y == e && i + 1 < ntot) << 1) |
+                                           ((int)(v[j].z == e && i + 2 < ntot) << 2) |
+                                           ((int)(v[j].w == e && i + 3 < ntot) << 3);
+                            const int c = __popc(mk);
+                            int incl = c;
+#pragma unroll
+                            for (int o = 1; o < 32; o <<= 1) {
+                                const int u = __shfl_up_sync(0xffffffffu, incl, o);
+                                if (lane >= o) incl += u;
+                            }
+                            int r = base + incl - c;
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                if ((mk >> q) & 1) p.R.perm[Un.seg + r++] = i + q;
+                            base += __shfl_sync(0xffffffffu, incl, 31);
+                        }
+                    }
+                    __syncwarp();
+                }
                 const uint4* src = reinterpret_cast<const uint4*>(p.W.x_img);
                 uint4* dst = reinterpret_cast<uint4*>(p.W.x_img_r);
                 for (int c = et; c < n * 8; c += NEPI * 32) {
                     const int rr = c >> 3, kc = c & 7;
-                    const int t = p.R.perm[Un.seg + rr] / K;
+                    const int t = ((volatile const int*)p.R.perm)[Un.seg + rr] / K;
                     uint4 v[TC_KBH];
 #pragma unroll
                     for (int kb = 0; kb < TC_KBH; ++kb) v[kb] = __ldg(src + img_index(p.W.tpad, t, kb * TC_KB + kc * 8) / 8);

@@ -50,6 +50,10 @@ struct RouterParams {
     const float* resid;   // NULL: out starts at zero; else out starts as a copy of resid
     uint16_t* x_img;      // NULL, or x in bf16 as an operand image (tensor-core path)
     int img_rows;         // its rows (T rounded up to 16)
+    // tensor-core path: only the per-expert assignment counts are produced here (added into these
+    // zeroed words); the expert kernel derives offsets and builds each expert's permutation
+    // segment itself, so no block of this grid waits for the others
+    int* tc_counts;
 };
 
 // counts / offsets / active list / stable permutation of n = T*6 <= 64 entries, by one warp.
@@ -376,6 +380,15 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
     }
     __syncthreads();
 
+    if (p.tc_counts) {
+        // per-expert totals of this block's entries, one atomic per expert present
+        if (tid < E) cnt[tid] = 0;
+        __syncthreads();
+        if (tid < nt * K) atomicAdd(&cnt[sidx[tid]], 1);
+        __syncthreads();
+        if (tid < E && cnt[tid] > 0) atomicAdd(&p.tc_counts[tid], cnt[tid]);
+        return;
+    }
     if (gridDim.x == RC) {     // one token block (T <= 8): one warp dispatches from shared memory
         if (warp == 0) dispatch_small(p, sidx, cnt);
         return;
@@ -395,7 +408,7 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
 
 cudaError_t launch_router(const float* x, int T, int /*T_ws*/, const LayerView& L, const RouteView& R, float* out,
                           const float* resid, uint16_t* x_img, int img_rows, cudaStream_t st) {
-    RouterParams p{x, T, L.router, R, out, resid, x_img, img_rows};
+    RouterParams p{x, T, L.router, R, out, resid, x_img, img_rows, x_img ? R.ctrl + CTRL_TC + TC_CNT : nullptr};
     const int TB = T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : 8));
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(((T + TB - 1) / TB) * RC);
