@@ -20,7 +20,8 @@
 //   down unit     (set, MT m-tiles of 128 output rows, [K part,] token chunk): D_t = Down_t a^T over
 //                 the set's intermediates (the shared set's in up to 8 K parts); the epilogue
 //                 writes fp32 rows y per (token, slot) or per (token, part)
-//   gather unit   (routed expert): its token rows of x, in dispatch order, into an operand image
+//   dispatch      (prologue of every CTA, epilogue warps): a share of the token -> expert entries
+//                 placed in their experts' segments (perm) and their x rows copied into an operand image
 //   combine       out[t] = resid + sum_parts y_shared + sum_{j<6} y_slot[t*6+j]
 // Units are handed out by a global atomic counter (gathers, shared gate/up, routed gate/up, shared
 // down, routed down), so a unit only ever waits on units with smaller numbers, which running CTAs
@@ -41,7 +42,7 @@
 //                scale, rounded to bf16 (q * s), written to a TMEM A stage with tcgen05.st;
 //                bf16 blocks are moved to TMEM as they are
 //   warps 16-19  epilogue: tcgen05.ld of the accumulators, SwiGLU or output rows, completion
-//                counts; gather units
+//                counts; first the prologue share of the dispatch
 // Every wait is bounded in time (%globaltimer); on expiry the kernel records an error word,
 // stops taking work, waits (bounded) for its own copies in flight, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -74,7 +75,7 @@ constexpr int DEVERR_TC_WAIT = 3;
 static_assert(WARP_DQ % 4 == 0 && WARP_EPI % 4 == 0, "a group of four warps covers the four TMEM lane quarters");
 static_assert(TM_A0 + NA * 64 <= TMEM_COLS, "TMEM budget");
 
-enum UnitKind { UK_GU_S = 0, UK_GU_R = 1, UK_DN_S = 2, UK_DN_R = 3, UK_XG = 4, UK_END = 5 };
+enum UnitKind { UK_GU_S = 0, UK_GU_R = 1, UK_DN_S = 2, UK_DN_R = 3, UK_END = 5 };
 
 // A stages: a unit's weight blocks (K-block kb, tile t) pass through TMEM two at a time, tiles
 // (2 i, 2 i + 1) of one K-block per stage (a single tile where mt is odd), so that the MMA issuer
@@ -104,7 +105,8 @@ struct Unit {
 
 struct Sched {
     int T, U, nchs, cs_s, P, KPP;
-    int n_xg, n_gu_s, n_gu_r, n_dn_s, n_dn_r, total;
+    unsigned m0, m1;     // experts 0-31 / 32-63 with tokens
+    int n_gu_s, n_gu_r, n_dn_s, n_dn_r, total;
     int e[E], n[E], off[E], poff[E], nch[E], cs[E];
     int gu_pre[E + 1], dn_pre[E + 1];
 };
@@ -136,7 +138,7 @@ struct TcSmem {
     static constexpr uint32_t units = bstage + NB * B_SLOT;                       // [UR] Unit
     static constexpr uint32_t sched = (units + UR * (uint32_t)sizeof(Unit) + 15u) & ~15u;
     static constexpr uint32_t bars = (sched + (uint32_t)sizeof(Sched) + 7u) & ~7u;
-    static constexpr int NBARS = 2 * NR + 2 * NB + 2 * NA + 2 * UR + 2 * NACC + 1;
+    static constexpr int NBARS = 2 * NR + 2 * NB + 2 * NA + 2 * UR + 2 * NACC + 2;
     static constexpr uint32_t misc = bars + 8u * NBARS;                           // tmem base, abort flag
     static constexpr uint32_t total = misc + 16u;
     static_assert(NR >= 4, "weight ring depth");
@@ -320,6 +322,95 @@ __device__ __forceinline__ const uint8_t* w_block(const TcView& V, const Unit& U
            tc_block_index(TC_MT, S.g.tiles, tile, kb, S.g.grp) * S.g.blk;
 }
 
+// Active index of expert e (its rank among the experts with tokens).
+__device__ __forceinline__ int active_index(const Sched& S, int e) {
+    return e < 32 ? __popc(S.m0 & ((1u << e) - 1u)) : __popc(S.m0) + __popc(S.m1 & ((1u << (e - 32)) - 1u));
+}
+
+// The epilogue warps' share of the dispatch (see the prologue in the kernel): warp ew of this CTA
+// takes entries i = blockIdx + gridDim * (ew + NEPI * j), GE of them per pass, each pass one
+// sweep over the entries before its last one.
+__device__ __forceinline__ void epilogue_gather(const TcParams& p, const Sched& S, int* ctrl, int ew, int lane) {
+    constexpr int GE = 4;    // entries per pass
+    constexpr int LB = 8;    // 16-byte index loads per lane in flight
+    const int ntot = p.T * K;
+    const int4* idx4 = reinterpret_cast<const int4*>(p.R.topk_idx);
+    const uint4* src = reinterpret_cast<const uint4*>(p.W.x_img);
+    uint4* dst = reinterpret_cast<uint4*>(p.W.x_img_r);
+    for (int j0 = ew;; j0 += NEPI * GE) {
+        int ii[GE], ee[GE], rk[GE];
+        int lim = 0;
+#pragma unroll
+        for (int g = 0; g < GE; ++g) {
+            const long long i = (long long)blockIdx.x + (long long)gridDim.x * (j0 + NEPI * g);
+            ii[g] = i < ntot ? (int)i : -1;
+            ee[g] = ii[g] >= 0 ? __ldcg(&p.R.topk_idx[ii[g]]) : -1;
+            rk[g] = 0;
+            if (ii[g] >= 0) lim = ii[g];
+        }
+        if (ii[0] < 0) break;
+        // rank of each entry among the earlier entries of its expert
+        for (int c0 = 0; c0 * 4 < lim; c0 += 32 * LB) {
+            int4 v[LB];
+#pragma unroll
+            for (int m = 0; m < LB; ++m) {
+                const int c = c0 + m * 32 + lane;
+                v[m] = c * 4 < lim ? __ldcg(idx4 + c) : make_int4(-1, -1, -1, -1);
+            }
+#pragma unroll
+            for (int m = 0; m < LB; ++m) {
+                const int i = (c0 + m * 32 + lane) * 4;
+#pragma unroll
+                for (int g = 0; g < GE; ++g) {
+                    rk[g] += (int)(v[m].x == ee[g] && i < ii[g]) + (int)(v[m].y == ee[g] && i + 1 < ii[g]) +
+                             (int)(v[m].z == ee[g] && i + 2 < ii[g]) + (int)(v[m].w == ee[g] && i + 3 < ii[g]);
+                }
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < GE; ++g)
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) rk[g] += __shfl_xor_sync(0xffffffffu, rk[g], o);
+        // perm entries and the rows: 20 K-blocks x 8 pieces of 16 bytes per row, 5 per lane, two
+        // rows in flight at a time
+#pragma unroll
+        for (int g0 = 0; g0 < GE; g0 += 2) {
+            uint4 buf[2][5];
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                if (ii[g0 + g] < 0) continue;
+                const int t = ii[g0 + g] / K;
+#pragma unroll
+                for (int m = 0; m < 5; ++m) {
+                    const int pc = m * 32 + lane, kb = pc >> 3, kc = pc & 7;
+                    buf[g][m] = __ldg(src + img_index(p.W.tpad, t, kb * TC_KB + kc * 8) / 8);
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                if (ii[g0 + g] < 0) continue;
+                const int a = active_index(S, ee[g0 + g]);
+                const int row = S.poff[a] + rk[g0 + g];
+                if (lane == 0) p.R.perm[S.off[a] + rk[g0 + g]] = ii[g0 + g];
+#pragma unroll
+                for (int m = 0; m < 5; ++m) {
+                    const int pc = m * 32 + lane, kb = pc >> 3, kc = pc & 7;
+                    dst[img_index(p.W.arows, row, kb * TC_KB + kc * 8) / 8] = buf[g][m];
+                }
+            }
+        }
+        // publish: the rows (read by the tensor-memory copies) and perm, then the counters
+        fence_proxy_async_all();
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+            for (int g = 0; g < GE; ++g)
+                if (ii[g] >= 0) atomicAdd(&ctrl[TC_DEP_X + ee[g]], 1);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ the kernel
 template <int RW, int SW, int G>
 __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
@@ -340,6 +431,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
     uint64_t* acc_full = u_empty + UR;
     uint64_t* acc_empty = acc_full + NACC;
     uint64_t* drain = acc_empty + NACC;   // the MMA thread's last commit before TMEM is freed
+    uint64_t* s_ready = drain + 1;        // the schedule summary S is written
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SL::misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SL::misc + 4);
     int* ctrl = p.R.ctrl + CTRL_TC;
@@ -367,6 +459,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             mbar_init(&acc_empty[i], NEPI);
         }
         mbar_init(drain, 1);
+        mbar_init(s_ready, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -484,14 +577,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             S.nchs = (T + S.cs_s - 1) / S.cs_s;
             S.P = tc_parts(sg.inter);
             S.KPP = tc_kpp(sg.inter);
-            S.n_xg = U;
+            S.m0 = m0;
+            S.m1 = m1;
             S.n_gu_s = sg.tiles * S.nchs;
             S.n_gu_r = sgu[1];
             S.n_dn_s = TC_MT * S.P * S.nchs;
             S.n_dn_r = sdn[1];
-            S.total = S.n_xg + S.n_gu_s + S.n_gu_r + S.n_dn_s + S.n_dn_r;
+            S.total = S.n_gu_s + S.n_gu_r + S.n_dn_s + S.n_dn_r;
         }
         __syncwarp();
+        if (lane == 0) mbar_arrive(s_ready);
 
         // ------------------------------------------------------------ scheduler loop
         for (int k = 0;; ++k) {
@@ -510,23 +605,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             int kind = UK_END;
             if (u < S.total) {
                 int v = u;
-                if (v < S.n_xg) {
-                    // gather unit of active expert v: its token rows of x into dispatch order
-                    kind = UK_XG;
-                    if (lane == 0) {
-                        Un.expert = S.e[v];
-                        Un.tile = Un.part = 0;
-                        Un.mt = 1;
-                        Un.kb0 = Un.nkb = 0;
-                        Un.c0 = 0;
-                        Un.ntok = S.n[v];
-                        Un.arow = S.poff[v];
-                        Un.seg = S.off[v];
-                        Un.wdep = -1;
-                        Un.wtarget = 0;
-                        Un.ddep = TC_DEP_X + S.e[v];
-                    }
-                } else if ((v -= S.n_xg) < S.n_gu_s) {
+                if (v < S.n_gu_s) {
                     kind = UK_GU_S;
                     const int tile = v / S.nchs, ch = v % S.nchs;
                     if (lane == 0) {
@@ -602,12 +681,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                         Un.seg = seg;
                         // gate/up waits for the expert's gathered rows, down for all its gate/up units
                         Un.wdep = g_u ? TC_DEP_X + S.e[a] : TC_DEP_R + S.e[a];
-                        Un.wtarget = g_u ? NEPI : (S.gu_pre[a + 1] - S.gu_pre[a]) * NEPI;
+                        Un.wtarget = g_u ? S.n[a] : (S.gu_pre[a + 1] - S.gu_pre[a]) * NEPI;
                         Un.ddep = g_u ? TC_DEP_R + S.e[a] : TC_DN_DONE;
                     }
-                    // the expert's permutation segment is written by its gather unit
+                    // the expert's permutation segment is written as its rows are gathered
                     bool dep = true;
-                    if (lane == 0) dep = wait_counter(&ctrl[TC_DEP_X + S.e[a]], NEPI);
+                    if (lane == 0) dep = wait_counter(&ctrl[TC_DEP_X + S.e[a]], S.n[a]);
                     if (!__shfl_sync(0xffffffffu, dep ? 1 : 0, 0)) {
                         if (lane == 0) fail(DEVERR_TC_WAIT);
                         kind = UK_END;
@@ -746,10 +825,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                     mbar_arrive(&u_empty[slot]);
                     break;
                 }
-                if (Un.kind == UK_XG) {   // no MMA work
-                    mbar_arrive(&u_empty[slot]);
-                    continue;
-                }
                 const int b = acc_i % NACC;
                 if (!mbar_wait_bounded(&acc_empty[b], ((acc_i / NACC) & 1) ^ 1, WAIT_LIMIT_NS)) {
                     fail(DEVERR_TC_WAIT);
@@ -871,7 +946,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;   // TMEM lane quarter this warp may access
         int acc_i = 0;
-        for (int k = 0;; ++k) {
+        bool go_on = true;
+        if (!p.shared_only) {
+            // Prologue: every CTA places a share of the dispatch entries.  Entry i = t * 6 + j of
+            // expert e goes to rank r = #{entries i' < i of expert e} of e's segment: perm[off_e + r]
+            // = i, and token t's row of the x image is copied to row poff_e + r of the dispatch-
+            // order image.  Each placed entry adds one to e's gathered-rows counter.
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait_bounded(s_ready, 0, WAIT_LIMIT_NS);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) {
+                if (lane == 0) fail(DEVERR_TC_WAIT);
+                go_on = false;
+            } else {
+                epilogue_gather(p, S, ctrl, warp - WARP_EPI, lane);
+            }
+        }
+        for (int k = 0; go_on; ++k) {
             const int slot = k % UR;
             bool ok = true;
             if (lane == 0) ok = mbar_wait_bounded(&u_full[slot], (k / UR) & 1, WAIT_LIMIT_NS);
@@ -884,68 +975,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
             if (kind == UK_END) {
                 if (lane == 0) mbar_arrive(&u_empty[slot]);
                 break;
-            }
-            if (kind == UK_XG) {
-                // the expert's token rows of x, in dispatch order, into its padded segment of the
-                // dispatch-order image.  Thread = (row, k-core) piece column: the row's token is read
-                // once, then its 20 K-blocks' 16-byte pieces are independent loads kept in flight.
-                const int et = (warp - WARP_EPI) * 32 + lane, n = Un.ntok;
-                {
-                    // the expert's segment of the dispatch order: its entries t * 6 + j in
-                    // ascending order.  Every epilogue warp scans all entries and writes the whole
-                    // segment (the same values), so that it can read back the rows it gathers
-                    // without waiting for the other warps.
-                    const int e = Un.expert, ntot = p.T * K;
-                    const int4* idx4 = reinterpret_cast<const int4*>(p.R.topk_idx);
-                    int base = 0;
-                    for (int b0 = 0; b0 < ntot; b0 += 32 * 4 * 8) {
-                        int4 v[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int i = b0 + (j * 32 + lane) * 4;
-                            v[j] = i < ntot ? __ldcg(idx4 + i / 4) : make_int4(-1, -1, -1, -1);
-                        }
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int i = b0 + (j * 32 + lane) * 4;
-                            const int mk = (int)(v[j].x == e && i < ntot) | ((int)(v[j].y == e && i + 1 < ntot) << 1) |
-                                           ((int)(v[j].z == e && i + 2 < ntot) << 2) |
-                                           ((int)(v[j].w == e && i + 3 < ntot) << 3);
-                            const int c = __popc(mk);
-                            int incl = c;
-#pragma unroll
-                            for (int o = 1; o < 32; o <<= 1) {
-                                const int u = __shfl_up_sync(0xffffffffu, incl, o);
-                                if (lane >= o) incl += u;
-                            }
-                            int r = base + incl - c;
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                if ((mk >> q) & 1) p.R.perm[Un.seg + r++] = i + q;
-                            base += __shfl_sync(0xffffffffu, incl, 31);
-                        }
-                    }
-                    __syncwarp();
-                }
-                const uint4* src = reinterpret_cast<const uint4*>(p.W.x_img);
-                uint4* dst = reinterpret_cast<uint4*>(p.W.x_img_r);
-                for (int c = et; c < n * 8; c += NEPI * 32) {
-                    const int rr = c >> 3, kc = c & 7;
-                    const int t = ((volatile const int*)p.R.perm)[Un.seg + rr] / K;
-                    uint4 v[TC_KBH];
-#pragma unroll
-                    for (int kb = 0; kb < TC_KBH; ++kb) v[kb] = __ldg(src + img_index(p.W.tpad, t, kb * TC_KB + kc * 8) / 8);
-#pragma unroll
-                    for (int kb = 0; kb < TC_KBH; ++kb) dst[img_index(p.W.arows, Un.arow + rr, kb * TC_KB + kc * 8) / 8] = v[kb];
-                }
-                fence_proxy_async_all();
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) {
-                    atomicAdd(&ctrl[Un.ddep], 1);
-                    mbar_arrive(&u_empty[slot]);
-                }
-                continue;
             }
             const int b = acc_i % NACC;
             if (lane == 0) ok = mbar_wait_bounded(&acc_full[b], (acc_i / NACC) & 1, WAIT_LIMIT_NS);
