@@ -428,6 +428,8 @@ def run_step_workload(args, rank, world, local_rank):
     lm_ws = torch.zeros(api.focr_lm_head_workspace_bytes(T), dtype=torch.uint8, device=dev)
     hb = [torch.empty(T, 1280, device=dev) for _ in range(2)]
     am = torch.empty(T, dtype=torch.int32, device=dev)
+    model = api.DecodeModel(mlp, layers, head, eps=1e-6) if kind == "stack" else None
+    step_ws = api.new_decode_step_workspace(T, dev) if kind == "stack" else None
     stream = torch.cuda.Stream(device=dev)
     per_dense = 2 if T <= 8 else 2            # (memset or x-rows) + expert kernel(s)
     per_moe = 3 if T <= 8 else 2
@@ -442,7 +444,11 @@ def run_step_workload(args, rank, world, local_rank):
         if kind == "dense":
             api.focr_dense_mlp_forward(mlp, x, out=hb[0], workspace=ws, stream=st)
             return
+        if debug_counts is None:   # the timed path: one C-ABI call for the whole decode step
+            api.focr_decode_step(model, x, argmax=am, workspace=step_ws, stream=st)
+            return
         # h <- RMSNorm(h + FFN(h)) for the dense layer and every MoE layer; the last norm feeds lm_head
+        # (layer by layer here only to read each layer's routing counts for the byte count)
         api.focr_dense_mlp_forward(mlp, x, out=hb[0], workspace=ws, flags=api.FWD_RESIDUAL, stream=st)
         api.focr_rmsnorm(hb[0], eps=1e-6, out=hb[1], stream=st)
         for li, L in enumerate(layers):

@@ -274,6 +274,42 @@ focr_status focr_lm_head_gemv(const focr_lm_head* head, const float* x, int32_t 
 focr_status focr_rmsnorm(const float* x, const float* gamma, int32_t T, float eps, float* out, void* stream);
 
 /*
+ * focr_decode_step -- one decode step of the decoder stack (frankenocr.pages.dev, "One forward
+ * pass", steps 6-7: layer 0 is the dense SwiGLU MLP, the other decoder layers are MoE layers,
+ * a final RMSNorm feeds the lm_head GEMV and greedy decoding takes the argmax):
+ *     h = RMSNorm_0(x + Dense(x));   h = RMSNorm_l(h + MoE_l(h)) for l = 1 .. n_moe;
+ *     logits = lm_head(h);           argmax[t] = index of the largest logit (ties: lowest row)
+ * The attention sub-layers of the decoder are outside this library; callers that run them
+ * chain their own kernels between steps on the same stream.  Every stage is an asynchronous
+ * launch on `stream` (programmatic dependent launch between the library's kernels), so the
+ * whole step can be captured into one CUDA graph.
+ *   m:          the model; layers and lm_head are packed handles, gamma[l] (l = 0 .. n_moe) the
+ *               RMSNorm weights (DEVICE fp32 [1280], 16-byte aligned) or gamma == NULL for all
+ *               ones; eps >= 0.  The library does not take ownership of anything in m.
+ *   x:          DEVICE fp32 [T, 1280], 16-byte aligned, 1 <= T <= FOCR_T_MAX.
+ *   logits:     DEVICE fp32 [T, 129280] or NULL;  argmax: DEVICE int32 [T].
+ *   hidden_out: DEVICE fp32 [T, 1280] (the final normed hidden state) or NULL.
+ *   workspace:  DEVICE, 256-byte aligned, >= focr_decode_step_workspace_bytes(T) bytes,
+ *               zero-filled once before its first use (every step that completes leaves its
+ *               control words zero; calls with different T may share it; calls on one
+ *               workspace must not overlap).  focr_moe_check on (workspace + 256) reports a
+ *               bounded device wait that ran out.
+ * Errors: FOCR_ERR_INVALID_ARG for a NULL or incomplete model, T out of range, misaligned or
+ * too small buffers; FOCR_ERR_CUDA if a launch fails (stages before it stay queued).
+ */
+typedef struct focr_decode_model {
+    const focr_dense_mlp* dense;        /* decoder layer 0 */
+    const focr_moe_layer* const* moe;   /* decoder layers 1 .. n_moe */
+    int32_t n_moe;
+    const float* const* gamma;          /* n_moe + 1 RMSNorm weights, or NULL */
+    float eps;
+    const focr_lm_head* head;
+} focr_decode_model;
+size_t focr_decode_step_workspace_bytes(int32_t T_max);
+focr_status focr_decode_step(const focr_decode_model* m, const float* x, int32_t T, float* logits, int32_t* argmax,
+                             float* hidden_out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * focr_tc_selftest -- diagnostic: one tensor-core tile through the library's tcgen05 primitives
  * (the ones the T > 8 grouped kernel uses), to check them against a host GEMM.
  * D[128, n] = A[128, k] * B[n, k]^T with A, B bf16 bit patterns (DEVICE, row-major, 16-byte

@@ -33,6 +33,7 @@ EXPORTED = (
     "focr_moe_layer_forward_ex", "focr_lm_head_pack", "focr_lm_head_free", "focr_lm_head_export",
     "focr_lm_head_workspace_bytes", "focr_lm_head_gemv", "focr_rmsnorm", "focr_dense_mlp_pack",
     "focr_dense_mlp_free", "focr_dense_mlp_export_quantized", "focr_dense_mlp_forward", "focr_tc_selftest",
+    "focr_decode_step_workspace_bytes", "focr_decode_step",
 )
 FWD_RESIDUAL = 1
 NOALLOC_T_MAX = 320
@@ -58,6 +59,11 @@ class RouteDebug(ctypes.Structure):
 
 _lib = None
 _lock = threading.Lock()
+
+
+class DecodeModelDesc(ctypes.Structure):
+    _fields_ = [("dense", ctypes.c_void_p), ("moe", ctypes.POINTER(ctypes.c_void_p)), ("n_moe", ctypes.c_int32),
+                ("gamma", ctypes.POINTER(ctypes.c_void_p)), ("eps", ctypes.c_float), ("head", ctypes.c_void_p)]
 
 
 def lib():
@@ -94,6 +100,8 @@ def lib():
                 "focr_dense_mlp_export_quantized": (i32, [P, i32, P, sz, P, sz]),
                 "focr_dense_mlp_forward": (i32, [P, P, i32, P, P, sz, i32, P]),
                 "focr_tc_selftest": (i32, [P, P, i32, i32, i32, P, P, P]),
+                "focr_decode_step_workspace_bytes": (sz, [i32]),
+                "focr_decode_step": (i32, [ctypes.POINTER(DecodeModelDesc), P, i32, P, P, P, P, sz, P]),
                 "focr_last_error": (ctypes.c_char_p, []),
                 "focr_version": (ctypes.c_char_p, []),
             }
@@ -350,3 +358,44 @@ def focr_tc_selftest(a, b, a_from_tmem: bool, stream=None):
     err = torch.zeros(1, dtype=torch.int32, device=a.device)
     _check(lib().focr_tc_selftest(_ptr(a), _ptr(b), n, k, int(a_from_tmem), _ptr(d), _ptr(err), _stream(stream)))
     return d, err
+
+
+# ---------------------------------------------------------------- decode step
+class DecodeModel:
+    """Handles of one decoder stack for focr_decode_step: the dense layer 0, the MoE layers, the
+    RMSNorm weights (device tensors [1280] or None for ones) and the lm_head.  Keeps the
+    Python objects alive; owns no device memory of its own."""
+
+    def __init__(self, dense: "DenseMLP", moe_layers, head: LMHead, gammas=None, eps: float = 1e-6):
+        self.dense, self.moe, self.head, self.gammas, self.eps = dense, list(moe_layers), head, gammas, float(eps)
+        self._moe = (ctypes.c_void_p * max(1, len(self.moe)))(*[m.handle for m in self.moe])
+        self._gam = None
+        if gammas is not None:
+            assert len(gammas) == len(self.moe) + 1
+            self._gam = (ctypes.c_void_p * len(gammas))(*[_ptr(g) for g in gammas])
+        self.desc = DecodeModelDesc(dense.handle, ctypes.cast(self._moe, ctypes.POINTER(ctypes.c_void_p)),
+                                    len(self.moe),
+                                    ctypes.cast(self._gam, ctypes.POINTER(ctypes.c_void_p)) if self._gam else None,
+                                    self.eps, head.handle)
+
+
+def new_decode_step_workspace(T_max: int, device=None):
+    """A zero-filled workspace for focr_decode_step calls with up to T_max tokens."""
+    import torch
+    n = lib().focr_decode_step_workspace_bytes(T_max)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def focr_decode_step(model: DecodeModel, x, argmax=None, logits=None, hidden_out=None, workspace=None, stream=None):
+    """One decode step of the stack (dense layer 0, MoE layers, RMSNorms, lm_head + argmax).
+    Returns argmax [T] int32 (device)."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous() and x.shape[-1] == H
+    T = x.shape[0]
+    if argmax is None:
+        argmax = torch.empty(T, dtype=torch.int32, device=x.device)
+    if workspace is None:
+        workspace = new_decode_step_workspace(T, x.device)
+    _check(lib().focr_decode_step(ctypes.byref(model.desc), _ptr(x), T, _ptr(logits), _ptr(argmax), _ptr(hidden_out),
+                                  _ptr(workspace), workspace.numel(), _stream(stream)))
+    return argmax

@@ -590,4 +590,68 @@ focr_status focr_moe_check(void* workspace, void* stream) {
     return FOCR_OK;
 }
 
+// ------------------------------------------------------------------ decode step
+// Workspace of one decode step: [lm_head ticket | MoE/dense workspace | lm_head keys | h0 | h1].
+// The ticket and the MoE workspace's zero prefix sit at offsets that do not depend on T, so
+// calls with different T may share one workspace.
+namespace {
+constexpr size_t kStepMoeOff = 256;
+size_t step_keys_off(int T) { return align_up(kStepMoeOff + focr_moe_workspace_bytes(T), 256); }
+size_t step_h0_off(int T) {
+    return align_up(step_keys_off(T) + sizeof(unsigned long long) * 1024 * (size_t)T, 256);
+}
+size_t step_h1_off(int T) { return align_up(step_h0_off(T) + sizeof(float) * H * (size_t)T, 256); }
+size_t step_bytes(int T) { return align_up(step_h1_off(T) + sizeof(float) * H * (size_t)T, 256); }
+}  // namespace
+
+size_t focr_decode_step_workspace_bytes(int32_t T_max) {
+    if (T_max < 1) T_max = 1;
+    if (T_max > FOCR_T_MAX) T_max = FOCR_T_MAX;
+    return step_bytes(T_max);
+}
+
+focr_status focr_decode_step(const focr_decode_model* m, const float* x, int32_t T, float* logits, int32_t* argmax,
+                             float* hidden_out, void* workspace, size_t ws_bytes, void* stream) {
+    g_err.clear();
+    if (!m || !m->dense || !m->head || m->n_moe < 0 || (m->n_moe > 0 && !m->moe))
+        return fail(FOCR_ERR_INVALID_ARG, "incomplete decode model");
+    for (int i = 0; i < m->n_moe; ++i)
+        if (!m->moe[i]) return fail(FOCR_ERR_INVALID_ARG, "MoE layer %d is NULL", i);
+    if (!(m->eps >= 0.f)) return fail(FOCR_ERR_INVALID_ARG, "eps must be >= 0");
+    if (T < 1 || T > FOCR_T_MAX) return fail(FOCR_ERR_INVALID_ARG, "T=%d outside [1, %d]", T, FOCR_T_MAX);
+    if (!x || !argmax || !workspace) return fail(FOCR_ERR_INVALID_ARG, "x, argmax and workspace must not be NULL");
+    if (!aligned(x, 16) || !aligned(workspace, 256) || (hidden_out && !aligned(hidden_out, 16)))
+        return fail(FOCR_ERR_INVALID_ARG, "misaligned x, hidden_out or workspace");
+    if (ws_bytes < step_bytes(T))
+        return fail(FOCR_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed for T=%d", ws_bytes, step_bytes(T), T);
+    if (lm_head_grid() > 1024) return fail(FOCR_ERR_UNSUPPORTED, "more SMs than the workspace plan");
+    char* w = static_cast<char*>(workspace);
+    void* mws = w + kStepMoeOff;
+    const size_t mws_bytes = focr_moe_workspace_bytes(T);
+    float* h0 = reinterpret_cast<float*>(w + step_h0_off(T));
+    float* h1 = reinterpret_cast<float*>(w + step_h1_off(T));
+    cudaStream_t st = (cudaStream_t)stream;
+    // h <- RMSNorm_l(h + FFN_l(h)) for the dense layer 0 and every MoE layer; the last norm feeds lm_head
+    auto gamma = [&](int l) -> const float* { return m->gamma ? m->gamma[l] : nullptr; };
+    focr_status s = focr_dense_mlp_forward(m->dense, x, T, h0, mws, mws_bytes, FOCR_FWD_RESIDUAL, stream);
+    if (s != FOCR_OK) return s;
+    float* last = (m->n_moe == 0 && hidden_out) ? hidden_out : h1;
+    s = focr_rmsnorm(h0, gamma(0), T, m->eps, last, stream);
+    if (s != FOCR_OK) return s;
+    for (int l = 0; l < m->n_moe; ++l) {
+        s = focr_moe_layer_forward_ex(m->moe[l], last, T, h0, mws, mws_bytes, nullptr, FOCR_FWD_RESIDUAL, stream);
+        if (s != FOCR_OK) return s;
+        float* dst = (l == m->n_moe - 1 && hidden_out) ? hidden_out : h1;
+        s = focr_rmsnorm(h0, gamma(l + 1), T, m->eps, dst, stream);
+        if (s != FOCR_OK) return s;
+        last = dst;
+    }
+    const focr_lm_head* L = m->head;
+    const uint4* codes = reinterpret_cast<const uint4*>(L->dev);
+    const float* scales = reinterpret_cast<const float*>(L->dev + (size_t)FOCR_VOCAB * H);
+    CUDA_TRY(launch_lm_head(codes, scales, last, T, logits, argmax, reinterpret_cast<int*>(w),
+                            reinterpret_cast<unsigned long long*>(w + step_keys_off(T)), st));
+    return FOCR_OK;
+}
+
 }  // extern "C"

@@ -342,8 +342,6 @@ cudaError_t launch_router(const float* x, int T, int T_ws, const LayerView& L, c
 // writes the x image itself.
 cudaError_t launch_expert_tc(const float* x, int T, const TcView& V, const RouteView& R, const TcWork& W,
                              float* out, bool resid, bool shared_only, cudaStream_t st);
-cudaError_t launch_expert_decode(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
-                                 bool shared_only, cudaStream_t st);
 // T <= SMALL_T: gate/up + swiglu kernel, then the down kernel (decode_small.cu)
 constexpr int SMALL_T = 8;
 cudaError_t launch_decode_small(const float* x, int T, const LayerView& L, const RouteView& R, float* out,

@@ -33,6 +33,7 @@
 // weights exact with bf16 hi + lo activations; fp32 accumulation throughout.
 #include "common.cuh"
 #include "fragments.cuh"
+#include "launch_state.h"
 
 namespace focr {
 namespace {
@@ -540,13 +541,10 @@ __global__ void __launch_bounds__(DN_WARPS * 32, 2) decode_down_kernel(SmallPara
     if (first) pdl_wait();   // every CTA waits before exiting (keeps the chain of forwards ordered)
 }
 
-int g_sms = 0;
-
 template <int RW, int SW, int G>
-cudaError_t launch_small_typed(const SmallParams& p, cudaStream_t st) {
+cudaError_t launch_small_typed(const SmallParams& p, int sms, cudaStream_t st) {
     using C = GuCfg<RW, SW, G>;
-    static bool configured = false;
-    if (!configured) {
+    cudaError_t e0 = once_per_device((const void*)decode_gu_kernel<RW, SW, G>, [] {
         cudaError_t e = cudaFuncSetAttribute(decode_gu_kernel<RW, SW, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)C::total);
         if (e != cudaSuccess) return e;
@@ -555,16 +553,15 @@ cudaError_t launch_small_typed(const SmallParams& p, cudaStream_t st) {
         e = cudaFuncSetAttribute(decode_gu_kernel<RW, SW, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(decode_down_kernel<RW, SW, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+        return cudaFuncSetAttribute(decode_down_kernel<RW, SW, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                    cudaSharedmemCarveoutMaxShared);
+    });
+    if (e0 != cudaSuccess) return e0;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(g_sms);
+    cfg.gridDim = dim3(sms);
     cfg.blockDim = dim3(C::NW * 32);
     cfg.dynamicSmemBytes = C::total;
     cfg.stream = st;
@@ -572,7 +569,7 @@ cudaError_t launch_small_typed(const SmallParams& p, cudaStream_t st) {
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, decode_gu_kernel<RW, SW, G>, p);
     if (e != cudaSuccess) return e;
-    cfg.gridDim = dim3(2 * g_sms);
+    cfg.gridDim = dim3(2 * sms);
     cfg.blockDim = dim3(DN_WARPS * 32);
     cfg.dynamicSmemBytes = 0;
     return cudaLaunchKernelEx(&cfg, decode_down_kernel<RW, SW, G>, p);
@@ -583,16 +580,13 @@ cudaError_t launch_small_typed(const SmallParams& p, cudaStream_t st) {
 cudaError_t launch_decode_small(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
                                 bool shared_only, cudaStream_t st) {
     if (T < 1 || T > 8 || L.sg.inter > IS_MAX || L.sg.inter % 8 != 0) return cudaErrorInvalidValue;
-    if (g_sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
-    }
+    const int sms = device_sms();
+    if (sms <= 0) return cudaErrorInvalidDevice;
     const SmallParams p{x, T, out, L, R, shared_only ? 1 : 0};
     const int rw = L.rg.wtype, sw = L.sg.wtype;
     const int g = is_quant(rw) ? L.rg.group : (is_quant(sw) ? L.sg.group : 128);
 #define FOCR_CASE(A, B, GG) \
-    if (rw == A && sw == B && g == GG) return launch_small_typed<A, B, GG>(p, st);
+    if (rw == A && sw == B && g == GG) return launch_small_typed<A, B, GG>(p, sms, st);
     FOCR_CASE(FOCR_W_INT4, FOCR_W_BF16, 32)
     FOCR_CASE(FOCR_W_INT4, FOCR_W_BF16, 64)
     FOCR_CASE(FOCR_W_INT4, FOCR_W_BF16, 128)

@@ -50,6 +50,7 @@
 #include "common.cuh"
 #include "fragments.cuh"
 #include "umma.cuh"
+#include "launch_state.h"
 
 namespace focr {
 namespace {
@@ -1112,20 +1113,16 @@ __global__ void x_image_kernel(const float* x, int T, int rows, uint16_t* img) {
     }
 }
 
-int g_tc_sms = 0;
-
 template <int RW, int SW, int G>
-cudaError_t launch_tc_typed(const TcParams& p, cudaStream_t st) {
+cudaError_t launch_tc_typed(const TcParams& p, int sms, cudaStream_t st) {
     using SL = TcSmem<RW, SW, G>;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(expert_tc_kernel<RW, SW, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SL::total);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    const cudaError_t e = once_per_device((const void*)expert_tc_kernel<RW, SW, G>, [] {
+        return cudaFuncSetAttribute(expert_tc_kernel<RW, SW, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)SL::total);
+    });
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(g_tc_sms);
+    cfg.gridDim = dim3(sms);
     cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = SL::total;
     cfg.stream = st;
@@ -1142,14 +1139,11 @@ cudaError_t launch_tc_typed(const TcParams& p, cudaStream_t st) {
 cudaError_t launch_expert_tc(const float* x, int T, const TcView& V, const RouteView& R, const TcWork& W, float* out,
                              bool resid, bool shared_only, cudaStream_t st) {
     if (T <= SMALL_T) return cudaErrorInvalidValue;
-    if (g_tc_sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&g_tc_sms, cudaDevAttrMultiProcessorCount, dev);
-    }
+    const int sms = device_sms();
+    if (sms <= 0) return cudaErrorInvalidDevice;
     if (shared_only) {
         cudaLaunchConfig_t cfg{};
-        cfg.gridDim = dim3(g_tc_sms);
+        cfg.gridDim = dim3(sms);
         cfg.blockDim = dim3(256);
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
@@ -1164,7 +1158,7 @@ cudaError_t launch_expert_tc(const float* x, int T, const TcView& V, const Route
     const int rw = V.r.g.wtype, sw = V.s.g.wtype;
     const int g = is_quant(rw) ? V.r.g.group : (is_quant(sw) ? V.s.g.group : 128);
 #define FOCR_CASE(A, B, GG) \
-    if (rw == A && sw == B && g == GG) return launch_tc_typed<A, B, GG>(p, st);
+    if (rw == A && sw == B && g == GG) return launch_tc_typed<A, B, GG>(p, sms, st);
     FOCR_CASE(FOCR_W_INT4, FOCR_W_BF16, 32)
     FOCR_CASE(FOCR_W_INT4, FOCR_W_BF16, 64)
     FOCR_CASE(FOCR_W_INT4, FOCR_W_BF16, 128)

@@ -18,6 +18,7 @@
 // its columns; warps and CTAs reduce packed (ordered logit, ~row) keys, and the last CTA
 // to finish (atomic ticket, reset after use) writes argmax[t].
 #include "common.cuh"
+#include "launch_state.h"
 #include "fragments.cuh"
 #include "lm_head.h"
 
@@ -194,22 +195,25 @@ __global__ void __launch_bounds__(LT, 1) lm_head_kernel(LmParams p) {
     if (tid == 0) *p.ticket = 0;
 }
 
-int g_sms = 0;
-
 }  // namespace
 
 size_t lm_head_smem_bytes() { return (size_t)KSTEPS * 4 * 32 * 16 + (size_t)LW * TCH * 8; }
 
 cudaError_t launch_lm_head(const uint4* codes, const float* scales, const float* x, int T, float* logits,
                            int32_t* argmax, void* ws, cudaStream_t st) {
-    static bool configured = false;   // independent of g_sms, which lm_head_grid() may set first
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(lm_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)lm_head_smem_bytes());
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
-    lm_head_grid();
+    return launch_lm_head(codes, scales, x, T, logits, argmax, reinterpret_cast<int*>(ws),
+                          reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(ws) + 256), st);
+}
+
+cudaError_t launch_lm_head(const uint4* codes, const float* scales, const float* x, int T, float* logits,
+                           int32_t* argmax, int* ticket, unsigned long long* keys, cudaStream_t st) {
+    const cudaError_t e = once_per_device((const void*)lm_head_kernel, [] {
+        return cudaFuncSetAttribute(lm_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)lm_head_smem_bytes());
+    });
+    if (e != cudaSuccess) return e;
+    const int sms = device_sms();
+    if (sms <= 0) return cudaErrorInvalidDevice;
     LmParams p;
     p.codes = codes;
     p.scales = scales;
@@ -217,10 +221,10 @@ cudaError_t launch_lm_head(const uint4* codes, const float* scales, const float*
     p.T = T;
     p.logits = logits;
     p.argmax = argmax;
-    p.ticket = reinterpret_cast<int*>(ws);
-    p.keys = reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(ws) + 256);
+    p.ticket = ticket;
+    p.keys = keys;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(g_sms);
+    cfg.gridDim = dim3(sms);
     cfg.blockDim = dim3(LT);
     cfg.dynamicSmemBytes = lm_head_smem_bytes();
     cfg.stream = st;
@@ -232,13 +236,6 @@ cudaError_t launch_lm_head(const uint4* codes, const float* scales, const float*
     return cudaLaunchKernelEx(&cfg, lm_head_kernel, p);
 }
 
-int lm_head_grid() {
-    if (g_sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
-    }
-    return g_sms;
-}
+int lm_head_grid() { return device_sms(); }
 
 }  // namespace focr

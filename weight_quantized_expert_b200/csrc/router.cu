@@ -22,6 +22,7 @@
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include "launch_state.h"
 
 namespace cg = cooperative_groups;
 
@@ -420,16 +421,17 @@ cudaError_t launch_router(const float* x, int T, int /*T_ws*/, const LayerView& 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    static bool configured = false;   // same shared-memory carveout as the expert kernels
-    if (!configured) {
+    // the same shared-memory carveout as the expert kernels
+    const cudaError_t e0 = once_per_device((const void*)router_kernel<1>, [] {
         for (const void* f : {(const void*)router_kernel<1>, (const void*)router_kernel<2>, (const void*)router_kernel<4>,
                               (const void*)router_kernel<8>}) {
             const cudaError_t e =
                 cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
             if (e != cudaSuccess) return e;
         }
-        configured = true;
-    }
+        return cudaSuccess;
+    });
+    if (e0 != cudaSuccess) return e0;
     switch (TB) {
         case 1: return cudaLaunchKernelEx(&cfg, router_kernel<1>, p);
         case 2: return cudaLaunchKernelEx(&cfg, router_kernel<2>, p);
