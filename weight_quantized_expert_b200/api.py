@@ -22,7 +22,7 @@ T_MAX = 8192
 W_BF16, W_INT8, W_INT4 = 0, 1, 2
 (MAT_GATE, MAT_UP, MAT_DOWN, MAT_SHARED_GATE, MAT_SHARED_UP, MAT_SHARED_DOWN, MAT_ROUTER) = range(7)
 STATUS = {0: "FOCR_OK", 1: "FOCR_ERR_INVALID_ARG", 2: "FOCR_ERR_UNSUPPORTED", 3: "FOCR_ERR_CUDA",
-          4: "FOCR_ERR_OOM", 5: "FOCR_ERR_TIMEOUT"}
+          4: "FOCR_ERR_OOM", 5: "FOCR_ERR_TIMEOUT", 6: "FOCR_ERR_RANGE"}
 
 # every symbol include/focr_moe.h declares
 EXPORTED = (

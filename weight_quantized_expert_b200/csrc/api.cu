@@ -585,6 +585,8 @@ focr_status focr_moe_check(void* workspace, void* stream) {
         const int32_t zero = 0;
         CUDA_TRY(cudaMemcpyAsync(ctrl + CTRL_ERROR, &zero, sizeof(zero), cudaMemcpyHostToDevice, st));
         CUDA_TRY(cudaStreamSynchronize(st));
+        if (v == DEVERR_RANGE)
+            return fail(FOCR_ERR_RANGE, "activations beyond the f16 operand range (|v| > 65504) met by a forward");
         return fail(FOCR_ERR_TIMEOUT, "device wait ran out (code %d)", v);
     }
     return FOCR_OK;

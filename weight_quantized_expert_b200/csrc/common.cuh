@@ -327,6 +327,10 @@ inline TcWork tc_work(void* ws, int T, int shared_inter) {
 }
 
 // error codes a kernel may store in the error word
+// activations outside the f16 operand range (finite |v| > 65504) met by a kernel; the
+// forward completes, and focr_moe_check reports FOCR_ERR_RANGE
+constexpr int DEVERR_RANGE = 8;
+__device__ __forceinline__ bool f16_out_of_range(float v) { return fabsf(v) > 65504.f && fabsf(v) <= 3.402823466e38f; }
 constexpr int DEVERR_FULL_WAIT = 1;
 constexpr int DEVERR_EMPTY_WAIT = 2;
 

@@ -64,7 +64,7 @@ __device__ __forceinline__ int abf_base(bool routed, int a) { return routed ? IS
 // and/or fp32 (xs, split into bf16 hi + lo at use by the bf16 sets).  All loads of a
 // thread are issued before its stores.
 template <int NT, bool F16, bool F32>
-__device__ __forceinline__ void build_x(const float* x, int T, uint2* xh, float4* xs) {
+__device__ __forceinline__ void build_x(const float* x, int T, uint2* xh, float4* xs, int* err) {
     constexpr int PER = (KSTEPS * 32 + NT - 1) / NT;
     float4 v[PER];
 #pragma unroll
@@ -83,7 +83,12 @@ __device__ __forceinline__ void build_x(const float* x, int T, uint2* xh, float4
     for (int k = 0; k < PER; ++k) {
         const int i = threadIdx.x + k * NT;
         if (i < KSTEPS * 32) {
-            if constexpr (F16) xh[i] = make_uint2(f32x2_to_f16x2(v[k].x, v[k].y), f32x2_to_f16x2(v[k].z, v[k].w));
+            if constexpr (F16) {
+                xh[i] = make_uint2(f32x2_to_f16x2(v[k].x, v[k].y), f32x2_to_f16x2(v[k].z, v[k].w));
+                if (f16_out_of_range(v[k].x) || f16_out_of_range(v[k].y) || f16_out_of_range(v[k].z) ||
+                    f16_out_of_range(v[k].w))
+                    atomicExch(err, DEVERR_RANGE);   // beyond the f16 operand range (reported, not fatal)
+            }
             if constexpr (F32) xs[i] = v[k];
         }
     }
@@ -224,6 +229,7 @@ __device__ __forceinline__ void store_a(const RouteView& R, bool routed, int a_s
             __half* a16 = reinterpret_cast<__half*>(R.a16);
             const int step = a16_base(routed, a_slot) + (ti >> 1);
             a16[((step * 32 + ln) * 2 + (ti & 1)) * 2 + (gr & 1)] = __float2half_rn(av[h]);
+            if (f16_out_of_range(av[h])) atomicExch(R.ctrl + CTRL_ERROR, DEVERR_RANGE);
         } else {
             __nv_bfloat16* abf = reinterpret_cast<__nv_bfloat16*>(R.abf);
             const int step = abf_base(routed, a_slot) + ti;
@@ -336,7 +342,7 @@ __global__ void __launch_bounds__(GuCfg<RW, SW, G>::NW * 32, 2) decode_gu_kernel
     __syncwarp();
     if (rho < s_units) gu_issue<SW, G>(p, false, -1, rho, buf, bar, lane, pol);
     build_x<C::NW * 32, C::F16, C::F32>(p.x, p.T, reinterpret_cast<uint2*>(smem + C::xh),
-                                         reinterpret_cast<float4*>(smem + C::xs));
+                                         reinterpret_cast<float4*>(smem + C::xs), p.R.ctrl + CTRL_ERROR);
     __syncthreads();
 
     uint32_t phase = 0;

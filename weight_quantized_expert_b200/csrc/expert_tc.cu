@@ -179,19 +179,34 @@ __device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b) {
     return d;
 }
 
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+constexpr uint32_t H2_MAGIC = 0x64006400u;    // f16 (1024, 1024): a nibble n under it reads as 1024 + n
+constexpr uint32_t H2_1032 = 0x64086408u;     // f16 (1032, 1032)
 constexpr uint32_t BF2_MAGIC = 0x43004300u;   // (128, 128): a nibble n under it reads as 128 + n
 constexpr uint32_t BF2_136 = 0x43084308u;     // (136, 136)
 
 // One k-core of int4 codes (element 2m in nibble m, 2m+1 in nibble m+4, q + 8) -> 8 bf16 q * s.
 // q = (128 + n) - 136 is exact in bf16; the product is rounded once (s2 = bf16 pair of the scale).
+template <bool F16>
 __device__ __forceinline__ void dq_int4_bf16(uint32_t w, uint32_t s2, uint32_t* r) {
-    r[0] = bf2_mul(bf2_sub((w & 0x000F000Fu) | BF2_MAGIC, BF2_136), s2);
-    r[1] = bf2_mul(bf2_sub(((w >> 4) & 0x000F000Fu) | BF2_MAGIC, BF2_136), s2);
-    r[2] = bf2_mul(bf2_sub(((w >> 8) & 0x000F000Fu) | BF2_MAGIC, BF2_136), s2);
-    r[3] = bf2_mul(bf2_sub(((w >> 12) & 0x000F000Fu) | BF2_MAGIC, BF2_136), s2);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t nib = (w >> (4 * i)) & 0x000F000Fu;
+        r[i] = F16 ? h2_mul(h2_sub(nib | H2_MAGIC, H2_1032), s2) : bf2_mul(bf2_sub(nib | BF2_MAGIC, BF2_136), s2);
+    }
 }
 
 // One k-core of int8 codes (q + 128 in bytes 0..7) -> 8 bf16 q * s (fp32 product, one rounding).
+template <bool F16>
 __device__ __forceinline__ void dq_int8_bf16(uint32_t w0, uint32_t w1, float s, uint32_t* r) {
     float f[8];
 #pragma unroll
@@ -200,50 +215,22 @@ __device__ __forceinline__ void dq_int8_bf16(uint32_t w0, uint32_t w1, float s, 
         f[4 + b] = (byte_to_float(w1, b) - 8388736.0f) * s;
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) r[m] = f32x2_to_bf16x2(f[2 * m], f[2 * m + 1]);
+    for (int m = 0; m < 4; ++m)
+        r[m] = F16 ? f32x2_to_f16x2(f[2 * m], f[2 * m + 1]) : f32x2_to_bf16x2(f[2 * m], f[2 * m + 1]);
 }
 
-// One row of a weight block into 32 registers (32-bit column c of the TMEM A stage = elements
-// 2c, 2c + 1 of the 64-wide K-block): thread = block row `row`.
-template <int W, int G>
-__device__ __forceinline__ void block_row(const uint8_t* blk, int row, uint32_t (&r)[32]) {
-    if constexpr (W == FOCR_W_BF16) {
-        // the operand image: k-core c of row r at [(r / 8) * 8 + c][r % 8] in 16-byte pieces
-        const uint8_t* base = blk + (row >> 3) * 1024 + (row & 7) * 16;
+// One row of a 16-bit weight block (stored as the operand image: k-core c of row r at
+// [(r / 8) * 8 + c][r % 8] in 16-byte pieces) into 32 registers: 32-bit column c of the TMEM A
+// stage holds elements 2c, 2c + 1 of the 64-wide K-block.  Thread = block row `row`.
+__device__ __forceinline__ void block_row_copy(const uint8_t* blk, int row, uint32_t (&r)[32]) {
+    const uint8_t* base = blk + (row >> 3) * 1024 + (row & 7) * 16;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint4 v = lds128(base + c * 128);
-            r[4 * c] = v.x;
-            r[4 * c + 1] = v.y;
-            r[4 * c + 2] = v.z;
-            r[4 * c + 3] = v.w;
-        }
-    } else {
-        constexpr int SPK = tc_spk(G);
-        constexpr uint32_t RB = tc_row_bytes(W);
-        const float* sc = reinterpret_cast<const float*>(blk + TC_M * RB) + row * SPK;
-        const float s0 = sc[0], s1 = sc[SPK - 1];   // k-cores 0-3, 4-7
-        if constexpr (W == FOCR_W_INT4) {
-            // pairs (c, c + 4), 8 bytes each: words k-core c, k-core c + 4
-            const uint4 p01 = lds128(blk + row * 32), p23 = lds128(blk + row * 32 + 16);
-            const uint32_t b0 = f32x2_to_bf16x2(s0, s0), b1 = SPK == 1 ? b0 : f32x2_to_bf16x2(s1, s1);
-            dq_int4_bf16(p01.x, b0, r + 0);
-            dq_int4_bf16(p01.y, b1, r + 16);
-            dq_int4_bf16(p01.z, b0, r + 4);
-            dq_int4_bf16(p01.w, b1, r + 20);
-            dq_int4_bf16(p23.x, b0, r + 8);
-            dq_int4_bf16(p23.y, b1, r + 24);
-            dq_int4_bf16(p23.z, b0, r + 12);
-            dq_int4_bf16(p23.w, b1, r + 28);
-        } else {
-            // pairs (c, c + 4), 16 bytes each
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint4 v = lds128(blk + row * 64 + c * 16);
-                dq_int8_bf16(v.x, v.y, s0, r + 4 * c);
-                dq_int8_bf16(v.z, v.w, s1, r + 4 * (c + 4));
-            }
-        }
+    for (int c = 0; c < 8; ++c) {
+        const uint4 v = lds128(base + c * 128);
+        r[4 * c] = v.x;
+        r[4 * c + 1] = v.y;
+        r[4 * c + 2] = v.z;
+        r[4 * c + 3] = v.w;
     }
 }
 
@@ -263,50 +250,56 @@ struct RowRaw {
         s0 = sc[0];
         s1 = sc[SPK - 1];
     }
+    // q * s in f16 (gate/up operands) or bf16 (down operands)
+    template <bool F16>
     __device__ __forceinline__ void cvt(uint32_t (&r)[32]) const {
         if constexpr (W == FOCR_W_INT4) {
             // pairs (c, c + 4), 8 bytes each: words k-core c, k-core c + 4
-            const uint32_t b0 = f32x2_to_bf16x2(s0, s0), b1 = tc_spk(G) == 1 ? b0 : f32x2_to_bf16x2(s1, s1);
-            dq_int4_bf16(c[0].x, b0, r + 0);
-            dq_int4_bf16(c[0].y, b1, r + 16);
-            dq_int4_bf16(c[0].z, b0, r + 4);
-            dq_int4_bf16(c[0].w, b1, r + 20);
-            dq_int4_bf16(c[1].x, b0, r + 8);
-            dq_int4_bf16(c[1].y, b1, r + 24);
-            dq_int4_bf16(c[1].z, b0, r + 12);
-            dq_int4_bf16(c[1].w, b1, r + 28);
+            const uint32_t b0 = F16 ? f32x2_to_f16x2(s0, s0) : f32x2_to_bf16x2(s0, s0);
+            const uint32_t b1 = tc_spk(G) == 1 ? b0 : (F16 ? f32x2_to_f16x2(s1, s1) : f32x2_to_bf16x2(s1, s1));
+            dq_int4_bf16<F16>(c[0].x, b0, r + 0);
+            dq_int4_bf16<F16>(c[0].y, b1, r + 16);
+            dq_int4_bf16<F16>(c[0].z, b0, r + 4);
+            dq_int4_bf16<F16>(c[0].w, b1, r + 20);
+            dq_int4_bf16<F16>(c[1].x, b0, r + 8);
+            dq_int4_bf16<F16>(c[1].y, b1, r + 24);
+            dq_int4_bf16<F16>(c[1].z, b0, r + 12);
+            dq_int4_bf16<F16>(c[1].w, b1, r + 28);
         } else {
             // pairs (c, c + 4), 16 bytes each
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                dq_int8_bf16(c[i].x, c[i].y, s0, r + 4 * i);
-                dq_int8_bf16(c[i].z, c[i].w, s1, r + 4 * (i + 4));
+                dq_int8_bf16<F16>(c[i].x, c[i].y, s0, r + 4 * i);
+                dq_int8_bf16<F16>(c[i].z, c[i].w, s1, r + 4 * (i + 4));
             }
         }
     }
 };
 
 // This thread's row of the `nb` (1 or 2) adjacent weight blocks at `bp` (`blk` bytes apart) into
-// the two 32-column halves of a TMEM A stage at `ta` (this warp's lane quarter).  Completes with
-// tcgen05.wait::st by the caller.
+// the two 32-column halves of a TMEM A stage at `ta` (this warp's lane quarter), as f16 for gate/up
+// units (`f16`) and bf16 for down units; 16-bit blocks are stored in the format their units use.
+// Completes with tcgen05.wait::st by the caller.
 template <int W, int G>
-__device__ __forceinline__ void dq_stage(const uint8_t* bp, uint32_t blk, int nb, int row, uint32_t ta) {
+__device__ __forceinline__ void dq_stage(const uint8_t* bp, uint32_t blk, int nb, int row, uint32_t ta, bool f16) {
     uint32_t r[32];
     if constexpr (W == FOCR_W_BF16) {
-        block_row<W, G>(bp, row, r);
+        block_row_copy(bp, row, r);
         umma::st32(ta, r);
         if (nb > 1) {
-            block_row<W, G>(bp + blk, row, r);
+            block_row_copy(bp + blk, row, r);
             umma::st32(ta + 32u, r);
         }
     } else {
         RowRaw<W, G> x0, x1;
         x0.load(bp, row);
         if (nb > 1) x1.load(bp + blk, row);
-        x0.cvt(r);
+        if (f16) x0.template cvt<true>(r);
+        else x0.template cvt<false>(r);
         umma::st32(ta, r);
         if (nb > 1) {
-            x1.cvt(r);
+            if (f16) x1.template cvt<true>(r);
+            else x1.template cvt<false>(r);
             umma::st32(ta + 32u, r);
         }
     }
@@ -833,7 +826,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                 }
                 umma::fence_after_sync();
                 const int N = Un.N, mt = Un.mt;
-                const uint32_t idesc = umma::idesc_bf16_f32(TC_M, N);
+                // gate/up: f16 weights and x; down: bf16 weights and a (range of the SwiGLU output)
+                const uint32_t idesc =
+                    Un.kind <= UK_GU_R ? umma::idesc_f16_f32(TC_M, N) : umma::idesc_bf16_f32(TC_M, N);
                 const uint32_t d0 = tmem_base + (uint32_t)(b * 128);
                 const int pp = stages_per_kb(mt), nst = Un.nkb * pp;
                 bool ok = true;
@@ -925,8 +920,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
                 const uint8_t* bp = reinterpret_cast<const uint8_t*>(smem + SL::braw + rs * SL::raw_slot) +
                                     (size_t)((kb % kq) * mt + t0) * blk;
                 const uint32_t ta = tmem_base + ((uint32_t)(32 * q) << 16) + TM_A0 + (uint32_t)(as * 64);
-                if (routed) dq_stage<RW, G>(bp, blk, nb, row, ta);
-                else dq_stage<SW, G>(bp, blk, nb, row, ta);
+                if (routed) dq_stage<RW, G>(bp, blk, nb, row, ta, kind <= UK_GU_R);
+                else dq_stage<SW, G>(bp, blk, nb, row, ta, kind <= UK_GU_R);
                 umma::wait_st();
                 umma::fence_before_sync();
                 __syncwarp();
@@ -1098,8 +1093,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) expert_tc_kernel(TcParams p) {
     }
 }
 
-// x (fp32) -> the bf16 operand image in token order (the dense layer has no router to write it)
-__global__ void x_image_kernel(const float* x, int T, int rows, uint16_t* img) {
+// x (fp32) -> the f16 operand image in token order (the dense layer has no router to write it);
+// a finite |x| beyond the f16 range sets the error word (DEVERR_RANGE)
+__global__ void x_image_kernel(const float* x, int T, int rows, uint16_t* img, int* err) {
     pdl_wait();
     pdl_launch_dependents();
     const int n = T * (H / 8);   // 16-byte pieces: 8 columns of one token
@@ -1107,9 +1103,12 @@ __global__ void x_image_kernel(const float* x, int T, int rows, uint16_t* img) {
         const int t = i / (H / 8), k = (i % (H / 8)) * 8;
         const float4 a = __ldg(reinterpret_cast<const float4*>(x + (size_t)t * H + k));
         const float4 b = __ldg(reinterpret_cast<const float4*>(x + (size_t)t * H + k + 4));
+        if (f16_out_of_range(a.x) || f16_out_of_range(a.y) || f16_out_of_range(a.z) || f16_out_of_range(a.w) ||
+            f16_out_of_range(b.x) || f16_out_of_range(b.y) || f16_out_of_range(b.z) || f16_out_of_range(b.w))
+            atomicExch(err, DEVERR_RANGE);
         reinterpret_cast<uint4*>(img)[img_index(rows, t, k) / 8] =
-            make_uint4(f32x2_to_bf16x2(a.x, a.y), f32x2_to_bf16x2(a.z, a.w), f32x2_to_bf16x2(b.x, b.y),
-                       f32x2_to_bf16x2(b.z, b.w));
+            make_uint4(f32x2_to_f16x2(a.x, a.y), f32x2_to_f16x2(a.z, a.w), f32x2_to_f16x2(b.x, b.y),
+                       f32x2_to_f16x2(b.z, b.w));
     }
 }
 
@@ -1151,7 +1150,7 @@ cudaError_t launch_expert_tc(const float* x, int T, const TcView& V, const Route
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, x_image_kernel, x, T, W.tpad, W.x_img);
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, x_image_kernel, x, T, W.tpad, W.x_img, R.ctrl + CTRL_ERROR);
         if (e != cudaSuccess) return e;
     }
     const TcParams p{x, T, out, resid ? 1 : 0, shared_only ? 1 : 0, V, R, W};

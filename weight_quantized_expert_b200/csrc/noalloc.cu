@@ -91,6 +91,13 @@ extern "C" focr_status focr_moe_check_noalloc(void* stream) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return report_error(FOCR_ERR_CUDA, cudaGetErrorString(e));
     if (v == 0) return FOCR_OK;
+    if (v == DEVERR_RANGE) {   // the forward completed; only the word is cleared
+        const int32_t zero = 0;
+        e = cudaMemcpyAsync(err, &zero, sizeof(zero), cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return report_error(FOCR_ERR_CUDA, cudaGetErrorString(e));
+        return report_error(FOCR_ERR_RANGE, "activations beyond the f16 operand range (|v| > 65504) met by a forward");
+    }
     // a wait ran out: the forward that set the word may have left counters and partial sums
     // behind, so the whole zero prefix (the error word included) is cleared
     e = cudaMemsetAsync(scratch, 0, kZeroBytes, st);

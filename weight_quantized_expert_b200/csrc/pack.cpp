@@ -129,9 +129,30 @@ namespace {
 
 // One block (128 rows x 64 input columns, K-block kb) of the tensor-core layout (common.cuh).
 // row_of(r) -> (matrix, row) of block row r.
+// f32 -> f16 bits, round to nearest even; finite values beyond the f16 range saturate to
+// +-65504 (no weight of a supported model comes near it), NaN stays NaN and +-inf stays inf.
+uint16_t host_f32_to_f16(float f) {
+    uint32_t x;
+    std::memcpy(&x, &f, 4);
+    const uint32_t sign = (x >> 16) & 0x8000u, ax = x & 0x7FFFFFFFu;
+    if (ax >= 0x7F800000u) return (uint16_t)(sign | (ax > 0x7F800000u ? 0x7E00u : 0x7C00u));
+    if (ax >= 0x477FF000u) return (uint16_t)(sign | 0x7BFFu);   // >= 65520 would round to inf
+    if (ax < 0x38800000u) {                                     // below 2^-14: a subnormal f16 (or zero)
+        float af;
+        std::memcpy(&af, &ax, 4);
+        return (uint16_t)(sign | (uint32_t)std::nearbyint(af * 16777216.0f));   // units of 2^-24
+    }
+    uint32_t h = ((((ax >> 23) - 127u + 15u) << 10) | ((ax & 0x7FFFFFu) >> 13));
+    const uint32_t rem = ax & 0x1FFFu;
+    if (rem > 0x1000u || (rem == 0x1000u && (h & 1u))) h += 1u;
+    return (uint16_t)(sign | h);
+}
+
+// One tensor-core block; 16-bit weights are written as bf16, or as f16 when `f16` (the gate/up
+// operands of the tensor-core kernel are f16).
 template <class RowOf>
 void tc_block(const Quantised* const* m3, const int64_t* cols3, const TcGeom& g, int kb, RowOf&& row_of,
-              uint8_t* blk) {
+              uint8_t* blk, bool f16) {
     const int wt = g.wtype;
     std::memset(blk, 0, g.blk);
     if (wt == FOCR_W_BF16) {
@@ -141,7 +162,13 @@ void tc_block(const Quantised* const* m3, const int64_t* cols3, const TcGeom& g,
             row_of(r, mat, row);
             const Quantised& m = *m3[mat];
             for (int k = 0; k < TC_KB; ++k) {
-                const uint16_t v = m.b[(size_t)(row * cols3[mat] + kb * TC_KB + k)];
+                uint16_t v = m.b[(size_t)(row * cols3[mat] + kb * TC_KB + k)];
+                if (f16) {
+                    const uint32_t u = (uint32_t)v << 16;
+                    float fv;
+                    std::memcpy(&fv, &u, 4);
+                    v = host_f32_to_f16(fv);
+                }
                 const size_t off = ((size_t)(r / 8) * 8 + k / 8) * 128 + (size_t)(r % 8) * 16 + (size_t)(k % 8) * 2;
                 std::memcpy(blk + off, &v, 2);
             }
@@ -190,7 +217,7 @@ void tc_pack(const Quantised& qg, const Quantised& qu, const Quantised& qd, cons
                          mat = (r >> 3) & 1;                      // rows 16 j + 8 h + r': h = 1 is up
                          row = (int64_t)TC_KB * p + 8 * (r >> 4) + (r & 7);
                      },
-                     gu + tc_block_index(g.tiles, TC_KBH, p, kb, g.grp) * g.blk);
+                     gu + tc_block_index(g.tiles, TC_KBH, p, kb, g.grp) * g.blk, true);
     for (int mt = 0; mt < TC_MT; ++mt)
         for (int kb = 0; kb < g.tiles; ++kb)
             tc_block(m3, cols3, g, kb,
@@ -198,7 +225,7 @@ void tc_pack(const Quantised& qg, const Quantised& qu, const Quantised& qd, cons
                          mat = 2;
                          row = (int64_t)TC_M * mt + r;
                      },
-                     dn + tc_block_index(TC_MT, g.tiles, mt, kb, g.grp) * g.blk);
+                     dn + tc_block_index(TC_MT, g.tiles, mt, kb, g.grp) * g.blk, false);
 }
 
 }  // namespace

@@ -29,9 +29,9 @@ namespace cg = cooperative_groups;
 namespace focr {
 namespace {
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     uint32_t d;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
     return d;
 }
 
@@ -221,22 +221,26 @@ __global__ void __cluster_dims__(RC, 1, 1) __launch_bounds__(RT_THREADS) router_
     pdl_wait();                 // x may come from the previous kernel on the stream
     pdl_launch_dependents();    // let the expert kernel start its routing-free work
 
+    bool out_of_range = false;   // a finite |x| the experts' f16 activation operands cannot hold
     for (int i = tid; i < TB * KCOLS; i += RT_THREADS) {
         const int t = i / KCOLS, c = i % KCOLS;
-        xs[t][c] = t < nt ? (double)p.x[(size_t)(t0 + t) * H + k0 + c] : 0.0;
+        const float v = t < nt ? p.x[(size_t)(t0 + t) * H + k0 + c] : 0.f;
+        out_of_range |= f16_out_of_range(v);
+        xs[t][c] = (double)v;
     }
+    if (out_of_range) atomicExch(&p.R.ctrl[CTRL_ERROR], DEVERR_RANGE);
     __syncthreads();
     if (p.x_img) {
-        // this CTA's 160 columns of its tokens, rounded to bf16 (the tensor-core path's B operand)
+        // this CTA's 160 columns of its tokens, rounded to f16 (the tensor-core path's gate/up operand)
         for (int i = tid; i < TB * (KCOLS / 8); i += RT_THREADS) {
             const int t = i / (KCOLS / 8), kc = i % (KCOLS / 8);
             if (t < nt) {
                 const double* v = &xs[t][kc * 8];
                 uint4 o;
-                o.x = pack_bf16x2((float)v[0], (float)v[1]);
-                o.y = pack_bf16x2((float)v[2], (float)v[3]);
-                o.z = pack_bf16x2((float)v[4], (float)v[5]);
-                o.w = pack_bf16x2((float)v[6], (float)v[7]);
+                o.x = pack_f16x2((float)v[0], (float)v[1]);
+                o.y = pack_f16x2((float)v[2], (float)v[3]);
+                o.z = pack_f16x2((float)v[4], (float)v[5]);
+                o.w = pack_f16x2((float)v[6], (float)v[7]);
                 *reinterpret_cast<uint4*>(p.x_img + img_index(p.img_rows, t0 + t, k0 + kc * 8)) = o;
             }
         }

@@ -16,6 +16,11 @@ namespace umma {
 // Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B, fp32 D, both operands K-major:
 // D format at bits 4-5 (1 = f32), A and B formats at 7-9 and 10-12 (1 = bf16), N >> 3 at bits 17-22,
 // M >> 4 at bits 24-28.
+// The same with f16 A and B (format 0).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
