@@ -80,8 +80,9 @@ def describe(name: str, world: int) -> dict:
 def precision(T: int):
     """(dtype, description) of the arithmetic the path runs for a batch of T tokens."""
     if T > 8:
-        return "bf16", ("tcgen05 MMAs with bf16 operands (int4/int8 weights dequantised to bf16 q*s, "
-                        "activations rounded to bf16), fp32 accumulation in TMEM; router fp64")
+        return "f16+bf16", ("tcgen05 MMAs: gate/up with f16 operands (x rounded to f16, weights dequantised to "
+                            "f16 q*s), down with bf16 operands (SwiGLU output and weights q*s rounded to bf16), "
+                            "fp32 accumulation in TMEM; router fp64")
     return "f16", ("mma.sync with f16 operands (int4/int8 codes exact, activations rounded to f16; bf16 "
                    "weights exact with bf16 hi+lo activations), fp32 accumulation; router fp64")
 

@@ -131,7 +131,7 @@ def test_dense_forward_matches_oracle(T):
     gr = api.focr_dense_mlp_forward(mlp, xd, flags=api.FWD_RESIDUAL)
     torch.cuda.synchronize()
     g, gr = g.cpu().numpy(), gr.cpu().numpy()
-    tol = 2e-3 if T <= 8 else 1e-2   # decode kernels / bf16 tensor-core path
+    tol = 2e-3 if T <= 8 else 1e-2   # decode kernels / tensor-core kernel (the dense layer takes it for T > 8)
     assert per_token_rel_err(g, r).max() <= tol
     # residual form: x + layer(x), against the oracle
     assert per_token_rel_err(gr - x, r).max() <= tol

@@ -1,8 +1,8 @@
 """Inputs with large-magnitude outlier channels (1e3 to 3e4 in a few hidden channels, the rest
 ~N(0, 1)) against the oracle.
 
-The tensor-core path (T > 8) takes x as f16 operands (finite up to 65504) and the SwiGLU
-output a as bf16, so such inputs keep their parity.  The small-batch kernels (T <= 8) take a
+The tensor-core path (T > 64) takes x as f16 operands (finite up to 65504) and the SwiGLU
+output a as bf16, so such inputs keep their parity.  The mma.sync kernels (T <= 64) take a
 as f16 as well; where an outlier drives |a| past 65504 the forward reports FOCR_ERR_RANGE
 through focr_moe_check instead of returning unflagged garbage.  A finite |x| above 65504 is
 reported the same way on both paths.
@@ -41,7 +41,7 @@ def _forward(packed, x):
 @pytest.mark.parametrize("magnitude", [1e3, 3e4])
 def test_tensor_core_path_keeps_parity_with_outlier_channels(magnitude):
     om, packed = moe_case(3, synth.W_INT4, synth.W_BF16, 64)
-    x = outlier_hidden(200 + int(magnitude) % 97, 33, magnitude)
+    x = outlier_hidden(200 + int(magnitude) % 97, 80, magnitude)
     r = om.forward(x, nthreads=NTHREADS)
     out, idx, ws = _forward(packed, x)
     api.focr_moe_check(ws)   # no range error: every |x| <= 65504
@@ -65,7 +65,7 @@ def test_small_batch_path_keeps_parity_or_reports_the_range(magnitude):
     assert per_token_rel_err(out.cpu().numpy(), r["out"]).max() <= 2e-3
 
 
-@pytest.mark.parametrize("T", [3, 33])
+@pytest.mark.parametrize("T", [3, 33, 80])
 def test_inputs_beyond_the_f16_range_are_reported(T):
     _, packed = moe_case(3, synth.W_INT4, synth.W_BF16, 64)
     x = synth.hidden(400 + T, T)

@@ -22,8 +22,8 @@ from weight_quantized_expert_b200 import api, synth
 
 pytestmark = pytest.mark.gpu
 NTHREADS = max(1, (os.cpu_count() or 1))
-TOL_DECODE = 2e-3   # T <= 8: f16 activations, fp32 accumulation
-TOL_TC = 1e-2       # T > 8: bf16 tensor-core operands, fp32 accumulation
+TOL_DECODE = 2e-3   # T <= 64: mma.sync kernels, f16 activations, fp32 accumulation
+TOL_TC = 1e-2       # T > 64: tensor-core kernel, f16 gate/up and bf16 down operands
 
 
 def _noalloc(packed, x):
@@ -49,7 +49,7 @@ def test_noalloc_chained_large_small_large_against_oracle(chain):
         np.testing.assert_array_equal(dbg["topk_idx"], r["idx"])
         np.testing.assert_array_equal(dbg["counts"], r["counts"])
         np.testing.assert_array_equal(dbg["perm"], r["perm"])
-        tol = TOL_DECODE if T <= 8 else TOL_TC
+        tol = TOL_DECODE if T <= 64 else TOL_TC
         assert per_token_rel_err(got, r["out"]).max() <= tol, (T, per_token_rel_err(got, r["out"]).max())
 
 
@@ -57,14 +57,14 @@ def test_noalloc_matches_the_regular_forward():
     # same kernels, same inputs: bit for bit where the kernels sum in a fixed order
     import torch
     _, packed = moe_case(1, synth.W_INT4, synth.W_BF16, 64)
-    for T in (7, 33):
+    for T in (7, 80):
         x = synth.hidden(61 + T, T)
         xd = torch.from_numpy(np.ascontiguousarray(x)).cuda()
         ref = api.focr_moe_layer_forward(packed, xd, workspace=api.new_workspace(T))
         got = api.focr_moe_layer_forward_noalloc(packed, xd)
         torch.cuda.synchronize()
         api.focr_moe_check_noalloc()
-        if T > 8:   # the tensor-core path sums in a fixed order
+        if T > 64:   # the tensor-core path sums in a fixed order
             np.testing.assert_array_equal(got.cpu().numpy(), ref.cpu().numpy())
         else:   # the small-batch kernels add their parts with fp32 atomics, in arrival order
             assert per_token_rel_err(got.cpu().numpy(), ref.cpu().numpy()).max() <= 1e-5

@@ -326,6 +326,9 @@ focr_status focr_moe_layer_forward_ex(const focr_moe_layer* L, const float* hidd
     if (T <= SMALL_T) {
         CUDA_TRY(launch_router(hidden, T, T, V, R, out, resid ? hidden : nullptr, nullptr, 0, st));
         CUDA_TRY(launch_decode_small(hidden, T, V, R, out, false, st));
+    } else if (T <= MID_T) {
+        CUDA_TRY(launch_router(hidden, T, T, V, R, out, resid ? hidden : nullptr, nullptr, 0, st));
+        CUDA_TRY(launch_expert_decode(hidden, T, V, R, out, false, st));
     } else {
         const TcWork W = tc_work(workspace, T, IS);
         CUDA_TRY(launch_router(hidden, T, T, V, R, nullptr, nullptr, W.x_img, W.tpad, st));

@@ -348,6 +348,12 @@ cudaError_t launch_expert_tc(const float* x, int T, const TcView& V, const Route
                              float* out, bool resid, bool shared_only, cudaStream_t st);
 // T <= SMALL_T: gate/up + swiglu kernel, then the down kernel (decode_small.cu)
 constexpr int SMALL_T = 8;
+// SMALL_T < T <= MID_T: the grouped mma.sync kernel (expert_decode.cu), behind the router's own
+// dispatch; larger batches take the tensor-core kernel (expert_tc.cu), which measured slower than
+// it up to 64 tokens (batch 32: 164 vs 122 us; batch 64: 180 vs 171 us)
+constexpr int MID_T = 64;
+cudaError_t launch_expert_decode(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
+                                 bool shared_only, cudaStream_t st);
 cudaError_t launch_decode_small(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
                                 bool shared_only, cudaStream_t st);
 
