@@ -1,5 +1,5 @@
-// Tensor-core grouped expert kernel for batches of more than 8 tokens (batched decode,
-// prefill): the shared expert and every selected routed expert as tcgen05 GEMMs with the
+// Tensor-core grouped expert kernel for batches of more than MID_T tokens (prefill; the dense
+// layer for more than 8): the shared expert and every selected routed expert as tcgen05 GEMMs with the
 // dequantised weights and the accumulators in tensor memory, SwiGLU fused into the gate/up
 // epilogue, and a combine that sums each token's parts in a fixed order (no atomics on the
 // output, so repeated calls are bit-identical).
@@ -17,15 +17,21 @@
 //                 K = 1280 (block rows interleave gate and up by 8, see the tensor-core layout in
 //                 common.cuh); the epilogue pairs each gate lane with its up lane (shuffle by 8)
 //                 and writes a = silu(g) * u * w_route as bf16 into the "a image"
+//                 (x arrives as an f16 image: the router writes it in token order, the prologue
+//                 copies each expert's rows into dispatch order)
 //   down unit     (set, MT m-tiles of 128 output rows, [K part,] token chunk): D_t = Down_t a^T over
 //                 the set's intermediates (the shared set's in up to 8 K parts); the epilogue
 //                 writes fp32 rows y per (token, slot) or per (token, part)
 //   dispatch      (prologue of every CTA, epilogue warps): a share of the token -> expert entries
 //                 placed in their experts' segments (perm) and their x rows copied into an operand image
 //   combine       out[t] = resid + sum_parts y_shared + sum_{j<6} y_slot[t*6+j]
-// Units are handed out by a global atomic counter (gathers, shared gate/up, routed gate/up, shared
-// down, routed down), so a unit only ever waits on units with smaller numbers, which running CTAs
-// hold: a unit's token-row loads wait (bounded) until the units that write those rows are done.
+// Units are handed out by a global atomic counter (shared gate/up, routed gate/up, shared down,
+// routed down), so a unit only ever waits on units with smaller numbers, which running CTAs hold,
+// or on the prologue, which every CTA runs first: a unit's token-row loads wait (bounded) until
+// the units (or dispatch entries) that write those rows are done.
+//
+// Operand types: gate/up MMAs take f16 (x rounded to f16, weights q * s formed in f16), down MMAs
+// bf16 (the SwiGLU output a and q * s rounded to bf16, for a's range); accumulation is fp32.
 //
 // Warp roles (one CTA per SM, 640 threads):
 //   warp 0       scheduler: takes units, publishes their descriptors
@@ -39,8 +45,8 @@
 //   warp 3       token-row loader: one bulk copy per K-block of N rows of an operand image
 //   warps 4-15   dequantisers, three groups of four (one warp per TMEM lane quarter): thread = one
 //                of the block's 128 rows; int4 (exponent-bias method) or int8 codes times the group
-//                scale, rounded to bf16 (q * s), written to a TMEM A stage with tcgen05.st;
-//                bf16 blocks are moved to TMEM as they are
+//                scale (q * s in f16 for gate/up, bf16 for down), written to a TMEM A stage with
+//                tcgen05.st; 16-bit blocks are stored in their units' type and moved as they are
 //   warps 16-19  epilogue: tcgen05.ld of the accumulators, SwiGLU or output rows, completion
 //                counts; first the prologue share of the dispatch
 // Every wait is bounded in time (%globaltimer); on expiry the kernel records an error word,
