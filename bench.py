@@ -474,6 +474,10 @@ def run_step_workload(args, rank, world, local_rank):
         for i in range(args.warmup):
             run(xs[i % pool_n], stream)
     stream.synchronize()
+    if kind == "stack":   # a device error in the warm-up ends the run before the timed steps
+        api.focr_moe_check(step_ws[256:], stream)
+    elif kind == "dense":
+        api.focr_moe_check(ws, stream)
     K = args.steps
     graphs, _ = capture_graphs(lambda i, st: run(xs[i % pool_n], st), K, stream)
     ms, clk = timed_replay(graphs, stream, world, dev, local_rank)
@@ -568,6 +572,7 @@ def run_ours(args, rank, world, local_rank):
         for i in range(args.warmup):
             step(i, stream)
     stream.synchronize()
+    api.focr_moe_check(ws, stream)   # a device error in the warm-up ends the run before the timed steps
     K = args.steps
     if args.eager:
         clocks = Clocks(local_rank)
