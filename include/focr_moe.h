@@ -181,7 +181,7 @@ focr_status focr_moe_layer_forward(const focr_moe_layer* layer, const float* hid
  *     returns before the GPU runs it): focr_moe_check_noalloc reports it.
  */
 #define FOCR_NOALLOC_T_MAX 320
-#define FOCR_NOALLOC_SCRATCH_BYTES 38216960
+#define FOCR_NOALLOC_SCRATCH_BYTES 50665216
 focr_status focr_moe_layer_forward_noalloc(const focr_moe_layer* layer, const float* hidden, int32_t T, float* out,
                                            const focr_moe_route_debug* dbg, void* stream);
 
@@ -196,6 +196,10 @@ focr_status focr_moe_check_noalloc(void* stream);
 
 /* Flags of the *_ex / dense forwards. */
 #define FOCR_FWD_RESIDUAL 1   /* out = hidden + layer(hidden) instead of layer(hidden) */
+/* Bit-identical results for identical calls on every path: T <= 8 then sums its parts as 64-bit
+ * fixed-point integers (each part rounded once to a multiple of 2^-32) instead of fp32 atomics.
+ * The tensor-core path (T > 64) always sums in a fixed order; 9 <= T <= 64 is not covered. */
+#define FOCR_FWD_DETERMINISTIC 2
 
 /*
  * focr_moe_layer_forward_ex -- focr_moe_layer_forward with flags (0 or FOCR_FWD_RESIDUAL).

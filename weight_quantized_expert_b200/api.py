@@ -36,6 +36,7 @@ EXPORTED = (
     "focr_decode_step_workspace_bytes", "focr_decode_step",
 )
 FWD_RESIDUAL = 1
+FWD_DETERMINISTIC = 2
 NOALLOC_T_MAX = 320
 
 

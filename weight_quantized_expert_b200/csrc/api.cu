@@ -299,14 +299,14 @@ size_t focr_moe_workspace_bytes(int32_t T_max) {
     return a > b ? a : b;
 }
 
-size_t focr_moe_workspace_zero_bytes(void) { return ws_layout(1).a16; }
+size_t focr_moe_workspace_zero_bytes(void) { return ws_layout(1).gpart; }
 
 focr_status focr_moe_layer_forward_ex(const focr_moe_layer* L, const float* hidden, int32_t T, float* out,
                                       void* workspace, size_t ws_bytes, const focr_moe_route_debug* dbg, int32_t flags,
                                       void* stream) {
     g_err.clear();
     if (!L || !L->dev) return fail(FOCR_ERR_INVALID_ARG, "layer is NULL");
-    if (flags & ~FOCR_FWD_RESIDUAL) return fail(FOCR_ERR_INVALID_ARG, "unknown flags 0x%x", (unsigned)flags);
+    if (flags & ~(FOCR_FWD_RESIDUAL | FOCR_FWD_DETERMINISTIC)) return fail(FOCR_ERR_INVALID_ARG, "unknown flags 0x%x", (unsigned)flags);
     if (T < 1 || T > FOCR_T_MAX) return fail(FOCR_ERR_INVALID_ARG, "T=%d outside [1, %d]", T, FOCR_T_MAX);
     if (!hidden || !out || !workspace) return fail(FOCR_ERR_INVALID_ARG, "hidden, out and workspace must not be NULL");
     if (!aligned(hidden, 16) || !aligned(out, 16)) return fail(FOCR_ERR_INVALID_ARG, "hidden/out must be 16-byte aligned");
@@ -325,7 +325,7 @@ focr_status focr_moe_layer_forward_ex(const focr_moe_layer* L, const float* hidd
     const bool resid = (flags & FOCR_FWD_RESIDUAL) != 0;
     if (T <= SMALL_T) {
         CUDA_TRY(launch_router(hidden, T, T, V, R, out, resid ? hidden : nullptr, nullptr, 0, st));
-        CUDA_TRY(launch_decode_small(hidden, T, V, R, out, false, st));
+        CUDA_TRY(launch_decode_small(hidden, T, V, R, out, false, (flags & FOCR_FWD_DETERMINISTIC) != 0, st));
     } else if (T <= MID_T) {
         CUDA_TRY(launch_router(hidden, T, T, V, R, out, resid ? hidden : nullptr, nullptr, 0, st));
         CUDA_TRY(launch_expert_decode(hidden, T, V, R, out, false, st));
@@ -541,7 +541,7 @@ focr_status focr_dense_mlp_forward(const focr_dense_mlp* M, const float* x, int3
                                    size_t ws_bytes, int32_t flags, void* stream) {
     g_err.clear();
     if (!M || !M->dev) return fail(FOCR_ERR_INVALID_ARG, "dense MLP is NULL");
-    if (flags & ~FOCR_FWD_RESIDUAL) return fail(FOCR_ERR_INVALID_ARG, "unknown flags 0x%x", (unsigned)flags);
+    if (flags & ~(FOCR_FWD_RESIDUAL | FOCR_FWD_DETERMINISTIC)) return fail(FOCR_ERR_INVALID_ARG, "unknown flags 0x%x", (unsigned)flags);
     if (T < 1 || T > FOCR_T_MAX) return fail(FOCR_ERR_INVALID_ARG, "T=%d outside [1, %d]", T, FOCR_T_MAX);
     if (!x || !out || !workspace) return fail(FOCR_ERR_INVALID_ARG, "x, out and workspace must not be NULL");
     if (!aligned(x, 16) || !aligned(out, 16) || !aligned(workspace, 256))
@@ -565,7 +565,8 @@ focr_status focr_dense_mlp_forward(const focr_dense_mlp* M, const float* x, int3
         v.routed_dscale = v.shared_dscale;
         v.rg = M->g;
         v.sg = M->g;
-        CUDA_TRY(launch_decode_small(x, T, v, route_view(workspace, T, IS_MAX), out, true, st));
+        CUDA_TRY(launch_decode_small(x, T, v, route_view(workspace, T, IS_MAX), out, true,
+                                     (flags & FOCR_FWD_DETERMINISTIC) != 0, st));
     } else {
         TcView v{};
         v.s = TcSetView{M->dev + M->off_tc_gu, M->dev + M->off_tc_dn, M->tg};

@@ -189,9 +189,12 @@ struct WsLayout {
     // regions that are zero on entry and that every forward leaves zero; their offsets do
     // not depend on T_max, so calls with different T may share one workspace
     size_t ctrl;          // int32 [MAX_TB tickets][1 global ticket][1 error word][pad][CTRL_TC_WORDS]
-    size_t gacc;          // f32 [GU_TILES][32 lanes][4]  gate/up sums of k-split tiles (T <= 8)
-    size_t tcnt;          // i32 [GU_TILES]               their arrival counters
+    size_t tcnt;          // i32 [GU_TILES]               arrival counters of the k-split gate/up tiles (T <= 8)
+    size_t dacc;          // i64 [8][1280]                the down projections' output sums (T <= 8), fixed point
+    size_t dflag;         // i32 [8][1280]                1: a non-finite or out-of-range part
+    size_t dcnt;          // i32 [80]                     units finished per 16-row output tile
     // regions every forward writes before reading
+    size_t gpart;         // f32 [GU_TILES][4 parts][32][4]  the k-split gate/up tiles' part sums (T <= 8)
     size_t a16;           // uint2 [A16_STEPS][32]   f16 a fragments (int4 / int8 down, T <= 8)
     size_t abf;           // uint2 [ABF_STEPS][32]   bf16 a hi, lo fragments (bf16 down, T <= 8)
     size_t logits;        // f32 [T_max][64]
@@ -237,8 +240,11 @@ constexpr WsLayout ws_layout(int T_max, int shared_inter = IS) {
     WsLayout w{};
     size_t o = 0;
     w.ctrl = o;      o = align_up(o + sizeof(int32_t) * (MAX_TB + 256), 256);
-    w.gacc = o;      o = align_up(o + sizeof(float) * 4 * 32 * (size_t)GU_TILES, 256);
     w.tcnt = o;      o = align_up(o + sizeof(int32_t) * (size_t)GU_TILES, 256);
+    w.dacc = o;      o = align_up(o + sizeof(int64_t) * 8 * H, 256);
+    w.dflag = o;     o = align_up(o + sizeof(int32_t) * 8 * H, 256);
+    w.dcnt = o;      o = align_up(o + sizeof(int32_t) * (H / 16), 256);
+    w.gpart = o;     o = align_up(o + sizeof(float) * 4 * 4 * 32 * (size_t)GU_TILES, 256);
     w.a16 = o;       o = align_up(o + 8 * 32 * (size_t)A16_STEPS, 256);
     w.abf = o;       o = align_up(o + 8 * 32 * (size_t)ABF_STEPS, 256);
     w.logits = o;    o = align_up(o + sizeof(float) * (size_t)T_max * E, 256);
@@ -284,8 +290,11 @@ struct RouteView {   // device pointers into the workspace
     int32_t* offsets;
     int32_t* active;
     int32_t* perm;
-    float* gacc;
     int32_t* tcnt;
+    unsigned long long* dacc;
+    int32_t* dflag;
+    int32_t* dcnt;
+    float* gpart;
     uint2* a16;
     uint2* abf;
 };
@@ -296,7 +305,8 @@ inline RouteView route_view(void* ws, int T_max, int shared_inter = IS) {
     return RouteView{(int32_t*)(b + L.ctrl), (float*)(b + L.logits),
                      (int32_t*)(b + L.topk_idx), (float*)(b + L.topk_w), (int32_t*)(b + L.counts),
                      (int32_t*)(b + L.offsets), (int32_t*)(b + L.active), (int32_t*)(b + L.perm),
-                     (float*)(b + L.gacc), (int32_t*)(b + L.tcnt), (uint2*)(b + L.a16), (uint2*)(b + L.abf)};
+                     (int32_t*)(b + L.tcnt), (unsigned long long*)(b + L.dacc), (int32_t*)(b + L.dflag),
+                     (int32_t*)(b + L.dcnt), (float*)(b + L.gpart), (uint2*)(b + L.a16), (uint2*)(b + L.abf)};
 }
 
 // workspace regions of the tensor-core grouped path
@@ -355,7 +365,7 @@ constexpr int MID_T = 64;
 cudaError_t launch_expert_decode(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
                                  bool shared_only, cudaStream_t st);
 cudaError_t launch_decode_small(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
-                                bool shared_only, cudaStream_t st);
+                                bool shared_only, bool deterministic, cudaStream_t st);
 
 }  // namespace focr
 
@@ -492,6 +502,21 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 // Named barrier over `count` threads (id != 0).
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Fixed-point accumulation, for sums whose value must not depend on the order in which their
+// parts arrive: each part is rounded once to a multiple of 2^-32 (|part| < 2^30), the parts add
+// exactly as 64-bit integers (any order gives the same total), and the total converts back to
+// fp32 once.  A part that is not finite or out of that range is recorded by the caller in a flag
+// instead, and the total then reads as NaN.
+constexpr double FX_ONE = 4294967296.0;   // 2^32
+__device__ __forceinline__ bool fx_ok(float v) { return fabsf(v) < 1073741824.f; }   // false for NaN / inf
+__device__ __forceinline__ unsigned long long fx_of(float v) {
+    return (unsigned long long)__double2ll_rn((double)v * FX_ONE);
+}
+__device__ __forceinline__ float fx_to_float(unsigned long long a) { return (float)((double)(long long)a * (1.0 / FX_ONE)); }
+__device__ __forceinline__ void red_add_u64(unsigned long long* addr, unsigned long long v) {
+    asm volatile("red.global.add.u64 [%0], %1;" ::"l"(addr), "l"(v) : "memory");
 }
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {

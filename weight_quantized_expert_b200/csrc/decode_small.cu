@@ -16,9 +16,9 @@
 //   bulk-copies a unit into its own shared-memory buffer (cp.async.bulk, own mbarrier,
 //   bounded wait), turns int4/int8 codes into exact f16 A fragments (bf16 weights enter
 //   bf16 MMAs with x split into hi + lo), scales each group's fp32 sum, and applies
-//   a = silu(g) * u * w_route to whole rows; tiles split along K add their partial sums into
-//   the workspace with vector atomics and the warp that completes a tile (arrival counter)
-//   applies it and clears the sums.  a goes to the workspace as the down projection's B
+//   a = silu(g) * u * w_route to whole rows; tiles split along K write each part's sums to
+//   its own workspace slot, and the warp that completes a tile (arrival counter) adds the
+//   parts in a fixed order and applies it.  a goes to the workspace as the down projection's B
 //   fragments.  Shared-set units run while the router is still working, routed units after
 //   griddepcontrol.wait; the first unit of every slice prefetches the slice's
 //   down-projection bytes into L2.
@@ -26,8 +26,9 @@
 //   over a chunk of 8-16 slices.  The 8 warps of a CTA take 8 tiles of one chunk; each
 //   loads its codes and scales (the first step before waiting on decode_gu), one bulk copy
 //   stages the chunk's B fragments of a in shared memory for all of them, and y = D a is
-//   scaled per row and group and added into the output with atomics (the router initialised
-//   it).
+//   scaled per row and group and added into fixed-point sums per output element; the unit that
+//   completes a 16-row tile (arrival counter) adds the tile's totals to the output the router
+//   initialised, once, and clears them.  So repeated calls give bit-identical outputs.
 //
 // Precision: int4/int8 codes exact in f16 with fp32 group scales and f16 activations; bf16
 // weights exact with bf16 hi + lo activations; fp32 accumulation throughout.
@@ -51,6 +52,7 @@ struct SmallParams {
     LayerView L;
     RouteView R;
     int shared_only;
+    int deterministic;   // fixed-point output sums (bit-identical repeats) instead of fp32 atomics
 };
 
 // Workspace indexing (shared set first, then the routed experts' active slots a = 0..U-1):
@@ -299,20 +301,28 @@ __device__ __forceinline__ bool gu_finish(const SmallParams& p, bool routed, int
     if constexpr (U::KP == 1) {
         store_a<W>(p.R, routed, a_slot, ti, lane, tot, wr);
     } else {
+        // each part's sums go to their own slot; the warp that completes the tile adds the parts in
+        // a fixed order, so the total does not depend on the order they arrive in
         const int tile = gu_tile_base(routed, a_slot) + ti;
-        float* ga = p.R.gacc + ((size_t)tile * 32 + lane) * 4;
-        red_add_v4(ga, tot[0], tot[1], tot[2], tot[3]);
+        float4* gp = reinterpret_cast<float4*>(p.R.gpart) + ((size_t)tile * 4) * 32 + lane;
+        __stcg(gp + part * 32, make_float4(tot[0], tot[1], tot[2], tot[3]));
         __threadfence();
         __syncwarp();
         int old = 0;
         if (lane == 0) old = atomicAdd(&p.R.tcnt[tile], 1);
         old = __shfl_sync(0xffffffffu, old, 0);
-        if (old == U::KP - 1) {   // the other parts' sums are in: apply and clear
+        if (old == U::KP - 1) {   // the other parts' sums are in: apply
             __threadfence();
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(ga));
-            __stcg(reinterpret_cast<float4*>(ga), make_float4(0.f, 0.f, 0.f, 0.f));
+            float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int q = 0; q < U::KP; ++q) {
+                const float4 v = __ldcg(gp + q * 32);
+                sum[0] += v.x;
+                sum[1] += v.y;
+                sum[2] += v.z;
+                sum[3] += v.w;
+            }
             if (lane == 0) p.R.tcnt[tile] = 0;
-            const float sum[4] = {v.x, v.y, v.z, v.w};
             store_a<W>(p.R, routed, a_slot, ti, lane, sum, wr);
         }
     }
@@ -414,7 +424,7 @@ __device__ __forceinline__ void down_load(const uint8_t* items, const ItemGeom& 
 // the group scales, and the atomic adds into the output rows 16m .. 16m+15
 template <int W, int G>
 __device__ __forceinline__ void down_finish(const DownA<W, G>& A, const uint2* bsm, int m, int T, float* out,
-                                            int lane) {
+                                            const RouteView& R, bool det, int lane) {
     using D = DownUnit<W, G>;
     constexpr int CH = D::CH;
     const int gr = lane >> 2, c = lane & 3;
@@ -456,15 +466,33 @@ __device__ __forceinline__ void down_finish(const DownA<W, G>& A, const uint2* b
 #pragma unroll
         for (int r = 0; r < 4; ++r) y[r] = acc[0][r] + acc[1][r];
     }
+    // deterministic: into the fixed-point sums of tile m (any arrival order gives the same totals),
+    // counted against the tile after the warp's last unit; otherwise fp32 atomics into the output
     const int row = 16 * m + gr;
-    if (2 * c < T) {
-        atomicAdd(out + (size_t)(2 * c) * H + row, y[0]);
-        atomicAdd(out + (size_t)(2 * c) * H + row + 8, y[2]);
+    const int tok[4] = {2 * c, 2 * c + 1, 2 * c, 2 * c + 1}, rr[4] = {row, row, row + 8, row + 8};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (tok[i] >= T) continue;
+        const size_t idx = (size_t)tok[i] * H + rr[i];
+        if (!det) atomicAdd(out + idx, y[i]);
+        else if (fx_ok(y[i])) red_add_u64(R.dacc + idx, fx_of(y[i]));
+        else R.dflag[idx] = 1;
     }
-    if (2 * c + 1 < T) {
-        atomicAdd(out + (size_t)(2 * c + 1) * H + row, y[1]);
-        atomicAdd(out + (size_t)(2 * c + 1) * H + row + 8, y[3]);
+}
+
+// The warp that completes 16-row tile m adds the tile's fixed-point totals to the output the
+// router initialised, once, and clears them.
+__device__ __forceinline__ void down_convert(const RouteView& R, float* out, int T, int m, int lane) {
+    __threadfence();
+    for (int i = lane; i < 16 * T; i += 32) {
+        const size_t idx = (size_t)(i >> 4) * H + 16 * m + (i & 15);
+        const unsigned long long a = __ldcg(R.dacc + idx);
+        const int f = __ldcg(R.dflag + idx);
+        out[idx] += f ? __int_as_float(0x7fc00000) : fx_to_float(a);
+        R.dacc[idx] = 0ull;
+        if (f) R.dflag[idx] = 0;
     }
+    if (lane == 0) R.dcnt[m] = 0;
 }
 
 // One step of a CTA: its 8 warps take 8 consecutive output tiles of one chunk of one set.
@@ -494,7 +522,7 @@ __device__ __forceinline__ bool down_step(const SmallParams& p, const uint8_t* i
         (void)mbar_wait_bounded(bar, phase ^ 1u, WAIT_LIMIT_NS);   // never leave the copy in flight
         return false;
     }
-    down_finish<W, G>(A, bsm, m, p.T, p.out, lane);
+    down_finish<W, G>(A, bsm, m, p.T, p.out, p.R, p.deterministic != 0, lane);
     return true;
 }
 
@@ -522,7 +550,9 @@ __global__ void __launch_bounds__(DN_WARPS * 32, 2) decode_down_kernel(SmallPara
     const int nch_r = (p.L.rg.slices + DR::CH - 1) / DR::CH;
     const int n_s = OTILES * nch_s;
     const int per_expert = OTILES * nch_r;
-    const int total = n_s + (p.shared_only ? 0 : __ldcg(&p.R.active[E]) * per_expert);
+    const int n_act = p.shared_only ? 0 : __ldcg(&p.R.active[E]);
+    const int total = n_s + n_act * per_expert;
+    const int tile_units = nch_s + n_act * nch_r;   // units adding into each 16-row output tile
     const uint2* bs = is_quant(SW) ? p.R.a16 : p.R.abf;
     const uint2* br = is_quant(RW) ? p.R.a16 : p.R.abf;
     uint32_t phase = 0;
@@ -543,6 +573,28 @@ __global__ void __launch_bounds__(DN_WARPS * 32, 2) decode_down_kernel(SmallPara
                                   rem / OTILES, rem % OTILES, first, bsm, &bar, phase, lane);
         }
         first = false;
+    }
+    if (ok && p.deterministic) {
+        // a warp's units are counted against their tiles once, after all of them: one fence, then
+        // one counter increment per unit with the units spread over the lanes
+        __syncwarp();
+        __threadfence();   // this warp's sums are visible before its units are counted
+        const int nunits = total > blockIdx.x * DN_WARPS ? (total - blockIdx.x * DN_WARPS + nwt - 1) / nwt : 0;
+        for (int j0 = 0; j0 < nunits; j0 += 32) {
+            const int j = j0 + lane;
+            int m = -1;
+            bool done = false;
+            if (j < nunits) {
+                m = (blockIdx.x * DN_WARPS + j * nwt + warp) % OTILES;
+                done = atomicAdd(&p.R.dcnt[m], 1) == tile_units - 1;
+            }
+            unsigned mask = __ballot_sync(0xffffffffu, done);
+            while (mask) {
+                const int src = __ffs(mask) - 1;
+                mask &= mask - 1;
+                down_convert(p.R, p.out, p.T, __shfl_sync(0xffffffffu, m, src), lane);
+            }
+        }
     }
     if (first) pdl_wait();   // every CTA waits before exiting (keeps the chain of forwards ordered)
 }
@@ -584,11 +636,11 @@ cudaError_t launch_small_typed(const SmallParams& p, int sms, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_decode_small(const float* x, int T, const LayerView& L, const RouteView& R, float* out,
-                                bool shared_only, cudaStream_t st) {
+                                bool shared_only, bool deterministic, cudaStream_t st) {
     if (T < 1 || T > 8 || L.sg.inter > IS_MAX || L.sg.inter % 8 != 0) return cudaErrorInvalidValue;
     const int sms = device_sms();
     if (sms <= 0) return cudaErrorInvalidDevice;
-    const SmallParams p{x, T, out, L, R, shared_only ? 1 : 0};
+    const SmallParams p{x, T, out, L, R, shared_only ? 1 : 0, deterministic ? 1 : 0};
     const int rw = L.rg.wtype, sw = L.sg.wtype;
     const int g = is_quant(rw) ? L.rg.group : (is_quant(sw) ? L.sg.group : 128);
 #define FOCR_CASE(A, B, GG) \

@@ -29,7 +29,7 @@ constexpr WsLayout kNoallocLayout = ws_layout(FOCR_NOALLOC_T_MAX, IS);
 static_assert(kNoallocLayout.total == FOCR_NOALLOC_SCRATCH_BYTES, "header constant out of date");
 // control words, k-split partial sums and their counters: zero before the first forward and
 // left zero by every forward that completes
-constexpr size_t kZeroBytes = kNoallocLayout.a16;
+constexpr size_t kZeroBytes = kNoallocLayout.gpart;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FOCR_NOALLOC_SCRATCH_BYTES];
 
