@@ -90,11 +90,13 @@ def lib():
             L.orc_dense_mlp.argtypes = [ctypes.POINTER(Mat)] * 3 + [P, ctypes.c_int, P, ctypes.c_int]
             L.orc_rmsnorm.argtypes = [P, ctypes.c_int, ctypes.c_int, P, dbl, P]
             L.orc_lm_head.argtypes = [P, P, P, ctypes.c_int, i64, ctypes.c_int, P, P, ctypes.c_int]
+            L.orc_w8a8_quantize_x.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P]
+            L.orc_w8a8_gemv.argtypes = [P, P, i64, ctypes.c_int, P, P, ctypes.c_int, P, P]
             L.orc_max_threads.restype = ctypes.c_int
             for name in ("orc_round_bf16_array", "orc_quantize_rows", "orc_nibble_pack",
                          "orc_nibble_unpack", "orc_gemv", "orc_swiglu", "orc_router_logits",
                          "orc_softmax_topk", "orc_dispatch", "orc_moe_forward", "orc_dense_mlp",
-                         "orc_rmsnorm", "orc_lm_head"):
+                         "orc_rmsnorm", "orc_lm_head", "orc_w8a8_quantize_x", "orc_w8a8_gemv"):
                 getattr(L, name).restype = None
             _lib = L
     return _lib
@@ -317,6 +319,34 @@ class OracleLMHead:
         am = np.empty(T, np.int32)
         lib().orc_lm_head(_p(self.q), _p(self.s), _p(x), T, self.V, self.H, _p(logits), _p(am), nthreads)
         return am, logits
+
+
+def w8a8_quantize_x(x):
+    """Per-token int8 activations and their fp32 scales ([P4-cpu] quantise-plus-GEMV)."""
+    x = _c(x, np.float32)
+    T, K = x.shape
+    qx = np.empty((T, K), np.int8)
+    sx = np.empty(T, np.float32)
+    lib().orc_w8a8_quantize_x(_p(x), T, K, _p(qx), _p(sx))
+    return qx, sx
+
+
+class OracleW8A8:
+    """An int8 weight matrix with one scale per row, applied to per-token int8 activations."""
+
+    def __init__(self, w):
+        w = _c(w, np.float32)
+        self.N, self.K = w.shape
+        q, s = quantize_rows(w, self.K, 8)
+        self.q, self.s = q, np.ascontiguousarray(s[:, 0])
+
+    def forward(self, x, want_acc: bool = False):
+        qx, sx = w8a8_quantize_x(x)
+        T = qx.shape[0]
+        y = np.empty((T, self.N), np.float32)
+        acc = np.empty((T, self.N), np.int64) if want_acc else None
+        lib().orc_w8a8_gemv(_p(self.q), _p(self.s), self.N, self.K, _p(qx), _p(sx), T, _p(y), _p(acc))
+        return (y, qx, sx, acc) if want_acc else (y, qx, sx)
 
 
 def max_threads() -> int:

@@ -20,6 +20,12 @@
  *             top-6, MoE intermediate 896, vocab 129280).
  *   [P4-arch] franken_ocr README, "Architecture" (each expert 1280 -> 896
  *             SiLU-gated, 2 always-on shared experts, final RMSNorm, lm_head).
+ *   [P4-cpu]  franken_ocr README, "CPU Backend and Optimizations" (int8 decode
+ *             linears as a quantise-plus-GEMV pass per token on integer dot
+ *             products with exact, non-saturating i32 accumulation) and
+ *             "Command Reference", `focr robot` (the selftest's worst-case
+ *             K = 6848 i32-accumulation case against a bit-identical scalar
+ *             oracle).
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   - scale s = fp32(max|w|) / Q as one fp32 division (Q = 7 int4, 127 int8);
@@ -325,6 +331,54 @@ void orc_lm_head(const int8_t* q, const float* s, const float* x, int T, int64_t
         argmax[t] = (int32_t)bi;
     }
     (void)nthreads;
+}
+
+/* ------------------------------------------------------------ W8A8 GEMV [P4-cpu] */
+/*
+ * Per-token activation quantisation (reading: symmetric, like the weights, one fp32
+ * scale per token): s_x = fp32(max_k |x_k|) / 127 as one fp32 division, q_k =
+ * clamp(round_half_even(x_k / s_x)) to [-127, 127] with the fp32 quotient; s_x = 0
+ * gives q = 0.
+ */
+void orc_w8a8_quantize_x(const float* x, int T, int K, int8_t* qx, float* sx) {
+    for (int t = 0; t < T; ++t) {
+        const float* xt = x + (int64_t)t * K;
+        float m = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            float a = fabsf(xt[k]);
+            if (a > m) m = a;
+        }
+        const float sc = m / 127.0f;
+        sx[t] = sc;
+        for (int k = 0; k < K; ++k) {
+            int v = 0;
+            if (sc != 0.0f) {
+                float rn = nearbyintf(xt[k] / sc);
+                if (rn > 127.0f) rn = 127.0f;
+                if (rn < -127.0f) rn = -127.0f;
+                v = (int)rn;
+            }
+            qx[(int64_t)t * K + k] = (int8_t)v;
+        }
+    }
+}
+
+/*
+ * y[t, n] = s_w[n] * s_x[t] * acc with acc = sum_k q_w[n, k] * q_x[t, k] over the
+ * whole row (exact integer; the pages' kernels accumulate it in i32, which holds for
+ * K <= 133143 at |q| <= 127), evaluated as fp32( (fp64(s_w) * fp64(s_x)) * fp64(acc) ).
+ * The sum is formed in int64 here and returned through acc_out (nullable) so that
+ * the tests can check the i32 bound.
+ */
+void orc_w8a8_gemv(const int8_t* qw, const float* sw, int64_t N, int K, const int8_t* qx, const float* sx,
+                   int T, float* y, int64_t* acc_out) {
+    for (int t = 0; t < T; ++t)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t acc = 0;
+            for (int k = 0; k < K; ++k) acc += (int64_t)qw[n * K + k] * (int64_t)qx[(int64_t)t * K + k];
+            if (acc_out) acc_out[(int64_t)t * N + n] = acc;
+            y[(int64_t)t * N + n] = (float)(((double)sw[n] * (double)sx[t]) * (double)acc);
+        }
 }
 
 int orc_max_threads(void) {

@@ -32,6 +32,12 @@ MUTATIONS = {
     "lm_head_ties_to_last": ("if (bi < 0 || lg > best) { best = lg; bi = n; }", "if (bi < 0 || lg >= best) { best = lg; bi = n; }"),
     "router_weight_transposed": ("(double)orc_bf16_to_f32(wr[(int64_t)e * H + k])", "(double)orc_bf16_to_f32(wr[(int64_t)k * E + e])"),
     "routed_weight_renormalised": ("acc[c] += wj * y[c];", "acc[c] += (wj / w[(int64_t)t * L->topk]) * y[c];"),
+    "w8a8_x_divisor_128": ("const float sc = m / 127.0f;", "const float sc = m / 128.0f;"),
+    "w8a8_x_round_half_away": ("float rn = nearbyintf(xt[k] / sc);", "float rn = roundf(xt[k] / sc);"),
+    "w8a8_activation_scale_dropped": ("(float)(((double)sw[n] * (double)sx[t]) * (double)acc)",
+                                      "(float)((double)sw[n] * (double)acc)"),
+    "w8a8_activation_transposed": ("(int64_t)qw[n * K + k] * (int64_t)qx[(int64_t)t * K + k]",
+                                   "(int64_t)qw[n * K + k] * (int64_t)qx[(int64_t)k * T + t]"),
 }
 
 

@@ -418,3 +418,88 @@ def test_bf16_rounding_is_nearest_even():
     exp = np.array([1.0, 1.0, 1.015625, 1.0078125, -1.0, 1.0078125], np.float32)
     np.testing.assert_array_equal(oracle.round_bf16(vals), exp)
     np.testing.assert_array_equal(oracle.f32_to_bf16(vals), synth.f32_to_bf16_bits(vals))
+
+
+# ------------------------------------------------------------------ W8A8 GEMV
+# franken_ocr README, "CPU Backend and Optimizations": the int8 decode linears quantise the
+# activation per token and run an integer GEMV with exact i32 accumulation; "Command Reference",
+# `focr robot`: the worst case is K = 6848.
+
+def _w8a8_golden():
+    out = []
+    with open(os.path.join(GOLDEN, "w8a8_activation_cases.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                x, s, q = [p.strip() for p in line.split("|")]
+                out.append((np.array(x.split(), np.float32), np.float32(s), np.array(q.split(), np.int8)))
+    return out
+
+
+@pytest.mark.parametrize("case", _w8a8_golden(), ids=lambda c: f"K{c[0].size}-s{c[1]}")
+def test_w8a8_activation_golden(case):
+    x, s_exp, q_exp = case
+    qx, sx = oracle.w8a8_quantize_x(x[None, :])
+    assert sx[0] == s_exp
+    np.testing.assert_array_equal(qx[0], q_exp)
+
+
+def test_w8a8_activation_error_bound_and_extreme_code():
+    rng = np.random.default_rng(81)
+    x = (rng.standard_normal((9, 333)) * rng.uniform(1e-3, 1e3, (9, 1))).astype(np.float32)
+    x[2, 5] = -50.0 * np.abs(x[2]).max()    # a negative outlier owns the scale
+    qx, sx = oracle.w8a8_quantize_x(x)
+    amax = np.abs(x).max(axis=1)
+    np.testing.assert_array_equal(np.abs(qx).max(axis=1), 127)
+    np.testing.assert_array_equal(qx[np.arange(9), np.abs(x).argmax(axis=1)],
+                                  (127 * np.sign(x[np.arange(9), np.abs(x).argmax(axis=1)])).astype(np.int8))
+    assert np.all(np.abs(sx.astype(np.float64) * 127 - amax) <= 1e-6 * amax)
+    err = np.abs(qx.astype(np.float64) * sx[:, None] - x)
+    assert np.all(err <= 0.5 * sx[:, None].astype(np.float64) * (1 + 1e-5))
+
+
+def test_w8a8_power_of_two_scales_give_the_exact_product():
+    # every max is 127 * 2^e and every entry a multiple of 2^e: both quantisers are exact, and
+    # K * 127^2 < 2^24 keeps the fp32 result exact, so y must equal the plain integer dot product
+    rng = np.random.default_rng(82)
+    N, K, T = 37, 64, 3
+    iw = rng.integers(-127, 128, (N, K)); iw[:, 7] = 127
+    ix = rng.integers(-127, 128, (T, K)); ix[:, 11] = -127
+    ew, ex = rng.integers(-6, 4, N), np.array([-3, 0, 5])
+    w = (iw * 2.0 ** ew[:, None]).astype(np.float32)
+    x = (ix * 2.0 ** ex[:, None]).astype(np.float32)
+    y, qx, sx = oracle.OracleW8A8(w).forward(x)
+    np.testing.assert_array_equal(qx, ix.astype(np.int8))
+    np.testing.assert_array_equal(sx, (2.0 ** ex).astype(np.float32))
+    exact = (ix.astype(np.int64) @ iw.T.astype(np.int64)) * 2.0 ** (ex[:, None] + ew[None, :])
+    np.testing.assert_array_equal(y, exact.astype(np.float32))
+
+
+def test_w8a8_worst_case_accumulator_fits_i32_at_k6848():
+    K = synth.DENSE_I
+    assert K == 6848
+    w = np.full((2, K), 127.0, np.float32)
+    w[1, 1::2] = -127.0
+    x = np.full((1, K), 127.0, np.float32)
+    y, _, _, acc = oracle.OracleW8A8(w).forward(x, want_acc=True)
+    assert acc[0, 0] == K * 127 * 127 == 110_451_392 < 2 ** 31 - 1
+    assert acc[0, 1] == 0
+    # s_w = s_x = 1, and 110,451,392 is a multiple of 8 (the fp32 spacing there): y is acc exactly
+    assert y[0, 0] == 110_451_392.0 and y[0, 1] == 0.0
+
+
+def test_w8a8_gemv_brute_force_integer_dot():
+    rng = np.random.default_rng(83)
+    N, K, T = 5, 29, 4
+    w = rng.standard_normal((N, K)).astype(np.float32)
+    x = rng.standard_normal((T, K)).astype(np.float32)
+    om = oracle.OracleW8A8(w)
+    y, qx, sx, acc = om.forward(x, want_acc=True)
+    for t in range(T):
+        for n in range(N):
+            a = sum(int(om.q[n, k]) * int(qx[t, k]) for k in range(K))
+            assert acc[t, n] == a
+            assert y[t, n] == np.float32((float(om.s[n]) * float(sx[t])) * a)
+    # against the unquantised product: the error of symmetric 8-bit codes on both sides
+    ref = x.astype(np.float64) @ w.T.astype(np.float64)
+    assert np.abs(y - ref).max() <= 0.05 * np.abs(ref).max()
