@@ -65,6 +65,9 @@ def describe(name: str, world: int) -> dict:
         w = synth.STEP_WORKLOADS[name]
         d = {"workload": name, "tokens_per_step": w["T"], "kind": w["kind"], "seed": w["seed"],
              "parallelism": f"replicas x{world}"}
+        if w["kind"] == "w8a8":
+            d.update(matrix="129280 x 1280 int8, one fp32 scale per row (the lm_head's shape)",
+                     activations="int8, one fp32 scale per token", accumulate="exact integer (i32)")
         if w["kind"] == "stack":
             d.update(wiring="h <- RMSNorm(h + FFN(h)) per layer (eps 1e-6, gamma 1); lm_head on the last norm",
                      moe_layers=w["moe_layers"], moe="int4 g64, bf16 router and shared expert",
@@ -248,6 +251,7 @@ def step_oracle_baseline(w: dict, budget_s: float = 12.0) -> dict:
     cores = oracle.max_threads()
     kind = w["kind"]
     lm = oracle.OracleLMHead(synth.lm_head(w["seed"])) if kind in ("lm_head", "stack") else None
+    w8 = oracle.OracleW8A8(synth.lm_head(w["seed"])) if kind == "w8a8" else None
     dn = None
     if kind in ("dense", "stack"):
         d = synth.dense_mlp(w["seed"])
@@ -258,6 +262,8 @@ def step_oracle_baseline(w: dict, budget_s: float = 12.0) -> dict:
     def run(x, th):
         if kind == "lm_head":
             lm.forward(x, nthreads=th)
+        elif kind == "w8a8":
+            w8.forward(x)
         elif kind == "dense":
             dn.forward(x, nthreads=th)
         else:
@@ -267,6 +273,8 @@ def step_oracle_baseline(w: dict, budget_s: float = 12.0) -> dict:
             lm.forward(h, nthreads=th)
 
     pool = synth.hidden(w["seed"] + 5000, 512)
+    if kind == "w8a8":   # the oracle's W8A8 GEMV is single-threaded
+        cores = 1
     batch = max(1, min(cores, 8)) if kind == "stack" else cores
     nall, tall = _timed_tokens(run, pool, batch, budget_s, cores)
     if nall == 0:   # one batch did not fit the budget: time one anyway
@@ -274,10 +282,11 @@ def step_oracle_baseline(w: dict, budget_s: float = 12.0) -> dict:
         run(pool[:batch], cores)
         nall, tall = batch, time.perf_counter() - t0
     used = min(cores, batch)
-    what = "dense layer 0, 11 MoE layers, RMSNorm, lm_head" if kind == "stack" else kind
+    what = {"stack": "dense layer 0, 11 MoE layers, RMSNorm, lm_head",
+            "w8a8": "W8A8 GEMV (129280 x 1280)"}.get(kind, kind)
     return {"value": nall / tall, "unit": UNIT, "cores": used, "kind": "oracle",
             "sample": f"{nall} tokens through the CPU oracle's {what} in batches of {batch} ({used} threads, "
-                      f"plain C, fp64, OpenMP) in {tall:.1f} s"}
+                      f"{'plain C, int64 dot' if kind == 'w8a8' else 'plain C, fp64, OpenMP'}) in {tall:.1f} s"}
 
 
 # ------------------------------------------------------------------ reference arm
@@ -294,7 +303,7 @@ def run_reference(args, rank, world):
         w = synth.STEP_WORKLOADS[args.workload]
         cpu = step_oracle_baseline(w, budget_s=60.0)
         v = cpu["value"]
-        dtype = "f64"
+        dtype = "int64" if w["kind"] == "w8a8" else "f64"
         print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
                           "steps": args.steps, "warmup": args.warmup, "ms_per_step": w["T"] / v * 1e3,
                           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
@@ -396,6 +405,8 @@ def step_bytes_companion(w: dict, moe_hits=None) -> int:
     dense = roofline.swiglu_bytes(roofline.DENSE_I, roofline.W_INT8, 128) + T * roofline.H * 4 * 2
     if w["kind"] == "lm_head":
         return lm
+    if w["kind"] == "w8a8":   # codes, row scales, x in, y out
+        return roofline.VOCAB * roofline.H + roofline.VOCAB * 4 + T * roofline.H * 4 + T * roofline.VOCAB * 4
     if w["kind"] == "dense":
         return dense
     moe = sum(roofline.moe_layer_bytes(T, roofline.W_INT4, roofline.W_BF16, 64, h) for h in moe_hits)
@@ -414,8 +425,13 @@ def run_step_workload(args, rank, world, local_rank):
     T, kind = w["T"], w["kind"]
     head = mlp = None
     layers = []
+    w8 = None
     if kind in ("lm_head", "stack"):
         head = api.focr_lm_head_pack(synth.lm_head(w["seed"]))
+    if kind == "w8a8":
+        w8 = api.focr_w8a8_pack(synth.lm_head(w["seed"]))
+        w8_ws = torch.zeros(api.focr_w8a8_workspace_bytes(w8, T), dtype=torch.uint8, device=dev)
+        w8_y = torch.empty(T, w8.N, device=dev)
     if kind in ("dense", "stack"):
         d = synth.dense_mlp(w["seed"])
         mlp = api.focr_dense_mlp_pack(d.gate, d.up, d.down, synth.W_INT8, 128)
@@ -434,13 +450,16 @@ def run_step_workload(args, rank, world, local_rank):
     stream = torch.cuda.Stream(device=dev)
     per_dense = 2 if T <= 8 else 2            # (memset or x-rows) + expert kernel(s)
     per_moe = 3 if T <= 8 else 2
-    launches = {"lm_head": 1, "dense": per_dense}.get(kind, 0)
+    launches = {"lm_head": 1, "dense": per_dense, "w8a8": 2}.get(kind, 0)
     if kind == "stack":
         launches = per_dense + 1 + (per_moe + 1) * len(layers) + 1
 
     def run(x, st, debug_counts=None):
         if kind == "lm_head":
             api.focr_lm_head_gemv(head, x, argmax=am, workspace=lm_ws, stream=st)
+            return
+        if kind == "w8a8":
+            api.focr_w8a8_gemv(w8, x, y=w8_y, workspace=w8_ws, stream=st)
             return
         if kind == "dense":
             api.focr_dense_mlp_forward(mlp, x, out=hb[0], workspace=ws, stream=st)
@@ -486,7 +505,7 @@ def run_step_workload(args, rank, world, local_rank):
     peak, _, _, peak_kind = peaks()
     achieved = bytes_step / (ms_step / 1e3) / 1e9
     # end to end: pinned host x in, the step, the step's result (argmax, or the dense output) out
-    out_t = hb[0] if kind == "dense" else am
+    out_t = hb[0] if kind == "dense" else (w8_y if kind == "w8a8" else am)
     hx = torch.from_numpy(synth.hidden(w["seed"] + 4000, T)).pin_memory()
     hy = torch.empty(out_t.shape, dtype=out_t.dtype).pin_memory()
     dx = torch.empty(T, 1280, device=dev)
@@ -512,6 +531,9 @@ def run_step_workload(args, rank, world, local_rank):
         cpu = step_oracle_baseline(w)
     if rank == 0:
         dtype, prec = precision(T)
+        if kind == "w8a8":
+            dtype, prec = "s8", ("int8 weights and per-token int8 activations, mma.sync m16n8k32 s8 with exact "
+                                 "s32 accumulation; scales applied in fp64, one rounding to fp32")
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
                 "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": dtype, "precision": prec, "data": "synthetic", "config": describe(args.workload, world),

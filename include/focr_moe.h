@@ -318,6 +318,61 @@ size_t focr_decode_step_workspace_bytes(int32_t T_max);
 focr_status focr_decode_step(const focr_decode_model* m, const float* x, int32_t T, float* logits, int32_t* argmax,
                              float* hidden_out, void* workspace, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------ W8A8 linear
+ * Source: franken_ocr README, "CPU Backend and Optimizations" -- the int8 decode linears run
+ * one quantise-plus-GEMV pass per token: the activation is quantised to int8, integer dot
+ * products accumulate exactly in i32 (no saturation) and the two scales are applied at the end;
+ * "Command Reference", `focr robot` -- K = 6848 is the worst case of that accumulation.
+ * Readings (the pages fix no formula): weights int8 with one scale per row and activations
+ * int8 with one scale per token, both symmetric:
+ *     s = fp32(max|v|) / 127 (one fp32 division), q = round-half-even(v / s) clamped to
+ *     [-127, 127]; an all-zero row or token has s = 0 and q = 0;
+ *     acc[t, n] = sum_k q_w[n, k] * q_x[t, k]    (exact: |acc| <= K * 127^2 < 2^31);
+ *     y[t, n]   = fp32((fp64(s_w[n]) * fp64(s_x[t])) * fp64(acc[t, n])).
+ * Every step is exact integer arithmetic or one correctly rounded IEEE operation, so results
+ * are bit-identical to any implementation of the same formula.  Inputs must be finite.
+ */
+#define FOCR_W8A8_T_MAX 64         /* most tokens one focr_w8a8_gemv call accepts */
+#define FOCR_W8A8_K_MAX 133143     /* largest K with K * 127^2 < 2^31 */
+#define FOCR_W8A8_N_MAX 67108864   /* most rows of one matrix */
+
+typedef struct focr_w8a8 focr_w8a8;   /* opaque, device-resident, library-owned */
+
+/*
+ * focr_w8a8_pack -- quantise w (HOST fp32 [N, K], row-major) to int8 with one scale per row
+ * and lay it out on the device (row tiles of 16, k-steps of 32, zero-padded; N * K bytes of
+ * codes after padding).  1 <= N <= FOCR_W8A8_N_MAX, 1 <= K <= FOCR_W8A8_K_MAX.  Synchronises.
+ * Errors: FOCR_ERR_INVALID_ARG (NULL, sizes out of range), FOCR_ERR_OOM, FOCR_ERR_CUDA.
+ */
+focr_status focr_w8a8_pack(const float* w, int64_t N, int32_t K, focr_w8a8** out, void* stream);
+void focr_w8a8_free(focr_w8a8* m);
+
+/* Canonical codes (int8 [N, K] row-major) and row scales (f32 [N]) to HOST memory; N and K of m. */
+focr_status focr_w8a8_export(const focr_w8a8* m, int8_t* codes_host, float* scales_host, int64_t* N, int32_t* K);
+
+/*
+ * focr_w8a8_quantize_x -- the activation quantiser alone: x (DEVICE fp32 [T, K], row-major) to
+ * qx (DEVICE int8 [T, K]) and sx (DEVICE fp32 [T]).  1 <= T <= FOCR_T_MAX, 1 <= K <=
+ * FOCR_W8A8_K_MAX.  Asynchronous on `stream`.
+ */
+focr_status focr_w8a8_quantize_x(const float* x, int32_t T, int32_t K, int8_t* qx, float* sx, void* stream);
+
+/* Workspace a focr_w8a8_gemv call on m with up to T_max tokens needs (bytes). */
+size_t focr_w8a8_workspace_bytes(const focr_w8a8* m, int32_t T_max);
+
+/*
+ * focr_w8a8_gemv -- y = W8A8(m, x): quantises x per token, then the integer GEMV and the
+ * scales (two launches, chained by programmatic dependent launch).
+ *   x: DEVICE fp32 [T, K] row-major (K of m), 1 <= T <= FOCR_W8A8_T_MAX;  y: DEVICE fp32 [T, N].
+ *   workspace: DEVICE, 256-byte aligned, >= focr_w8a8_workspace_bytes(m, T) bytes, zero-filled
+ *   once before its first use (every completed call leaves its sums and counters zero; calls
+ *   on one workspace must not overlap).  Asynchronous on `stream`.
+ * Errors: FOCR_ERR_INVALID_ARG (NULL, T out of range, misaligned or short workspace),
+ * FOCR_ERR_CUDA (a launch failed).
+ */
+focr_status focr_w8a8_gemv(const focr_w8a8* m, const float* x, int32_t T, float* y, void* workspace,
+                           size_t ws_bytes, void* stream);
+
 /*
  * focr_tc_selftest -- diagnostic: one tensor-core tile through the library's tcgen05 primitives
  * (the ones the T > 8 grouped kernel uses), to check them against a host GEMM.

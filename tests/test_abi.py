@@ -86,3 +86,22 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(api, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         api.lib()
+
+
+def test_w8a8_rejects_bad_arguments_without_launching():
+    L = api.lib()
+    h = ctypes.c_void_p()
+    w = (ctypes.c_float * 16)()
+    p = ctypes.cast(w, ctypes.c_void_p).value
+    assert L.focr_w8a8_pack(None, 1, 1, ctypes.byref(h), None) == 1
+    for n, k in ((0, 16), (1, 0), (1, api.W8A8_K_MAX + 1), (1 << 27, 16)):
+        assert L.focr_w8a8_pack(p, n, k, ctypes.byref(h), None) == 1
+        assert "outside" in api.focr_last_error() and not h.value
+    assert L.focr_w8a8_gemv(None, p, 1, p, p, 1 << 20, None) == 1
+    assert L.focr_w8a8_workspace_bytes(None, 1) == 0
+    assert L.focr_w8a8_export(None, None, None, None, None) == 1
+    q = (ctypes.c_int8 * 16)()
+    qp = ctypes.cast(q, ctypes.c_void_p).value
+    for T, K in ((0, 16), (api.T_MAX + 1, 16), (1, 0),
+                 (1, api.W8A8_K_MAX + 1)):
+        assert L.focr_w8a8_quantize_x(p, T, K, qp, p, None) == 1

@@ -33,7 +33,8 @@ EXPORTED = (
     "focr_moe_layer_forward_ex", "focr_lm_head_pack", "focr_lm_head_free", "focr_lm_head_export",
     "focr_lm_head_workspace_bytes", "focr_lm_head_gemv", "focr_rmsnorm", "focr_dense_mlp_pack",
     "focr_dense_mlp_free", "focr_dense_mlp_export_quantized", "focr_dense_mlp_forward", "focr_tc_selftest",
-    "focr_decode_step_workspace_bytes", "focr_decode_step",
+    "focr_decode_step_workspace_bytes", "focr_decode_step", "focr_w8a8_pack", "focr_w8a8_free",
+    "focr_w8a8_export", "focr_w8a8_quantize_x", "focr_w8a8_workspace_bytes", "focr_w8a8_gemv",
 )
 FWD_RESIDUAL = 1
 FWD_DETERMINISTIC = 2
@@ -75,7 +76,7 @@ def lib():
             if not os.path.exists(LIB_PATH):
                 raise RuntimeError(f"{LIB_PATH} is missing: build it with weight_quantized_expert_b200/build.py")
             L = ctypes.CDLL(LIB_PATH)
-            P, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+            P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
             sigs = {
                 "focr_moe_pack_weights": (i32, [ctypes.POINTER(WeightsDesc), ctypes.POINTER(P), P]),
                 "focr_moe_layer_clone": (i32, [P, ctypes.POINTER(P), P]),
@@ -103,6 +104,12 @@ def lib():
                 "focr_tc_selftest": (i32, [P, P, i32, i32, i32, P, P, P]),
                 "focr_decode_step_workspace_bytes": (sz, [i32]),
                 "focr_decode_step": (i32, [ctypes.POINTER(DecodeModelDesc), P, i32, P, P, P, P, sz, P]),
+                "focr_w8a8_pack": (i32, [P, i64, i32, ctypes.POINTER(P), P]),
+                "focr_w8a8_free": (None, [P]),
+                "focr_w8a8_export": (i32, [P, P, P, ctypes.POINTER(i64), ctypes.POINTER(i32)]),
+                "focr_w8a8_quantize_x": (i32, [P, i32, i32, P, P, P]),
+                "focr_w8a8_workspace_bytes": (sz, [P, i32]),
+                "focr_w8a8_gemv": (i32, [P, P, i32, P, P, sz, P]),
                 "focr_last_error": (ctypes.c_char_p, []),
                 "focr_version": (ctypes.c_char_p, []),
             }
@@ -292,6 +299,71 @@ def focr_lm_head_gemv(head: LMHead, x, argmax=None, logits=None, workspace=None,
     _check(lib().focr_lm_head_gemv(ctypes.c_void_p(head.handle), _ptr(x), T, _ptr(logits), _ptr(argmax),
                                    _ptr(workspace), workspace.numel(), _stream(stream)))
     return argmax
+
+
+# ---------------------------------------------------------------- W8A8 linear
+
+W8A8_T_MAX = 64
+W8A8_K_MAX = 133143
+
+
+class W8A8:
+    """A packed int8 matrix with one scale per row, for the W8A8 GEMV (owns its device memory)."""
+
+    def __init__(self, handle: int, N: int, K: int):
+        self.handle, self.N, self.K = handle, N, K
+
+    def __del__(self):
+        h, self.handle = getattr(self, "handle", None), None
+        if h and _lib is not None:
+            _lib.focr_w8a8_free(ctypes.c_void_p(h))
+
+
+def focr_w8a8_pack(w, stream=None) -> W8A8:
+    w = np.ascontiguousarray(w, np.float32)
+    N, K = w.shape
+    h = ctypes.c_void_p()
+    _check(lib().focr_w8a8_pack(w.ctypes.data, N, K, ctypes.byref(h), _stream(stream)))
+    return W8A8(h.value, N, K)
+
+
+def focr_w8a8_export(m: W8A8):
+    codes = np.empty((m.N, m.K), np.int8)
+    scales = np.empty(m.N, np.float32)
+    n, k = ctypes.c_int64(), ctypes.c_int32()
+    _check(lib().focr_w8a8_export(ctypes.c_void_p(m.handle), codes.ctypes.data, scales.ctypes.data,
+                                  ctypes.byref(n), ctypes.byref(k)))
+    assert (n.value, k.value) == (m.N, m.K)
+    return codes, scales
+
+
+def focr_w8a8_quantize_x(x, stream=None):
+    """Per-token int8 codes [T, K] and fp32 scales [T] of x (DEVICE fp32 [T, K])."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous() and x.dim() == 2
+    T, K = x.shape
+    qx = torch.empty(T, K, dtype=torch.int8, device=x.device)
+    sx = torch.empty(T, dtype=torch.float32, device=x.device)
+    _check(lib().focr_w8a8_quantize_x(_ptr(x), T, K, _ptr(qx), _ptr(sx), _stream(stream)))
+    return qx, sx
+
+
+def focr_w8a8_workspace_bytes(m: W8A8, T_max: int) -> int:
+    return int(lib().focr_w8a8_workspace_bytes(ctypes.c_void_p(m.handle), int(T_max)))
+
+
+def focr_w8a8_gemv(m: W8A8, x, y=None, workspace=None, stream=None):
+    """y[T, N] = W8A8(m, x) for x DEVICE fp32 [T, K]."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous() and x.shape[-1] == m.K
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty(T, m.N, dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.zeros(focr_w8a8_workspace_bytes(m, T), dtype=torch.uint8, device=x.device)
+    _check(lib().focr_w8a8_gemv(ctypes.c_void_p(m.handle), _ptr(x), T, _ptr(y), _ptr(workspace),
+                                workspace.numel(), _stream(stream)))
+    return y
 
 
 def focr_rmsnorm(x, gamma=None, eps: float = 1e-6, out=None, stream=None):

@@ -9,6 +9,7 @@
 #include "common.cuh"
 #include "lm_head.h"
 #include "pack.h"
+#include "w8a8.h"
 
 using namespace focr;
 
@@ -423,6 +424,138 @@ focr_status focr_lm_head_gemv(const focr_lm_head* L, const float* x, int32_t T, 
     const uint4* codes = reinterpret_cast<const uint4*>(L->dev);
     const float* scales = reinterpret_cast<const float*>(L->dev + (size_t)FOCR_VOCAB * H);
     CUDA_TRY(launch_lm_head(codes, scales, x, T, logits, argmax, workspace, (cudaStream_t)stream));
+    return FOCR_OK;
+}
+
+// ------------------------------------------------------------------ W8A8 linear
+
+struct focr_w8a8 {
+    uint8_t* dev = nullptr;   // codes (tiles * KS * 512 bytes) then scales (16 * tiles floats)
+    int64_t N = 0;
+    int32_t K = 0;
+    int64_t tiles = 0;
+    int64_t KS = 0;
+    size_t code_bytes = 0;
+};
+
+namespace {
+
+// workspace: [cnt: tiles u32][sx: FOCR_W8A8_T_MAX f32][qx fragments: KS x 8 groups x 256 B][acc: T x 16 tiles i32];
+// every offset is independent of T, so calls with different T can share one workspace
+struct W8a8Ws {
+    size_t cnt = 0, sx = 0, qxf = 0, acc = 0;
+};
+
+W8a8Ws w8a8_ws(const focr_w8a8* m) {
+    W8a8Ws o;
+    o.sx = align_up(sizeof(uint32_t) * (size_t)m->tiles, 256);
+    o.qxf = align_up(o.sx + sizeof(float) * FOCR_W8A8_T_MAX, 256);
+    o.acc = align_up(o.qxf + (size_t)m->KS * 256 * (FOCR_W8A8_T_MAX / 8), 256);
+    return o;
+}
+
+}  // namespace
+
+focr_status focr_w8a8_pack(const float* w, int64_t N, int32_t K, focr_w8a8** out, void* stream) {
+    g_err.clear();
+    if (!w || !out) return fail(FOCR_ERR_INVALID_ARG, "w and out must not be NULL");
+    *out = nullptr;
+    if (N < 1 || N > FOCR_W8A8_N_MAX) return fail(FOCR_ERR_INVALID_ARG, "N=%lld outside [1, %d]", (long long)N, FOCR_W8A8_N_MAX);
+    if (K < 1 || K > FOCR_W8A8_K_MAX) return fail(FOCR_ERR_INVALID_ARG, "K=%d outside [1, %d]", K, FOCR_W8A8_K_MAX);
+    const int64_t tiles = (N + 15) / 16, KS = ((int64_t)K + 31) / 32;
+    const size_t code_bytes = (size_t)(tiles * KS * 512), bytes = code_bytes + sizeof(float) * (size_t)(16 * tiles);
+    std::vector<uint8_t> host;
+    try {
+        host.resize(bytes);
+    } catch (...) {
+        return fail(FOCR_ERR_OOM, "host staging of %zu bytes failed", bytes);
+    }
+    host_pack_w8a8(w, N, K, host.data(), reinterpret_cast<float*>(host.data() + code_bytes));
+    focr_w8a8* M = new (std::nothrow) focr_w8a8();
+    if (!M) return fail(FOCR_ERR_OOM, "host allocation failed");
+    M->N = N;
+    M->K = K;
+    M->tiles = tiles;
+    M->KS = KS;
+    M->code_bytes = code_bytes;
+    cudaError_t e = cudaMalloc(&M->dev, bytes);
+    if (e != cudaSuccess) {
+        delete M;
+        return fail(e == cudaErrorMemoryAllocation ? FOCR_ERR_OOM : FOCR_ERR_CUDA, "cudaMalloc(%zu): %s", bytes,
+                    cudaGetErrorString(e));
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    e = cudaMemcpyAsync(M->dev, host.data(), bytes, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) {
+        cudaFree(M->dev);
+        delete M;
+        return cuda_fail(e, "upload of packed W8A8 matrix");
+    }
+    *out = M;
+    return FOCR_OK;
+}
+
+void focr_w8a8_free(focr_w8a8* M) {
+    if (!M) return;
+    if (M->dev) cudaFree(M->dev);
+    delete M;
+}
+
+focr_status focr_w8a8_export(const focr_w8a8* M, int8_t* codes, float* scales, int64_t* N, int32_t* K) {
+    g_err.clear();
+    if (!M || !M->dev) return fail(FOCR_ERR_INVALID_ARG, "matrix is NULL");
+    if (N) *N = M->N;
+    if (K) *K = M->K;
+    if (!codes && !scales) return FOCR_OK;
+    if (!codes || !scales) return fail(FOCR_ERR_INVALID_ARG, "codes and scales must both be given");
+    std::vector<uint8_t> host(M->code_bytes);
+    CUDA_TRY(cudaMemcpy(host.data(), M->dev, M->code_bytes, cudaMemcpyDeviceToHost));
+    CUDA_TRY(cudaMemcpy(scales, M->dev + M->code_bytes, sizeof(float) * (size_t)M->N, cudaMemcpyDeviceToHost));
+    host_unpack_w8a8(host.data(), M->N, M->K, codes);
+    return FOCR_OK;
+}
+
+focr_status focr_w8a8_quantize_x(const float* x, int32_t T, int32_t K, int8_t* qx, float* sx, void* stream) {
+    g_err.clear();
+    if (!x || !qx || !sx) return fail(FOCR_ERR_INVALID_ARG, "x, qx and sx must not be NULL");
+    if (T < 1 || T > FOCR_T_MAX) return fail(FOCR_ERR_INVALID_ARG, "T=%d outside [1, %d]", T, FOCR_T_MAX);
+    if (K < 1 || K > FOCR_W8A8_K_MAX) return fail(FOCR_ERR_INVALID_ARG, "K=%d outside [1, %d]", K, FOCR_W8A8_K_MAX);
+    if (!aligned(x, 4) || !aligned(sx, 4)) return fail(FOCR_ERR_INVALID_ARG, "x and sx must be 4-byte aligned");
+    CUDA_TRY(launch_w8a8_quantize(x, T, K, qx, nullptr, sx, (cudaStream_t)stream));
+    return FOCR_OK;
+}
+
+size_t focr_w8a8_workspace_bytes(const focr_w8a8* M, int32_t T_max) {
+    if (!M) return 0;
+    if (T_max < 1) T_max = 1;
+    if (T_max > FOCR_W8A8_T_MAX) T_max = FOCR_W8A8_T_MAX;
+    const W8a8Ws o = w8a8_ws(M);
+    const W8a8Plan pl = w8a8_plan(M->tiles, (int)M->KS);
+    const size_t acc = pl.S > 1 ? sizeof(int32_t) * (size_t)T_max * (size_t)(16 * M->tiles) : 0;
+    return align_up(o.acc + acc, 256);
+}
+
+focr_status focr_w8a8_gemv(const focr_w8a8* M, const float* x, int32_t T, float* y, void* workspace,
+                           size_t ws_bytes, void* stream) {
+    g_err.clear();
+    if (!M || !M->dev) return fail(FOCR_ERR_INVALID_ARG, "matrix is NULL");
+    if (!x || !y || !workspace) return fail(FOCR_ERR_INVALID_ARG, "x, y and workspace must not be NULL");
+    if (T < 1 || T > FOCR_W8A8_T_MAX) return fail(FOCR_ERR_INVALID_ARG, "T=%d outside [1, %d]", T, FOCR_W8A8_T_MAX);
+    if (!aligned(x, 4) || !aligned(y, 4) || !aligned(workspace, 256))
+        return fail(FOCR_ERR_INVALID_ARG, "misaligned x, y or workspace");
+    const size_t need = focr_w8a8_workspace_bytes(M, T);
+    if (ws_bytes < need) return fail(FOCR_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, need);
+    const W8a8Ws o = w8a8_ws(M);
+    char* ws = reinterpret_cast<char*>(workspace);
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(ws + o.cnt);
+    float* sx = reinterpret_cast<float*>(ws + o.sx);
+    uint32_t* qxf = reinterpret_cast<uint32_t*>(ws + o.qxf);
+    int32_t* acc = reinterpret_cast<int32_t*>(ws + o.acc);
+    cudaStream_t st = (cudaStream_t)stream;
+    CUDA_TRY(launch_w8a8_quantize(x, T, M->K, nullptr, qxf, sx, st));
+    const float* sw = reinterpret_cast<const float*>(M->dev + M->code_bytes);
+    CUDA_TRY(launch_w8a8_gemv(M->dev, sw, M->N, M->K, qxf, sx, T, y, acc, cnt, st));
     return FOCR_OK;
 }
 

@@ -366,3 +366,37 @@ void host_unpack_lm_head(const uint8_t* codes, int64_t V, int8_t* q) {
 }
 
 }  // namespace focr
+
+namespace focr {
+
+int64_t w8a8_code_offset(int64_t row, int64_t col, int64_t KS) {
+    const int64_t tile = row / 16, rr = row % 16, q = col / 32, kl = col % 32;
+    const int64_t gr = rr % 8, hi_row = rr / 8, half = kl / 16, c = (kl % 16) / 4, e = kl % 4;
+    const int64_t lane = 4 * gr + c, reg = 2 * half + hi_row;
+    return ((tile * KS + q) * 32 + lane) * 16 + reg * 4 + e;
+}
+
+void host_pack_w8a8(const float* w, int64_t N, int64_t K, uint8_t* codes, float* scales) {
+    const int64_t KS = (K + 31) / 32, tiles = (N + 15) / 16;
+    std::memset(codes, 0, (size_t)(tiles * KS * 512));
+    std::memset(scales, 0, sizeof(float) * (size_t)(tiles * 16));
+    parallel_for((int)tiles, [&](int r) {
+        const int64_t r0 = (int64_t)r * 16, rows = std::min<int64_t>(16, N - r0);
+        std::vector<int8_t> q((size_t)(rows * K));
+        host_quantize(w + r0 * K, rows, K, (int)K, 8, q.data(), scales + r0);
+        for (int64_t rr = 0; rr < rows; ++rr)
+            for (int64_t col = 0; col < K; ++col)
+                codes[w8a8_code_offset(r0 + rr, col, KS)] = (uint8_t)q[(size_t)(rr * K + col)];
+    });
+}
+
+void host_unpack_w8a8(const uint8_t* codes, int64_t N, int64_t K, int8_t* q) {
+    const int64_t KS = (K + 31) / 32;
+    parallel_for((int)((N + 15) / 16), [&](int r) {
+        const int64_t r1 = std::min<int64_t>(N, (int64_t)r * 16 + 16);
+        for (int64_t row = (int64_t)r * 16; row < r1; ++row)
+            for (int64_t col = 0; col < K; ++col) q[row * K + col] = (int8_t)codes[w8a8_code_offset(row, col, KS)];
+    });
+}
+
+}  // namespace focr

@@ -23,3 +23,14 @@ namespace focr {
 void host_pack_lm_head(const float* w, int64_t V, uint8_t* codes, float* scales);
 void host_unpack_lm_head(const uint8_t* codes, int64_t V, int8_t* q);
 }  // namespace focr
+
+namespace focr {
+// W8A8 linear: int8 codes with one scale per row (s = max|w| / 127), N rows padded to tiles of
+// 16 and K columns padded to k-steps of 32 with zero codes.  For row tile r and k-step q, lane
+// L = 4 gr + c of a warp holds the 16 bytes of an m16n8k32 s8 A fragment: {row gr, row gr + 8}
+// x {columns 32q + 4c .. +3, columns 32q + 16 + 4c .. +3}, as four 32-bit registers in the
+// order (gr, lo), (gr + 8, lo), (gr, hi), (gr + 8, hi).  codes: tiles * KS * 512 bytes.
+int64_t w8a8_code_offset(int64_t row, int64_t col, int64_t KS);
+void host_pack_w8a8(const float* w, int64_t N, int64_t K, uint8_t* codes, float* scales);
+void host_unpack_w8a8(const uint8_t* codes, int64_t N, int64_t K, int8_t* q);
+}  // namespace focr

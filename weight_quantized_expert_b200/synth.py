@@ -194,6 +194,9 @@ STEP_WORKLOADS = {
     "dense_t1": dict(kind="dense", seed=4, T=1),
     "stack_t1": dict(kind="stack", seed=4, T=1, moe_layers=11),
     "stack_t32": dict(kind="stack", seed=4, T=32, moe_layers=11),
+    # W8A8 GEMV on the lm_head's shape (129280 x 1280 int8, one scale per row; 165 MB > L2)
+    "w8a8_lm_head_t1": dict(kind="w8a8", seed=4, T=1),
+    "w8a8_lm_head_t8": dict(kind="w8a8", seed=4, T=8),
 }
 
 
