@@ -366,12 +366,20 @@ size_t focr_w8a8_workspace_bytes(const focr_w8a8* m, int32_t T_max);
  *   x: DEVICE fp32 [T, K] row-major (K of m), 1 <= T <= FOCR_W8A8_T_MAX;  y: DEVICE fp32 [T, N].
  *   workspace: DEVICE, 256-byte aligned, >= focr_w8a8_workspace_bytes(m, T) bytes, zero-filled
  *   once before its first use (every completed call leaves its sums and counters zero; calls
- *   on one workspace must not overlap).  Asynchronous on `stream`.
+ *   on one workspace must not overlap).  Asynchronous on `stream`; focr_w8a8_check reports a
+ *   device wait that ran out.
  * Errors: FOCR_ERR_INVALID_ARG (NULL, T out of range, misaligned or short workspace),
  * FOCR_ERR_CUDA (a launch failed).
  */
 focr_status focr_w8a8_gemv(const focr_w8a8* m, const float* x, int32_t T, float* y, void* workspace,
                            size_t ws_bytes, void* stream);
+
+/*
+ * focr_w8a8_check -- synchronises `stream` and reports whether a focr_w8a8_gemv call on this
+ * workspace met a device wait that ran out (its shared-memory pipeline waits are bounded):
+ * FOCR_ERR_TIMEOUT (the outputs of that call are not valid; the word is cleared) or FOCR_OK.
+ */
+focr_status focr_w8a8_check(void* workspace, void* stream);
 
 /*
  * focr_tc_selftest -- diagnostic: one tensor-core tile through the library's tcgen05 primitives

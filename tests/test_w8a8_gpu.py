@@ -46,8 +46,9 @@ def _packed(seed, N, K):
 
 def _gemv(m, x):
     import torch
-    y = api.focr_w8a8_gemv(m, torch.from_numpy(x).cuda())
-    torch.cuda.synchronize()
+    ws = torch.zeros(api.focr_w8a8_workspace_bytes(m, x.shape[0]), dtype=torch.uint8, device="cuda")
+    y = api.focr_w8a8_gemv(m, torch.from_numpy(x).cuda(), workspace=ws)
+    api.focr_w8a8_check(ws)
     return y.cpu().numpy()
 
 
@@ -121,8 +122,9 @@ def test_workspace_is_shared_across_token_counts_and_left_zero():
     np.testing.assert_array_equal(outs[0], outs[3])
     np.testing.assert_array_equal(outs[1], outs[0][:1])
     np.testing.assert_array_equal(outs[2], outs[0][:9])
+    api.focr_w8a8_check(ws)                          # no bounded wait ran out
     tiles = (1280 + 15) // 16
-    assert int(ws[: 4 * tiles].abs().sum()) == 0    # per-tile counters back at zero
+    assert int(ws[: 256 + 4 * tiles].sum()) == 0     # error word and per-tile counters back at zero
     np.testing.assert_array_equal(outs[0], om.forward(_x(300, 64, 6848))[0])
 
 

@@ -440,15 +440,15 @@ struct focr_w8a8 {
 
 namespace {
 
-// workspace: [cnt: tiles u32][sx: FOCR_W8A8_T_MAX f32][qx fragments: KS x 8 groups x 256 B][acc: T x 16 tiles i32];
-// every offset is independent of T, so calls with different T can share one workspace
+// workspace: [err word, 256 B][cnt: tiles u32][sx: FOCR_W8A8_T_MAX f32][qx fragments: KS x 8 groups x 256 B]
+// [acc: T x 16 tiles i32]; every offset is independent of T, so calls with different T can share one workspace
 struct W8a8Ws {
-    size_t cnt = 0, sx = 0, qxf = 0, acc = 0;
+    size_t err = 0, cnt = 256, sx = 0, qxf = 0, acc = 0;
 };
 
 W8a8Ws w8a8_ws(const focr_w8a8* m) {
     W8a8Ws o;
-    o.sx = align_up(sizeof(uint32_t) * (size_t)m->tiles, 256);
+    o.sx = align_up(o.cnt + sizeof(uint32_t) * (size_t)m->tiles, 256);
     o.qxf = align_up(o.sx + sizeof(float) * FOCR_W8A8_T_MAX, 256);
     o.acc = align_up(o.qxf + (size_t)m->KS * 256 * (FOCR_W8A8_T_MAX / 8), 256);
     return o;
@@ -552,11 +552,25 @@ focr_status focr_w8a8_gemv(const focr_w8a8* M, const float* x, int32_t T, float*
     float* sx = reinterpret_cast<float*>(ws + o.sx);
     uint32_t* qxf = reinterpret_cast<uint32_t*>(ws + o.qxf);
     int32_t* acc = reinterpret_cast<int32_t*>(ws + o.acc);
+    uint32_t* err = reinterpret_cast<uint32_t*>(ws + o.err);
     cudaStream_t st = (cudaStream_t)stream;
     CUDA_TRY(launch_w8a8_quantize(x, T, M->K, nullptr, qxf, sx, st));
     const float* sw = reinterpret_cast<const float*>(M->dev + M->code_bytes);
-    CUDA_TRY(launch_w8a8_gemv(M->dev, sw, M->N, M->K, qxf, sx, T, y, acc, cnt, st));
+    CUDA_TRY(launch_w8a8_gemv(M->dev, sw, M->N, M->K, qxf, sx, T, y, acc, cnt, err, st));
     return FOCR_OK;
+}
+
+focr_status focr_w8a8_check(void* workspace, void* stream) {
+    g_err.clear();
+    if (!workspace || !aligned(workspace, 256)) return fail(FOCR_ERR_INVALID_ARG, "workspace is NULL or misaligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t word = 0;
+    CUDA_TRY(cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st));
+    CUDA_TRY(cudaStreamSynchronize(st));
+    if (!word) return FOCR_OK;
+    CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(word), st));
+    CUDA_TRY(cudaStreamSynchronize(st));
+    return fail(FOCR_ERR_TIMEOUT, "a bounded wait of the W8A8 GEMV ran out; the outputs of that call are not valid");
 }
 
 focr_status focr_rmsnorm(const float* x, const float* gamma, int32_t T, float eps, float* out, void* stream) {

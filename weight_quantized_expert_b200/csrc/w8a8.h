@@ -18,8 +18,9 @@ cudaError_t launch_w8a8_quantize(const float* x, int T, int K, int8_t* qx, uint3
                                  cudaStream_t st);
 // y[T, N] from packed codes (tiles * KS * 512 bytes), row scales, qxf and sx.  acc (int32
 // [T, 16 * tiles]) and cnt (uint32 [tiles]) are zero before the launch and left zero; they are
-// touched only when the plan splits K (S > 1).
+// touched only when the plan splits K (S > 1).  *err is set to 1 if a bounded wait runs out.
 cudaError_t launch_w8a8_gemv(const void* codes, const float* sw, int64_t N, int K, const uint32_t* qxf,
-                             const float* sx, int T, float* y, int32_t* acc, uint32_t* cnt, cudaStream_t st);
+                             const float* sx, int T, float* y, int32_t* acc, uint32_t* cnt, uint32_t* err,
+                             cudaStream_t st);
 
 }  // namespace focr
