@@ -499,6 +499,8 @@ def run_step_workload(args, rank, world, local_rank):
         api.focr_moe_check(ws, stream)
     elif kind == "w8a8":
         api.focr_w8a8_check(w8_ws, stream)
+    elif kind == "lm_head":
+        api.focr_lm_head_check(lm_ws, stream)
     K = args.steps
     graphs, _ = capture_graphs(lambda i, st: run(xs[i % pool_n], st), K, stream)
     ms, clk = timed_replay(graphs, stream, world, dev, local_rank)

@@ -276,6 +276,13 @@ focr_status focr_lm_head_gemv(const focr_lm_head* head, const float* x, int32_t 
                               int32_t* argmax, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * focr_lm_head_check -- synchronises `stream` and reports whether a focr_lm_head_gemv call on this
+ * workspace met a device wait that ran out (the T <= 8 kernel's shared-memory pipeline waits are
+ * bounded): FOCR_ERR_TIMEOUT (that call's outputs are not valid; the word is cleared) or FOCR_OK.
+ */
+focr_status focr_lm_head_check(void* workspace, void* stream);
+
+/*
  * focr_rmsnorm -- out[t] = x[t] / sqrt(mean(x[t]^2) + eps) * gamma (gamma NULL: 1).
  * x, out: DEVICE fp32 [T, 1280], 16-byte aligned (may be the same buffer); gamma: DEVICE
  * fp32 [1280] or NULL.  Asynchronous on `stream`.

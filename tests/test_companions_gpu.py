@@ -62,7 +62,7 @@ def _check_argmax(got_idx, ref_logits, bound):
             assert got_idx[t] == top[0]
 
 
-@pytest.mark.parametrize("T", [1, 5, 32, 40])
+@pytest.mark.parametrize("T", [1, 5, 8, 9, 32, 40])
 def test_lm_head_logits_and_argmax(T):
     torch = _torch()
     ref, head = lm_case()
@@ -80,6 +80,25 @@ def test_lm_head_logits_and_argmax(T):
     am2 = api.focr_lm_head_gemv(head, xd)
     torch.cuda.synchronize()
     assert np.array_equal(am2.cpu().numpy(), am.cpu().numpy())
+
+
+def test_lm_head_ring_kernel_agrees_with_the_streaming_kernel():
+    # T <= 8 runs the bulk-copy ring kernel, T > 8 the streaming kernel: the same fragments and
+    # MMAs, the ring kernel summing each tile as two halves, so the first 8 tokens' logits agree to
+    # fp32 rounding of the partial sums
+    torch = _torch()
+    _, head = lm_case()
+    x = torch.from_numpy(synth.normal_f32(71, 1, (9, 1280))).cuda()
+    out = []
+    for T in (8, 9):
+        ws = torch.zeros(api.focr_lm_head_workspace_bytes(T), dtype=torch.uint8, device="cuda")
+        logits = torch.empty(T, 129280, device="cuda")
+        am = api.focr_lm_head_gemv(head, x[:T].contiguous(), logits=logits, workspace=ws)
+        api.focr_lm_head_check(ws)
+        out.append((logits[:8].cpu().numpy(), am[:8].cpu().numpy()))
+    scale = np.abs(out[1][0]).max()
+    np.testing.assert_allclose(out[0][0], out[1][0], rtol=0, atol=2e-6 * scale)
+    _check_argmax(out[0][1], out[1][0].astype(np.float64), 4e-6 * scale)
 
 
 def test_lm_head_tie_goes_to_the_lower_row():

@@ -35,6 +35,7 @@ EXPORTED = (
     "focr_dense_mlp_free", "focr_dense_mlp_export_quantized", "focr_dense_mlp_forward", "focr_tc_selftest",
     "focr_decode_step_workspace_bytes", "focr_decode_step", "focr_w8a8_pack", "focr_w8a8_free",
     "focr_w8a8_export", "focr_w8a8_quantize_x", "focr_w8a8_workspace_bytes", "focr_w8a8_gemv", "focr_w8a8_check",
+    "focr_lm_head_check",
 )
 FWD_RESIDUAL = 1
 FWD_DETERMINISTIC = 2
@@ -111,6 +112,7 @@ def lib():
                 "focr_w8a8_workspace_bytes": (sz, [P, i32]),
                 "focr_w8a8_gemv": (i32, [P, P, i32, P, P, sz, P]),
                 "focr_w8a8_check": (i32, [P, P]),
+                "focr_lm_head_check": (i32, [P, P]),
                 "focr_last_error": (ctypes.c_char_p, []),
                 "focr_version": (ctypes.c_char_p, []),
             }
@@ -365,6 +367,10 @@ def focr_w8a8_gemv(m: W8A8, x, y=None, workspace=None, stream=None):
     _check(lib().focr_w8a8_gemv(ctypes.c_void_p(m.handle), _ptr(x), T, _ptr(y), _ptr(workspace),
                                 workspace.numel(), _stream(stream)))
     return y
+
+
+def focr_lm_head_check(workspace, stream=None):
+    _check(lib().focr_lm_head_check(_ptr(workspace), _stream(stream)))
 
 
 def focr_w8a8_check(workspace, stream=None):

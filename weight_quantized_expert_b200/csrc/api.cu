@@ -573,6 +573,20 @@ focr_status focr_w8a8_check(void* workspace, void* stream) {
     return fail(FOCR_ERR_TIMEOUT, "a bounded wait of the W8A8 GEMV ran out; the outputs of that call are not valid");
 }
 
+focr_status focr_lm_head_check(void* workspace, void* stream) {
+    g_err.clear();
+    if (!workspace || !aligned(workspace, 256)) return fail(FOCR_ERR_INVALID_ARG, "workspace is NULL or misaligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    int32_t* word = reinterpret_cast<int32_t*>(workspace) + 1;
+    int32_t v = 0;
+    CUDA_TRY(cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, st));
+    CUDA_TRY(cudaStreamSynchronize(st));
+    if (!v) return FOCR_OK;
+    CUDA_TRY(cudaMemsetAsync(word, 0, sizeof(v), st));
+    CUDA_TRY(cudaStreamSynchronize(st));
+    return fail(FOCR_ERR_TIMEOUT, "a bounded wait of the lm_head GEMV ran out; the outputs of that call are not valid");
+}
+
 focr_status focr_rmsnorm(const float* x, const float* gamma, int32_t T, float eps, float* out, void* stream) {
     g_err.clear();
     if (T < 1 || T > FOCR_T_MAX) return fail(FOCR_ERR_INVALID_ARG, "T=%d outside [1, %d]", T, FOCR_T_MAX);
@@ -802,8 +816,10 @@ focr_status focr_decode_step(const focr_decode_model* m, const float* x, int32_t
     const focr_lm_head* L = m->head;
     const uint4* codes = reinterpret_cast<const uint4*>(L->dev);
     const float* scales = reinterpret_cast<const float*>(L->dev + (size_t)FOCR_VOCAB * H);
+    // a bounded wait of the lm_head that runs out is reported by focr_moe_check(workspace + 256)
+    int32_t* err = reinterpret_cast<int32_t*>(w + kStepMoeOff + ws_layout(1).ctrl) + CTRL_ERROR;
     CUDA_TRY(launch_lm_head(codes, scales, last, T, logits, argmax, reinterpret_cast<int*>(w),
-                            reinterpret_cast<unsigned long long*>(w + step_keys_off(T)), st));
+                            reinterpret_cast<unsigned long long*>(w + step_keys_off(T)), err, st));
     return FOCR_OK;
 }
 
