@@ -546,7 +546,8 @@ def run_step_workload(args, rank, world, local_rank):
                            "l2": "one step streams every layer once (> 1.5 GB)" if kind == "stack" else
                                  "inputs re-read every step"},
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                             "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                             "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
+                             "peak_kind": peak_kind,
                              "kernel": "one step of the workload (all its launches, timed together)",
                              "algorithmic_bytes_per_step": bytes_step},
                 "cpu_baseline": cpu,
