@@ -92,11 +92,13 @@ def lib():
             L.orc_lm_head.argtypes = [P, P, P, ctypes.c_int, i64, ctypes.c_int, P, P, ctypes.c_int]
             L.orc_w8a8_quantize_x.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P]
             L.orc_w8a8_gemv.argtypes = [P, P, i64, ctypes.c_int, P, P, ctypes.c_int, P, P]
+            L.orc_rswa_decode.argtypes = [P, P, P, P, P, P, ctypes.c_int, P, P, P] + [ctypes.c_int] * 4 + [P]
             L.orc_max_threads.restype = ctypes.c_int
             for name in ("orc_round_bf16_array", "orc_quantize_rows", "orc_nibble_pack",
                          "orc_nibble_unpack", "orc_gemv", "orc_swiglu", "orc_router_logits",
                          "orc_softmax_topk", "orc_dispatch", "orc_moe_forward", "orc_dense_mlp",
-                         "orc_rmsnorm", "orc_lm_head", "orc_w8a8_quantize_x", "orc_w8a8_gemv"):
+                         "orc_rmsnorm", "orc_lm_head", "orc_w8a8_quantize_x", "orc_w8a8_gemv",
+                         "orc_rswa_decode"):
                 getattr(L, name).restype = None
             _lib = L
     return _lib
@@ -347,6 +349,25 @@ class OracleW8A8:
         acc = np.empty((T, self.N), np.int64) if want_acc else None
         lib().orc_w8a8_gemv(_p(self.q), _p(self.s), self.N, self.K, _p(qx), _p(sx), T, _p(y), _p(acc))
         return (y, qx, sx, acc) if want_acc else (y, qx, sx)
+
+
+RSWA_HEADS, RSWA_DIM, RSWA_RING = 10, 128, 128
+
+
+def rswa_decode(q, k_new, v_new, k_ref, v_ref, ref_len, k_ring, v_ring, n_gen, W: int = RSWA_RING):
+    """One R-SWA decode step ([P4-rswa]).  q, k_new, v_new [B, H, D]; k_ref, v_ref [B, H, Rcap, D];
+    k_ring, v_ring [B, H, W, D]; ref_len, n_gen [B].  Returns (out [B, H, D], k_ring', v_ring')."""
+    q, k_new, v_new = (_c(a, np.float32) for a in (q, k_new, v_new))
+    k_ref, v_ref = _c(k_ref, np.float32), _c(v_ref, np.float32)
+    k_ring, v_ring = np.array(k_ring, np.float32, copy=True), np.array(v_ring, np.float32, copy=True)
+    ref_len, n_gen = _c(ref_len, np.int32), _c(n_gen, np.int32)
+    B, H, D = q.shape
+    Rcap = k_ref.shape[2]
+    assert k_ring.shape == (B, H, W, D) and v_ref.shape == k_ref.shape
+    out = np.empty((B, H, D), np.float32)
+    lib().orc_rswa_decode(_p(q), _p(k_new), _p(v_new), _p(k_ref), _p(v_ref), _p(ref_len), Rcap, _p(k_ring),
+                          _p(v_ring), _p(n_gen), B, H, D, W, _p(out))
+    return out, k_ring, v_ring
 
 
 def max_threads() -> int:

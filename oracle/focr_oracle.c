@@ -20,6 +20,13 @@
  *             top-6, MoE intermediate 896, vocab 129280).
  *   [P4-arch] franken_ocr README, "Architecture" (each expert 1280 -> 896
  *             SiLU-gated, 2 always-on shared experts, final RMSNorm, lm_head).
+ *   [P4-rswa] franken_ocr README, "Design Philosophy", bounded generated-token
+ *             KV, and "Architecture", R-SWA (every decoder attention layer:
+ *             each generated token attends to all reference tokens, a frozen
+ *             never-evicted block, plus the previous 128 generated tokens held
+ *             in a ring buffer); frankenocr.pages.dev, "One forward pass",
+ *             step 6 (ten heads of dimension 128; a read-only reference block
+ *             plus a 128-slot sliding ring).
  *   [P4-cpu]  franken_ocr README, "CPU Backend and Optimizations" (int8 decode
  *             linears as a quantise-plus-GEMV pass per token on integer dot
  *             products with exact, non-saturating i32 accumulation) and
@@ -379,6 +386,80 @@ void orc_w8a8_gemv(const int8_t* qw, const float* sw, int64_t N, int K, const in
             if (acc_out) acc_out[(int64_t)t * N + n] = acc;
             y[(int64_t)t * N + n] = (float)(((double)sw[n] * (double)sx[t]) * (double)acc);
         }
+}
+
+/* ------------------------------------------------------------ R-SWA decode attention [P4-rswa] */
+/*
+ * One decode step of one attention layer for B sequences, H heads of dimension D, ring of W slots.
+ * Sequence b holds ref_len[b] reference rows (row stride D, head stride Rcap * D) and has generated
+ * n_gen[b] >= 1 tokens, the current one included; generated token p lives in ring slot p mod W.
+ * The current token attends to every reference row and to the last min(n_gen, W) generated
+ * tokens, itself included:
+ *     s_j = (q . k_j) / sqrt(D),  a_j = exp(s_j - max_i s_i) / sum_i exp(s_i - max_i s_i),
+ *     out = sum_j a_j v_j.
+ * Its own k and v come from k_new / v_new; afterwards they are stored in slot (n_gen - 1) mod W.
+ * Readings where the pages are silent: the scale is 1/sqrt(head dim); q and k arrive with any
+ * position encoding already applied; "the previous 128 generated tokens" counts the current one,
+ * so the window is exactly the ring's W slots.  A sequence with ref_len outside [0, Rcap] or
+ * n_gen < 1 gets NaN outputs and leaves its ring unchanged.
+ */
+void orc_rswa_decode(const float* q, const float* k_new, const float* v_new, const float* k_ref,
+                     const float* v_ref, const int32_t* ref_len, int Rcap, float* k_ring, float* v_ring,
+                     const int32_t* n_gen, int B, int H, int D, int W, float* out) {
+    double* sc = (double*)malloc(sizeof(double) * ((size_t)Rcap + (size_t)W));
+    const double inv = 1.0 / sqrt((double)D);
+    for (int b = 0; b < B; ++b) {
+        const int R = ref_len[b], n = n_gen[b];
+        const int valid = R >= 0 && R <= Rcap && n >= 1;
+        const int p0 = n > W ? n - W : 0;   /* oldest generated token in the window */
+        for (int h = 0; h < H; ++h) {
+            const size_t bh = (size_t)b * H + h;
+            const float* qv = q + bh * D;
+            const float* kr = k_ref + bh * (size_t)Rcap * D;
+            const float* vr = v_ref + bh * (size_t)Rcap * D;
+            float* kg = k_ring + bh * (size_t)W * D;
+            float* vg = v_ring + bh * (size_t)W * D;
+            float* o = out + bh * D;
+            if (!valid) {
+                for (int d = 0; d < D; ++d) o[d] = NAN;
+                continue;
+            }
+            /* keys in order: reference rows, then generated tokens oldest to newest */
+            int nk = 0;
+            for (int r = 0; r < R; ++r) {
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += (double)qv[d] * (double)kr[(size_t)r * D + d];
+                sc[nk++] = acc * inv;
+            }
+            for (int p = p0; p < n; ++p) {
+                const float* kp = p == n - 1 ? k_new + bh * D : kg + (size_t)(p % W) * D;
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += (double)qv[d] * (double)kp[d];
+                sc[nk++] = acc * inv;
+            }
+            double m = sc[0];
+            for (int j = 1; j < nk; ++j)
+                if (sc[j] > m) m = sc[j];
+            double den = 0.0;
+            for (int j = 0; j < nk; ++j) den += exp(sc[j] - m);
+            for (int d = 0; d < D; ++d) {
+                double acc = 0.0;
+                int j = 0;
+                for (int r = 0; r < R; ++r, ++j) acc += exp(sc[j] - m) * (double)vr[(size_t)r * D + d];
+                for (int p = p0; p < n; ++p, ++j) {
+                    const float* vp = p == n - 1 ? v_new + bh * D : vg + (size_t)(p % W) * D;
+                    acc += exp(sc[j] - m) * (double)vp[d];
+                }
+                o[d] = (float)(acc / den);
+            }
+            const int slot = (n - 1) % W;
+            for (int d = 0; d < D; ++d) {
+                kg[(size_t)slot * D + d] = k_new[bh * D + d];
+                vg[(size_t)slot * D + d] = v_new[bh * D + d];
+            }
+        }
+    }
+    free(sc);
 }
 
 int orc_max_threads(void) {

@@ -36,6 +36,12 @@ MUTATIONS = {
     "w8a8_x_round_half_away": ("float rn = nearbyintf(xt[k] / sc);", "float rn = roundf(xt[k] / sc);"),
     "w8a8_activation_scale_dropped": ("(float)(((double)sw[n] * (double)sx[t]) * (double)acc)",
                                       "(float)((double)sw[n] * (double)acc)"),
+    "rswa_scale_dropped": ("const double inv = 1.0 / sqrt((double)D);", "const double inv = 1.0;"),
+    "rswa_window_129": ("const int p0 = n > W ? n - W : 0;", "const int p0 = n > W ? n - W - 1 : 0;"),
+    "rswa_reference_ignored": ("for (int r = 0; r < R; ++r) {\n                double acc = 0.0;",
+                               "for (int r = 0; r < 0; ++r) {\n                double acc = 0.0;"),
+    "rswa_no_max_subtraction": ("for (int j = 1; j < nk; ++j)\n                if (sc[j] > m) m = sc[j];", "m = 0.0;"),
+    "rswa_ring_slot_off_by_one": ("const int slot = (n - 1) % W;", "const int slot = n % W;"),
     "w8a8_activation_transposed": ("(int64_t)qw[n * K + k] * (int64_t)qx[(int64_t)t * K + k]",
                                    "(int64_t)qw[n * K + k] * (int64_t)qx[(int64_t)k * T + t]"),
 }

@@ -503,3 +503,119 @@ def test_w8a8_gemv_brute_force_integer_dot():
     # against the unquantised product: the error of symmetric 8-bit codes on both sides
     ref = x.astype(np.float64) @ w.T.astype(np.float64)
     assert np.abs(y - ref).max() <= 0.05 * np.abs(ref).max()
+
+
+# ------------------------------------------------------------------ R-SWA decode attention
+# franken_ocr README, "Design Philosophy" (bounded generated-token KV) and "Architecture" (R-SWA):
+# a generated token attends to every reference row plus the last 128 generated tokens, which a
+# 128-slot ring holds; frankenocr.pages.dev, "One forward pass", step 6: 10 heads of dimension 128.
+
+RH, RD, RW = oracle.RSWA_HEADS, oracle.RSWA_DIM, oracle.RSWA_RING
+
+
+def _rswa_inputs(seed, B, Rcap, fill=0.0):
+    rng = np.random.default_rng(seed)
+    f = lambda *s: rng.standard_normal(s).astype(np.float32)
+    return dict(q=f(B, RH, RD), k_new=f(B, RH, RD), v_new=f(B, RH, RD), k_ref=f(B, RH, Rcap, RD),
+                v_ref=f(B, RH, Rcap, RD), k_ring=f(B, RH, RW, RD) + fill, v_ring=f(B, RH, RW, RD) + fill)
+
+
+def _rswa(a, ref_len, n_gen):
+    return oracle.rswa_decode(a["q"], a["k_new"], a["v_new"], a["k_ref"], a["v_ref"], ref_len, a["k_ring"],
+                              a["v_ring"], n_gen)
+
+
+def test_rswa_single_key_returns_its_value():
+    a = _rswa_inputs(91, 2, 4)
+    out, kg, vg = _rswa(a, [0, 0], [1, 1])
+    np.testing.assert_array_equal(out, a["v_new"])                  # one key: weight exactly 1
+    np.testing.assert_array_equal(kg[:, :, 0], a["k_new"])         # token 0 goes to slot 0
+    np.testing.assert_array_equal(vg[:, :, 1:], a["v_ring"][:, :, 1:])
+
+
+def test_rswa_two_keys_take_hand_computed_weights():
+    # q . k_ref / sqrt(128) = ln 3 and q . k_new = 0: softmax weights 3/4 and 1/4
+    a = _rswa_inputs(92, 1, 3)
+    a["q"][:] = 0.0
+    a["q"][0, :, 5] = 2.0
+    a["k_ref"][:] = 0.0
+    a["k_ref"][0, :, 0, 5] = np.float32(np.sqrt(128.0) * np.log(3.0) / 2.0)
+    a["k_new"][:] = 0.0
+    out, _, _ = _rswa(a, [1], [1])
+    exp = 0.75 * a["v_ref"][:, :, 0].astype(np.float64) + 0.25 * a["v_new"].astype(np.float64)
+    np.testing.assert_allclose(out, exp, rtol=0, atol=1e-6)
+
+
+def test_rswa_zero_query_averages_the_window():
+    # q = 0 gives equal weights: the output is the mean of the attended values
+    a = _rswa_inputs(93, 1, 40)
+    a["q"][:] = 0.0
+    R, n = 17, 300
+    out, _, _ = _rswa(a, [R], [n])
+    cur = (n - 1) % RW
+    ring = a["v_ring"][0].astype(np.float64).copy()
+    ring[:, cur] = a["v_new"][0]
+    vals = np.concatenate([a["v_ref"][0, :, :R].astype(np.float64), ring], axis=1)
+    np.testing.assert_allclose(out[0], vals.mean(axis=1), rtol=0, atol=1e-6)
+
+
+@pytest.mark.parametrize("n", [5, 128, 129, 300])
+def test_rswa_window_is_the_last_128_generated_tokens(n):
+    # slots outside the window, and the current slot's stale token (n - 129), must not matter
+    a = _rswa_inputs(94, 1, 8)
+    base, kg, vg = _rswa(a, [6], [n])
+    b = {k: v.copy() for k, v in a.items()}
+    cur = (n - 1) % RW
+    outside = [s for s in range(RW) if s >= n] + [cur]
+    b["k_ring"][:, :, outside] = 1e4
+    b["v_ring"][:, :, outside] = -7e3
+    other, kg2, vg2 = _rswa(b, [6], [n])
+    np.testing.assert_array_equal(other, base)
+    np.testing.assert_array_equal(kg2[:, :, cur], a["k_new"])     # the current token is stored at (n - 1) mod 128
+    np.testing.assert_array_equal(vg2[:, :, cur], a["v_new"])
+    keep = [s for s in range(RW) if s != cur]
+    np.testing.assert_array_equal(vg2[:, :, keep], b["v_ring"][:, :, keep])
+    # a slot inside the window does matter
+    if n > 1:
+        c = {k: v.copy() for k, v in a.items()}
+        c["v_ring"][:, :, (n - 2) % RW] += 1.0
+        assert not np.array_equal(_rswa(c, [6], [n])[0], base)
+
+
+def test_rswa_reference_rows_are_attended():
+    a = _rswa_inputs(95, 1, 10)
+    base, _, _ = _rswa(a, [7], [3])
+    b = {k: v.copy() for k, v in a.items()}
+    b["v_ref"][:, :, 6] += 1.0                   # the last reference row counts
+    assert not np.array_equal(_rswa(b, [7], [3])[0], base)
+    c = {k: v.copy() for k, v in a.items()}
+    c["k_ref"][:, :, 7:] = 1e4                   # rows beyond ref_len do not
+    c["v_ref"][:, :, 7:] = 1e6
+    np.testing.assert_array_equal(_rswa(c, [7], [3])[0], base)
+
+
+def test_rswa_one_dominant_key_with_huge_scores():
+    # scores near 1e4: the largest key takes all the weight and nothing overflows
+    a = _rswa_inputs(96, 1, 5)
+    a["q"][:] = 0.0
+    a["q"][0, :, 0] = 100.0
+    a["k_ref"][:] = 0.0
+    a["k_ref"][0, :, :, 0] = np.array([10, 12, 20, 11, 9], np.float32)[None, :] * 100.0
+    a["k_new"][:] = 0.0
+    out, _, _ = _rswa(a, [5], [1])
+    assert np.isfinite(out).all()
+    np.testing.assert_allclose(out[0], a["v_ref"][0, :, 2], rtol=0, atol=1e-6)
+
+
+def test_rswa_sequences_are_independent_and_bad_lengths_give_nan():
+    a = _rswa_inputs(97, 3, 12)
+    lens, gens = [12, 0, 5], [1, 200, 64]
+    out, kg, vg = _rswa(a, lens, gens)
+    for b in range(3):
+        one = {k: v[b:b + 1] for k, v in a.items()}
+        o1, k1, v1 = _rswa(one, [lens[b]], [gens[b]])
+        np.testing.assert_array_equal(out[b], o1[0])
+        np.testing.assert_array_equal(kg[b], k1[0])
+    bad, kgb, _ = _rswa(a, [13, -1, 5], [1, 5, 0])
+    assert np.isnan(bad).all()
+    np.testing.assert_array_equal(kgb, a["k_ring"])   # rings unchanged
