@@ -65,6 +65,9 @@ def describe(name: str, world: int) -> dict:
         w = synth.STEP_WORKLOADS[name]
         d = {"workload": name, "tokens_per_step": w["T"], "kind": w["kind"], "seed": w["seed"],
              "parallelism": f"replicas x{world}"}
+        if w["kind"] == "rswa":
+            d.update(sequences=w["T"], reference_rows=w["R"], generated=w["n_gen"], heads=10, head_dim=128,
+                     ring=128, kv="fp32")
         if w["kind"] == "w8a8":
             d.update(matrix="129280 x 1280 int8, one fp32 scale per row (the lm_head's shape)",
                      activations="int8, one fp32 scale per token", accumulate="exact integer (i32)")
@@ -301,7 +304,7 @@ def run_reference(args, rank, world):
     cores = oracle.max_threads()
     if args.workload in synth.STEP_WORKLOADS:
         w = synth.STEP_WORKLOADS[args.workload]
-        cpu = step_oracle_baseline(w, budget_s=60.0)
+        cpu = rswa_oracle_baseline(w, budget_s=60.0) if w["kind"] == "rswa" else step_oracle_baseline(w, budget_s=60.0)
         v = cpu["value"]
         dtype = "int64" if w["kind"] == "w8a8" else "f64"
         print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
@@ -557,6 +560,114 @@ def run_step_workload(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ R-SWA decode attention
+
+def rswa_step_bytes(w: dict) -> int:
+    """Algorithmic bytes of one R-SWA decode step: every attended key and value row read once
+    (reference rows and the 128-slot window), q / k_new / v_new read, out written, the ring slot written."""
+    B, R, n = w["T"], w["R"], w["n_gen"]
+    row = 10 * 128 * 4
+    return B * ((R + min(n, 128)) * 2 * row + 4 * row + 2 * row)
+
+
+def rswa_oracle_baseline(w: dict, budget_s: float = 12.0) -> dict:
+    """sequences/s of the CPU oracle's R-SWA step (single-threaded) on the workload's shapes."""
+    import oracle
+    from weight_quantized_expert_b200 import synth
+    B, R = w["T"], w["R"]
+    a = synth.rswa_inputs(w["seed"], B, R)
+    done, t = 0, 0.0
+    while t < budget_s and done < 4096:
+        t0 = time.perf_counter()
+        oracle.rswa_decode(a["q"], a["k_new"], a["v_new"], a["k_ref"], a["v_ref"], [R] * B, a["k_ring"],
+                           a["v_ring"], [w["n_gen"]] * B)
+        t += time.perf_counter() - t0
+        done += B
+    return {"value": done / t, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{done} sequence-steps of workload rswa (B = {B}, {R} reference rows, 128-slot window) "
+                      f"through the CPU oracle (plain C, fp64, 1 thread) in {t:.1f} s"}
+
+
+def run_rswa_workload(args, rank, world, local_rank):
+    """One R-SWA decode attention step (focr_rswa_decode) for T sequences; same JSON contract."""
+    import torch
+    from weight_quantized_expert_b200 import api, synth
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.STEP_WORKLOADS[args.workload]
+    B, R, n = w["T"], w["R"], w["n_gen"]
+    per_copy = (R + 128) * 2 * 10 * 128 * 4 * B
+    ncopy = max(2, -(-160 * 2 ** 20 // per_copy))   # copies of the KV cache, together above L2
+    a = synth.rswa_inputs(w["seed"], B, R)
+    copies = []
+    for c in range(ncopy):
+        t = {k: torch.from_numpy(v).to(dev) for k, v in a.items()} if c == 0 else \
+            {k: v.clone() for k, v in copies[0].items()}
+        copies.append(t)
+    rl = torch.full((B,), R, dtype=torch.int32, device=dev)
+    ng = torch.full((B,), n, dtype=torch.int32, device=dev)
+    out = torch.empty(B, 10, 128, device=dev)
+    ws = torch.empty(api.focr_rswa_workspace_bytes(B, R), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def run(i, st, q=None):
+        c = copies[i % ncopy]
+        api.focr_rswa_decode(c["q"] if q is None else q, c["k_new"], c["v_new"], c["k_ref"], c["v_ref"], rl,
+                             c["k_ring"], c["v_ring"], ng, out=out, workspace=ws, stream=st)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            run(i, stream)
+    stream.synchronize()
+    K = args.steps
+    graphs, _ = capture_graphs(lambda i, st: run(i, st), K, stream)
+    ms, clk = timed_replay(graphs, stream, world, dev, local_rank)
+    ms_step = ms / K
+    value = job_rate(B, K, world, ms)
+    bytes_step = rswa_step_bytes(w)
+    peak, _, _, peak_kind = peaks()
+    achieved = bytes_step / (ms_step / 1e3) / 1e9
+    # end to end: the step's q in from pinned host memory, its output read back
+    hq = torch.from_numpy(a["q"]).pin_memory()
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq = torch.empty_like(copies[0]["q"])
+    K_e2e = min(K, 200)
+    with torch.cuda.stream(stream):
+        for i in range(5):
+            dq.copy_(hq, non_blocking=True)
+            run(i, stream, dq)
+            ho.copy_(out, non_blocking=True)
+        stream.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(K_e2e):
+            dq.copy_(hq, non_blocking=True)
+            run(i, stream, dq)
+            ho.copy_(out, non_blocking=True)
+        f1.record(stream)
+        stream.synchronize()
+    e2e = job_rate(B, K_e2e, world, max_over_ranks(f0.elapsed_time(f1), world, dev))
+    cpu = rswa_oracle_baseline(w) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+                "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32", "precision": "fp32 dot products and online softmax, split keys merged in fp32",
+                "data": "synthetic", "config": describe(args.workload, world),
+                "timing": {"graph": f"CUDA graph replay ({min(K, GRAPH_STEPS)} steps per graph, every graph "
+                                    "replayed once before the timed region)",
+                           "l2": f"steps rotate over {ncopy} copies of the KV cache ({ncopy * per_copy / 2**20:.0f} MB, "
+                                 "above L2)"},
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                             "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
+                             "peak_kind": peak_kind, "kernel": "one step (rswa_partial_kernel + rswa_combine_kernel)",
+                             "algorithmic_bytes_per_step": bytes_step},
+                "cpu_baseline": cpu,
+                "e2e": {"value": e2e, "unit": UNIT, "h2d_bytes_per_step": int(hq.numel() * 4),
+                        "d2h_bytes_per_step": int(ho.numel() * 4), "steps": K_e2e},
+                "gpu_launches": 2 * K, "clocks": clk}
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -706,7 +817,9 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
         from weight_quantized_expert_b200 import synth
-        if args.workload in synth.STEP_WORKLOADS:
+        if args.workload in synth.STEP_WORKLOADS and synth.STEP_WORKLOADS[args.workload]["kind"] == "rswa":
+            run_rswa_workload(args, rank, world, local_rank)
+        elif args.workload in synth.STEP_WORKLOADS:
             run_step_workload(args, rank, world, local_rank)
         else:
             run_ours(args, rank, world, local_rank)

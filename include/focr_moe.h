@@ -388,6 +388,47 @@ focr_status focr_w8a8_gemv(const focr_w8a8* m, const float* x, int32_t T, float*
  */
 focr_status focr_w8a8_check(void* workspace, void* stream);
 
+/* ------------------------------------------------------------------ R-SWA decode attention
+ * Source: franken_ocr README, "Design Philosophy" (bounded generated-token KV) and "Architecture"
+ * (R-SWA: each generated token attends to every reference token -- visual prefill plus prompt, a
+ * frozen block never evicted -- plus the previous 128 generated tokens through a ring buffer);
+ * frankenocr.pages.dev, "One forward pass", step 6 (10 heads of dimension 128, a 128-slot ring).
+ * Readings (the pages fix no formula): scores are scaled by 1/sqrt(128); q and k arrive with any
+ * position encoding applied; the window counts the current token, so it is the ring's 128 slots;
+ * generated token p lives in slot p mod 128.  For sequence b with R = ref_len[b] and n = n_gen[b]
+ * (generated tokens so far, the current one included):
+ *     keys: reference rows 0 .. R-1, generated tokens max(0, n-128) .. n-1 (the current one from
+ *     k_new / v_new);  out = sum_j softmax_j(q . k_j / sqrt(128)) v_j, per head;
+ *     afterwards slot (n-1) mod 128 of the ring holds k_new / v_new.
+ */
+#define FOCR_RSWA_HEADS 10
+#define FOCR_RSWA_DIM 128
+#define FOCR_RSWA_RING 128
+#define FOCR_RSWA_RCAP_MAX 32768   /* most reference rows per sequence */
+#define FOCR_RSWA_B_MAX 4096       /* most sequences per call */
+
+/* Workspace a focr_rswa_decode call with B sequences and capacity Rcap needs (bytes). */
+size_t focr_rswa_workspace_bytes(int32_t B, int32_t Rcap);
+
+/*
+ * focr_rswa_decode -- one decode step of one R-SWA attention layer for B sequences.
+ *   q, k_new, v_new, out: DEVICE fp32 [B][10][128].
+ *   k_ref, v_ref: DEVICE fp32 [B][10][Rcap][128] (row r of sequence b, head h at ((b*10+h)*Rcap+r)*128);
+ *     read only.  1 <= Rcap <= FOCR_RSWA_RCAP_MAX.
+ *   k_ring, v_ring: DEVICE fp32 [B][10][128][128], read, and slot (n_gen[b]-1) mod 128 written.
+ *   ref_len, n_gen: DEVICE int32 [B].  A sequence with ref_len outside [0, Rcap] or n_gen < 1 gets
+ *     NaN outputs and keeps its ring.
+ *   workspace: DEVICE, 256-byte aligned, >= focr_rswa_workspace_bytes(B, Rcap) bytes (no zero fill
+ *     needed).  Every float pointer 16-byte aligned; inputs finite.  1 <= B <= FOCR_RSWA_B_MAX.
+ *   Two launches on `stream` (programmatic dependent launch between them); asynchronous.
+ * Errors: FOCR_ERR_INVALID_ARG (NULL, misaligned, sizes out of range, short workspace);
+ * FOCR_ERR_CUDA (a launch failed).
+ */
+focr_status focr_rswa_decode(const float* q, const float* k_new, const float* v_new, const float* k_ref,
+                             const float* v_ref, const int32_t* ref_len, int32_t Rcap, float* k_ring, float* v_ring,
+                             const int32_t* n_gen, int32_t B, float* out, void* workspace, size_t ws_bytes,
+                             void* stream);
+
 /*
  * focr_tc_selftest -- diagnostic: one tensor-core tile through the library's tcgen05 primitives
  * (the ones the T > 8 grouped kernel uses), to check them against a host GEMM.

@@ -105,3 +105,14 @@ def test_w8a8_rejects_bad_arguments_without_launching():
     for T, K in ((0, 16), (api.T_MAX + 1, 16), (1, 0),
                  (1, api.W8A8_K_MAX + 1)):
         assert L.focr_w8a8_quantize_x(p, T, K, qp, p, None) == 1
+
+
+def test_rswa_workspace_and_argument_checks_without_launching():
+    L = api.lib()
+    assert api.focr_rswa_workspace_bytes(1, 289) % 256 == 0
+    assert api.focr_rswa_workspace_bytes(8, 289) >= api.focr_rswa_workspace_bytes(1, 289)
+    buf = (ctypes.c_float * 64)()
+    p = ctypes.cast(buf, ctypes.c_void_p).value
+    assert L.focr_rswa_decode(None, p, p, p, p, p, 1, p, p, p, 1, p, p, 1 << 20, None) == 1
+    assert L.focr_rswa_decode(p, p, p, p, p, p, 0, p, p, p, 1, p, p, 1 << 20, None) == 1
+    assert L.focr_rswa_decode(p, p, p, p, p, p, 1, p, p, p, 5000, p, p, 1 << 20, None) == 1

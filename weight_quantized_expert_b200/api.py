@@ -35,7 +35,7 @@ EXPORTED = (
     "focr_dense_mlp_free", "focr_dense_mlp_export_quantized", "focr_dense_mlp_forward", "focr_tc_selftest",
     "focr_decode_step_workspace_bytes", "focr_decode_step", "focr_w8a8_pack", "focr_w8a8_free",
     "focr_w8a8_export", "focr_w8a8_quantize_x", "focr_w8a8_workspace_bytes", "focr_w8a8_gemv", "focr_w8a8_check",
-    "focr_lm_head_check",
+    "focr_lm_head_check", "focr_rswa_workspace_bytes", "focr_rswa_decode",
 )
 FWD_RESIDUAL = 1
 FWD_DETERMINISTIC = 2
@@ -113,6 +113,8 @@ def lib():
                 "focr_w8a8_gemv": (i32, [P, P, i32, P, P, sz, P]),
                 "focr_w8a8_check": (i32, [P, P]),
                 "focr_lm_head_check": (i32, [P, P]),
+                "focr_rswa_workspace_bytes": (sz, [i32, i32]),
+                "focr_rswa_decode": (i32, [P, P, P, P, P, P, i32, P, P, P, i32, P, P, sz, P]),
                 "focr_last_error": (ctypes.c_char_p, []),
                 "focr_version": (ctypes.c_char_p, []),
             }
@@ -375,6 +377,35 @@ def focr_lm_head_check(workspace, stream=None):
 
 def focr_w8a8_check(workspace, stream=None):
     _check(lib().focr_w8a8_check(_ptr(workspace), _stream(stream)))
+
+
+# ---------------------------------------------------------------- R-SWA decode attention
+
+RSWA_HEADS, RSWA_DIM, RSWA_RING = 10, 128, 128
+
+
+def focr_rswa_workspace_bytes(B: int, Rcap: int) -> int:
+    return int(lib().focr_rswa_workspace_bytes(int(B), int(Rcap)))
+
+
+def focr_rswa_decode(q, k_new, v_new, k_ref, v_ref, ref_len, k_ring, v_ring, n_gen, out=None, workspace=None,
+                     stream=None):
+    """out [B, 10, 128]: one R-SWA decode step; k_ring / v_ring [B, 10, 128, 128] get the current token."""
+    import torch
+    B, H, D = q.shape
+    Rcap = k_ref.shape[2]
+    for t in (q, k_new, v_new, k_ref, v_ref, k_ring, v_ring):
+        assert t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()
+    assert (H, D) == (RSWA_HEADS, RSWA_DIM) and k_ring.shape == (B, H, RSWA_RING, D) and v_ref.shape == k_ref.shape
+    assert ref_len.dtype == torch.int32 and n_gen.dtype == torch.int32 and ref_len.is_cuda and n_gen.is_cuda
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.empty(focr_rswa_workspace_bytes(B, Rcap), dtype=torch.uint8, device=q.device)
+    _check(lib().focr_rswa_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_ref), _ptr(v_ref), _ptr(ref_len), Rcap,
+                                  _ptr(k_ring), _ptr(v_ring), _ptr(n_gen), B, _ptr(out), _ptr(workspace),
+                                  workspace.numel(), _stream(stream)))
+    return out
 
 
 def focr_rmsnorm(x, gamma=None, eps: float = 1e-6, out=None, stream=None):

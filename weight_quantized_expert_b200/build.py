@@ -11,7 +11,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libfocr_moe.so")
-SOURCES = ["api.cu", "router.cu", "expert_tc.cu", "tcgen05_selftest.cu", "expert_decode.cu", "decode_small.cu", "noalloc.cu", "lm_head.cu", "rmsnorm.cu", "w8a8.cu", "pack.cpp"]
+SOURCES = ["api.cu", "router.cu", "expert_tc.cu", "tcgen05_selftest.cu", "expert_decode.cu", "decode_small.cu", "noalloc.cu", "lm_head.cu", "rmsnorm.cu", "w8a8.cu", "rswa.cu", "pack.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

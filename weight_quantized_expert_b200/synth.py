@@ -173,6 +173,19 @@ def lm_head(seed: int, vocab: int = VOCAB) -> np.ndarray:
     return weights_f32(seed, 3001, (vocab, H))
 
 
+RSWA_HEADS, RSWA_DIM, RSWA_RING = 10, 128, 128
+RSWA_REF = 289   # reference block of the prefill workload: 273 visual rows + 16 prompt rows
+
+
+def rswa_inputs(seed: int, B: int, Rcap: int) -> dict:
+    """One R-SWA decode step's tensors for B sequences, all ~N(0, 1) (so q . k / sqrt(128) ~ N(0, 1)):
+    q, k_new, v_new [B, 10, 128]; k_ref, v_ref [B, 10, Rcap, 128]; k_ring, v_ring [B, 10, 128, 128]."""
+    sh, sr, sg = (B, RSWA_HEADS, RSWA_DIM), (B, RSWA_HEADS, Rcap, RSWA_DIM), (B, RSWA_HEADS, RSWA_RING, RSWA_DIM)
+    return dict(q=normal_f32(seed, 4001, sh), k_new=normal_f32(seed, 4002, sh), v_new=normal_f32(seed, 4003, sh),
+                k_ref=normal_f32(seed, 4004, sr), v_ref=normal_f32(seed, 4005, sr),
+                k_ring=normal_f32(seed, 4006, sg), v_ring=normal_f32(seed, 4007, sg))
+
+
 # ---------------------------------------------------------------- workloads
 # The five measured workloads of the method (one MoE layer at hidden 1280).
 WORKLOADS = {
@@ -197,6 +210,9 @@ STEP_WORKLOADS = {
     # W8A8 GEMV on the lm_head's shape (129280 x 1280 int8, one scale per row; 165 MB > L2)
     "w8a8_lm_head_t1": dict(kind="w8a8", seed=4, T=1),
     "w8a8_lm_head_t8": dict(kind="w8a8", seed=4, T=8),
+    # R-SWA decode attention: T sequences, a 289-row reference block, 600 tokens generated (ring wrapped)
+    "rswa_t1": dict(kind="rswa", seed=5, T=1, R=289, n_gen=600),
+    "rswa_b8": dict(kind="rswa", seed=5, T=8, R=289, n_gen=600),
 }
 
 
