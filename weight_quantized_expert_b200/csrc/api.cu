@@ -9,7 +9,6 @@
 #include "common.cuh"
 #include "lm_head.h"
 #include "pack.h"
-#include "rswa.h"
 #include "w8a8.h"
 
 using namespace focr;
@@ -572,38 +571,6 @@ focr_status focr_w8a8_check(void* workspace, void* stream) {
     CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(word), st));
     CUDA_TRY(cudaStreamSynchronize(st));
     return fail(FOCR_ERR_TIMEOUT, "a bounded wait of the W8A8 GEMV ran out; the outputs of that call are not valid");
-}
-
-// ------------------------------------------------------------------ R-SWA decode attention
-
-size_t focr_rswa_workspace_bytes(int32_t B, int32_t Rcap) {
-    if (B < 1) B = 1;
-    if (B > FOCR_RSWA_B_MAX) B = FOCR_RSWA_B_MAX;
-    if (Rcap < 1) Rcap = 1;
-    if (Rcap > FOCR_RSWA_RCAP_MAX) Rcap = FOCR_RSWA_RCAP_MAX;
-    return align_up(rswa_part_bytes(B, Rcap), 256);
-}
-
-focr_status focr_rswa_decode(const float* q, const float* k_new, const float* v_new, const float* k_ref,
-                             const float* v_ref, const int32_t* ref_len, int32_t Rcap, float* k_ring, float* v_ring,
-                             const int32_t* n_gen, int32_t B, float* out, void* workspace, size_t ws_bytes,
-                             void* stream) {
-    g_err.clear();
-    if (!q || !k_new || !v_new || !k_ref || !v_ref || !ref_len || !k_ring || !v_ring || !n_gen || !out || !workspace)
-        return fail(FOCR_ERR_INVALID_ARG, "NULL argument");
-    if (B < 1 || B > FOCR_RSWA_B_MAX) return fail(FOCR_ERR_INVALID_ARG, "B=%d outside [1, %d]", B, FOCR_RSWA_B_MAX);
-    if (Rcap < 1 || Rcap > FOCR_RSWA_RCAP_MAX)
-        return fail(FOCR_ERR_INVALID_ARG, "Rcap=%d outside [1, %d]", Rcap, FOCR_RSWA_RCAP_MAX);
-    const void* f[] = {q, k_new, v_new, k_ref, v_ref, k_ring, v_ring, out};
-    for (const void* ptr : f)
-        if (!aligned(ptr, 16)) return fail(FOCR_ERR_INVALID_ARG, "float buffers must be 16-byte aligned");
-    if (!aligned(ref_len, 4) || !aligned(n_gen, 4) || !aligned(workspace, 256))
-        return fail(FOCR_ERR_INVALID_ARG, "misaligned lengths or workspace");
-    const size_t need = focr_rswa_workspace_bytes(B, Rcap);
-    if (ws_bytes < need) return fail(FOCR_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, need);
-    CUDA_TRY(launch_rswa(q, k_new, v_new, k_ref, v_ref, ref_len, Rcap, k_ring, v_ring, n_gen, B, out,
-                         reinterpret_cast<float*>(workspace), (cudaStream_t)stream));
-    return FOCR_OK;
 }
 
 focr_status focr_lm_head_check(void* workspace, void* stream) {

@@ -26,6 +26,7 @@
 // A sequence whose ref_len lies outside [0, Rcap] or whose n_gen < 1 gets NaN outputs and keeps its
 // ring.
 #include <math.h>
+#include <stdio.h>
 
 #include <algorithm>
 
@@ -260,3 +261,56 @@ cudaError_t launch_rswa(const float* q, const float* k_new, const float* v_new, 
 }
 
 }  // namespace focr
+
+// ------------------------------------------------------------------ C ABI
+namespace focr {
+focr_status report_error(focr_status s, const char* msg);   // the library's focr_last_error() record
+}  // namespace focr
+
+extern "C" {
+
+size_t focr_rswa_workspace_bytes(int32_t B, int32_t Rcap) {
+    if (B < 1) B = 1;
+    if (B > FOCR_RSWA_B_MAX) B = FOCR_RSWA_B_MAX;
+    if (Rcap < 1) Rcap = 1;
+    if (Rcap > FOCR_RSWA_RCAP_MAX) Rcap = FOCR_RSWA_RCAP_MAX;
+    return (focr::rswa_part_bytes(B, Rcap) + 255) & ~(size_t)255;
+}
+
+focr_status focr_rswa_decode(const float* q, const float* k_new, const float* v_new, const float* k_ref,
+                             const float* v_ref, const int32_t* ref_len, int32_t Rcap, float* k_ring, float* v_ring,
+                             const int32_t* n_gen, int32_t B, float* out, void* workspace, size_t ws_bytes,
+                             void* stream) {
+    using focr::report_error;
+    report_error(FOCR_OK, "");
+    char msg[160];
+    if (!q || !k_new || !v_new || !k_ref || !v_ref || !ref_len || !k_ring || !v_ring || !n_gen || !out || !workspace)
+        return report_error(FOCR_ERR_INVALID_ARG, "NULL argument");
+    if (B < 1 || B > FOCR_RSWA_B_MAX) {
+        snprintf(msg, sizeof(msg), "B=%d outside [1, %d]", B, FOCR_RSWA_B_MAX);
+        return report_error(FOCR_ERR_INVALID_ARG, msg);
+    }
+    if (Rcap < 1 || Rcap > FOCR_RSWA_RCAP_MAX) {
+        snprintf(msg, sizeof(msg), "Rcap=%d outside [1, %d]", Rcap, FOCR_RSWA_RCAP_MAX);
+        return report_error(FOCR_ERR_INVALID_ARG, msg);
+    }
+    const void* f[] = {q, k_new, v_new, k_ref, v_ref, k_ring, v_ring, out};
+    for (const void* ptr : f)
+        if ((uintptr_t)ptr % 16) return report_error(FOCR_ERR_INVALID_ARG, "float buffers must be 16-byte aligned");
+    if ((uintptr_t)ref_len % 4 || (uintptr_t)n_gen % 4 || (uintptr_t)workspace % 256)
+        return report_error(FOCR_ERR_INVALID_ARG, "misaligned lengths or workspace");
+    const size_t need = focr_rswa_workspace_bytes(B, Rcap);
+    if (ws_bytes < need) {
+        snprintf(msg, sizeof(msg), "workspace of %zu bytes < %zu needed", ws_bytes, need);
+        return report_error(FOCR_ERR_INVALID_ARG, msg);
+    }
+    const cudaError_t e = focr::launch_rswa(q, k_new, v_new, k_ref, v_ref, ref_len, Rcap, k_ring, v_ring, n_gen, B,
+                                            out, reinterpret_cast<float*>(workspace), (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        snprintf(msg, sizeof(msg), "launch_rswa: %s (%s)", cudaGetErrorName(e), cudaGetErrorString(e));
+        return report_error(FOCR_ERR_CUDA, msg);
+    }
+    return FOCR_OK;
+}
+
+}  // extern "C"
