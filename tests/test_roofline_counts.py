@@ -55,3 +55,16 @@ def test_profile_identity_ignores_comments_only(tmp_path, monkeypatch):
     assert bench.sources_hash() == h0
     f.write_text(f.read_text().replace("1e-6", "2e-6") + "\nstatic int focr_extra_symbol = 1;\n")
     assert bench.sources_hash() != h0
+
+
+def test_w8a8_and_rswa_bench_bytes():
+    import bench
+    from weight_quantized_expert_b200 import synth
+    # W8A8 at the lm_head's shape, T = 1: 165,478,400 codes + 517,120 scale bytes + 5,120 B of x + 517,120 B of y
+    assert bench.step_bytes_companion(synth.STEP_WORKLOADS["w8a8_lm_head_t1"]) == 166_517_760
+    # R-SWA, one sequence, 289 reference rows + a full 128-slot window: 417 keys x (k + v) x 10 heads x 512 B,
+    # plus q, k_new, v_new, out and the two ring-slot rows (6 x 5,120 B)
+    assert bench.rswa_step_bytes(synth.STEP_WORKLOADS["rswa_t1"]) == 417 * 2 * 5_120 + 6 * 5_120 == 4_300_800
+    assert bench.rswa_step_bytes(synth.STEP_WORKLOADS["rswa_b8"]) == 8 * 4_300_800
+    # a window that has not filled yet counts only the generated tokens so far
+    assert bench.rswa_step_bytes(dict(T=1, R=10, n_gen=5)) == (10 + 5) * 2 * 5_120 + 6 * 5_120
