@@ -22,9 +22,10 @@
 //                         up to 20 KB) into a ring of shared-memory stages (up to 8, 160 KB in
 //                         flight per SM).  Up to eight consumer warps take the units in turn, each
 //                         owning the same stages throughout (no phase aliasing): a 16-byte
-//                         A fragment per lane per k-step from shared memory, the B fragments from
-//                         L1, integer tensor-core MMAs (mma.sync m16n8k32 s8 with s32 accumulate:
-//                         exact integer arithmetic).  When a tile's K is split over several units,
+//                         A fragment per lane per k-step from shared memory, the B fragments (the
+//                         activation codes) staged once per CTA in shared memory (read through L1
+//                         when they do not fit beside 3 stages), integer tensor-core MMAs
+//                         (mma.sync m16n8k32 s8 with s32 accumulate: exact integer arithmetic).  When a tile's K is split over several units,
 //                         their partial sums meet by integer atomics (exact, so the order does not
 //                         matter) and the tile's last unit (a per-tile counter) applies the scales
 //                         and returns the sums and the counter to zero.  The producer starts before
